@@ -1,0 +1,273 @@
+"""Pins for the float64 oracle (CPU only).
+
+Each check ties the oracle to something other than itself: closed forms of the
+softmax, invariances the definition implies, a 50-digit brute force written in
+the textbook exp(s)/sum(exp(s)) form (no max subtraction), torch's own CPU
+float64 scaled_dot_product_attention, and values printed on the pages.  The
+checks are chosen so that a dropped scale, a wrong sign, an off-by-one causal
+mask, a transposed operand or a missing normalisation each fails at least one.
+"""
+
+import json
+import math
+import os
+
+import mpmath
+import numpy as np
+import pytest
+import torch
+
+from oracle import (
+    allowed_keys,
+    attention,
+    attention_batched,
+    attention_rows,
+    attention_tiled_online,
+    online_softmax_step,
+    resolve_scale,
+)
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+RNG = np.random.default_rng(1234)
+
+
+def rnd(*shape, scale=1.0):
+    return RNG.standard_normal(shape) * scale
+
+
+# ---------------------------------------------------------------- brute force
+def brute(q, k, v, scale, causal):
+    """50-digit brute force: p_ij = exp(s_ij) / sum_j' exp(s_ij'), no max shift."""
+    mpmath.mp.dps = 50
+    nq, d = q.shape
+    nkv = k.shape[0]
+    o = np.empty((nq, v.shape[1]))
+    lse = np.empty(nq)
+    for i in range(nq):
+        js = range(nkv) if not causal else range(min(i + 1, nkv))
+        s = {j: mpmath.mpf(scale) * mpmath.fsum(mpmath.mpf(q[i, c]) * mpmath.mpf(k[j, c]) for c in range(d))
+             for j in js}
+        ex = {j: mpmath.exp(s[j]) for j in js}
+        z = mpmath.fsum(ex.values())
+        for c in range(v.shape[1]):
+            o[i, c] = float(mpmath.fsum(ex[j] * mpmath.mpf(v[j, c]) for j in js) / z)
+        lse[i] = float(mpmath.log(z))
+    return o, lse
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("nq,nkv,d", [(1, 1, 1), (3, 5, 2), (5, 3, 4), (8, 8, 8), (7, 2, 3)])
+def test_brute_force_tiny(nq, nkv, d, causal):
+    q, k, v = rnd(nq, d), rnd(nkv, d), rnd(nkv, d)
+    sc = 0.7
+    o, lse = attention(q, k, v, scale=sc, causal=causal)
+    ob, lb = brute(q, k, v, sc, causal)
+    assert np.max(np.abs(o - ob)) <= 1e-13
+    assert np.max(np.abs(lse - lb)) <= 1e-13
+
+
+@pytest.mark.parametrize("kind", ["all_ones", "large_random", "alternating_extremes"])
+def test_page1_regression_inputs_vs_brute(kind):
+    """Page 1 section 数值安全的边界条件 lists three regression input families:
+    all-ones, large random values and alternating extremes."""
+    nq, nkv, d = 6, 7, 4
+    if kind == "all_ones":
+        q, k, v = np.ones((nq, d)), np.ones((nkv, d)), rnd(nkv, d)
+    elif kind == "large_random":
+        q, k, v = rnd(nq, d, scale=30), rnd(nkv, d, scale=30), rnd(nkv, d)
+    else:
+        sign = np.where(np.arange(nkv) % 2 == 0, 1.0, -1.0)[:, None]
+        q = np.where(np.arange(nq)[:, None] % 2 == 0, 60.0, -60.0) * np.ones((nq, d))
+        k = sign * 60.0 * np.ones((nkv, d))
+        v = rnd(nkv, d)
+    for causal in (False, True):
+        o, lse = attention(q, k, v, scale=0.125, causal=causal)
+        ob, lb = brute(q, k, v, 0.125, causal)
+        assert np.all(np.isfinite(o)) and np.all(np.isfinite(lse))
+        assert np.max(np.abs(o - ob)) <= 1e-12
+        assert np.max(np.abs(lse - lb)) <= 1e-12 * max(1.0, np.max(np.abs(lb)))
+    if kind == "all_ones":  # uniform weights: O is the plain mean of V
+        o, _ = attention(q, k, v, scale=0.125)
+        assert np.allclose(o, v.mean(axis=0)[None, :], atol=1e-14)
+
+
+def test_worked_example_closed_form():
+    """q = (1, 0), keys e1, e2, scale 1: weights e/(e+1) and 1/(e+1)."""
+    q = np.array([[1.0, 0.0]])
+    k = np.array([[1.0, 0.0], [0.0, 1.0]])
+    v = np.array([[1.0, 2.0], [3.0, 4.0]])
+    o, lse = attention(q, k, v, scale=1.0)
+    e = math.e
+    assert np.allclose(o[0], [(e + 3) / (e + 1), (2 * e + 4) / (e + 1)], atol=1e-15)
+    assert abs(lse[0] - math.log(e + 1)) < 1e-15
+
+
+# ---------------------------------------------------------------- closed forms
+@pytest.mark.parametrize("causal", [False, True])
+def test_zero_query_gives_mean_of_visible_values(causal):
+    nq, nkv, d = 37, 29, 16
+    q, k, v = np.zeros((nq, d)), rnd(nkv, d), rnd(nkv, d)
+    o, lse = attention(q, k, v, causal=causal)
+    for i in range(nq):
+        a = allowed_keys(i, nkv, causal)
+        assert np.allclose(o[i], v[a].mean(axis=0), atol=1e-13)
+        assert abs(lse[i] - math.log(len(a))) < 1e-13
+
+
+def test_allowed_keys_is_top_left_triu():
+    """Page 3 section 6.1: mask = triu(ones(Nq, Nkv), diagonal=1)."""
+    for nq, nkv in [(5, 5), (3, 7), (7, 3)]:
+        mask = torch.triu(torch.ones(nq, nkv), diagonal=1).bool().numpy()
+        for i in range(nq):
+            vis = np.zeros(nkv, bool)
+            vis[allowed_keys(i, nkv, True)] = True
+            assert np.array_equal(vis, ~mask[i])
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_constant_value_rows_pass_through(causal):
+    nq, nkv, d = 20, 33, 8
+    c = rnd(d)
+    q, k = rnd(nq, d, scale=3), rnd(nkv, d, scale=3)
+    v = np.tile(c, (nkv, 1))
+    o, _ = attention(q, k, v, causal=causal)
+    assert np.allclose(o, c[None, :], atol=1e-13)
+
+
+def test_causal_row0_and_single_key():
+    nq, nkv, d = 9, 9, 5
+    q, k, v = rnd(nq, d), rnd(nkv, d), rnd(nkv, d)
+    sc = 0.31
+    o, lse = attention(q, k, v, scale=sc, causal=True)
+    assert np.allclose(o[0], v[0], atol=1e-15)
+    assert abs(lse[0] - sc * q[0] @ k[0]) < 1e-14
+    o1, lse1 = attention(q, k[:1], v[:1], scale=sc)
+    assert np.allclose(o1, np.tile(v[0], (nq, 1)), atol=1e-15)
+    assert np.allclose(lse1, sc * q @ k[0], atol=1e-14)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_key_shift_invariance(causal):
+    nq, nkv, d = 15, 21, 6
+    q, k, v = rnd(nq, d), rnd(nkv, d), rnd(nkv, d)
+    c = rnd(d, scale=2)
+    sc = 0.4
+    o, lse = attention(q, k, v, scale=sc, causal=causal)
+    o2, lse2 = attention(q, k + c[None, :], v, scale=sc, causal=causal)
+    assert np.allclose(o, o2, atol=1e-12)
+    assert np.allclose(lse2, lse + sc * (q @ c), atol=1e-12)
+
+
+def test_permutation_invariance_noncausal():
+    nq, nkv, d = 11, 17, 4
+    q, k, v = rnd(nq, d), rnd(nkv, d), rnd(nkv, d)
+    perm = RNG.permutation(nkv)
+    o, lse = attention(q, k, v)
+    o2, lse2 = attention(q, k[perm], v[perm])
+    assert np.allclose(o, o2, atol=1e-13) and np.allclose(lse, lse2, atol=1e-13)
+
+
+def test_scale_resolution():
+    """Page 3 Config: softmax_scale = -1 means 1/sqrt(d)."""
+    assert resolve_scale(None, 64) == 0.125
+    assert resolve_scale(-1.0, 64) == 0.125
+    assert resolve_scale(0.0, 16) == 0.25
+    assert resolve_scale(float("nan"), 4) == 0.5
+    assert resolve_scale(0.3, 4) == 0.3
+
+
+# ---------------------------------------------------------------- tiled twin
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("br,bc", [(1, 1), (3, 16), (16, 3), (64, 128), (128, 64), (128, 128)])
+def test_tiled_online_equals_naive(br, bc, causal):
+    """Page 1 section 分块 Tiling 的计算骨架: the tiled result equals the global
+    softmax exactly (up to rounding)."""
+    nq, nkv, d = 150, 173, 8
+    q, k, v = rnd(nq, d, scale=2), rnd(nkv, d, scale=2), rnd(nkv, d)
+    o, lse = attention(q, k, v, causal=causal)
+    o2, lse2 = attention_tiled_online(q, k, v, br, bc, causal=causal)
+    assert np.max(np.abs(o - o2)) <= 1e-12
+    assert np.max(np.abs(lse - lse2)) <= 1e-12
+
+
+def test_online_step_matches_direct_sums():
+    """Page 1 section 在线 Softmax: merging block statistics equals the direct sum."""
+    x = rnd(300, scale=4)
+    m, l = -math.inf, 0.0
+    for c0 in range(0, 300, 37):
+        m, l = online_softmax_step(m, l, x[c0:c0 + 37])
+    assert abs(m - x.max()) == 0
+    assert abs(l - np.exp(x - x.max()).sum()) <= 1e-12 * l
+
+
+def test_golden_rescale_underflow():
+    """Page 1 numerical-safety figure: a max jump of 100 rescales the previous
+    sum by exp(-100) ~ 3.7e-44 (below float32's smallest normal ~1.2e-38); in
+    float64 the merge is still exact."""
+    g = json.load(open(os.path.join(GOLDEN, "page1_numerical_safety.json")))
+    f = math.exp(-100.0)
+    assert abs(f - g["exp_minus_100"]) <= g["exp_minus_100_rel_tol"] * g["exp_minus_100"]
+    assert f < float(np.finfo(np.float32).tiny)
+    assert abs(float(np.finfo(np.float32).tiny) - g["float32_min_normal"]) <= \
+        g["float32_min_normal_rel_tol"] * g["float32_min_normal"]
+    x1 = np.array([0.0, -1.0, -2.0])
+    x2 = np.array([100.0, 99.0])
+    m, l = online_softmax_step(-math.inf, 0.0, x1)
+    m, l = online_softmax_step(m, l, x2)
+    direct = np.exp(np.concatenate([x1, x2]) - 100.0).sum()
+    assert m == 100.0 and abs(l - direct) <= 1e-15 * direct
+    # the same jump inside the tiled attention: one key dominates by 100
+    q = np.array([[1.0]])
+    k = np.array([[0.0], [100.0]])
+    v = np.array([[5.0], [7.0]])
+    o, lse = attention_tiled_online(q, k, v, 1, 1, scale=1.0)
+    assert abs(o[0, 0] - (5.0 * f + 7.0) / (1.0 + f)) <= 1e-15
+    assert abs(lse[0] - (100.0 + math.log1p(f))) <= 1e-13
+
+
+# ---------------------------------------------------------------- library cross-check
+@pytest.mark.parametrize("causal", [False, True])
+def test_torch_sdpa_float64_cross_check(causal):
+    B, H, N, d = 2, 3, 97, 16
+    q, k, v = rnd(B, H, N, d), rnd(B, H, N, d), rnd(B, H, N, d)
+    o, lse = attention_batched(q, k, v, causal=causal)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q), torch.from_numpy(k), torch.from_numpy(v), is_causal=causal).numpy()
+    assert np.max(np.abs(o - ref)) <= 1e-12
+
+
+def test_layouts_and_rows_agree():
+    B, H, nq, nkv, d = 2, 3, 19, 23, 8
+    q, k, v = rnd(B, H, nq, d), rnd(B, H, nkv, d), rnd(B, H, nkv, d)
+    for causal in (False, True):
+        o, lse = attention_batched(q, k, v, causal=causal, layout="BHND")
+        o2, lse2 = attention_batched(q.transpose(0, 2, 1, 3), k.transpose(0, 2, 1, 3),
+                                     v.transpose(0, 2, 1, 3), causal=causal, layout="BSND")
+        assert np.array_equal(o, o2.transpose(0, 2, 1, 3)) and np.array_equal(lse, lse2)
+        rows = [0, 5, 18]
+        orow, lrow = attention_rows(q[1, 2, rows], k[1, 2], v[1, 2], rows, causal=causal)
+        assert np.max(np.abs(orow - o[1, 2, rows])) <= 1e-13
+        assert np.max(np.abs(lrow - lse[1, 2, rows])) <= 1e-13
+
+
+def test_row_blocking_is_invisible():
+    """Query rows beyond one internal row block give the same rows as alone."""
+    import oracle.attention_ref as ar
+
+    nq, nkv, d = 40, 31, 4
+    q, k, v = rnd(nq, d), rnd(nkv, d), rnd(nkv, d)
+    old = ar.ROW_BLOCK
+    try:
+        ar.ROW_BLOCK = 7
+        o, lse = attention(q, k, v, causal=True)
+    finally:
+        ar.ROW_BLOCK = old
+    o2, lse2 = attention(q, k, v, causal=True)
+    assert np.max(np.abs(o - o2)) <= 1e-14 and np.max(np.abs(lse - lse2)) <= 1e-14
+
+
+def test_empty_and_invalid():
+    o, lse = attention(np.zeros((0, 4)), rnd(3, 4), rnd(3, 4))
+    assert o.shape == (0, 4) and lse.shape == (0,)
+    with pytest.raises(ValueError):
+        attention(rnd(2, 4), np.zeros((0, 4)), np.zeros((0, 4)))

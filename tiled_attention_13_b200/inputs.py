@@ -1,0 +1,136 @@
+"""Seeded synthetic inputs for the attention forward (shared by tests and bench).
+
+This module holds no attention arithmetic: it only draws Q, K and V.  It is the
+one module that both the CUDA-side tests and the CPU oracle checks read.
+
+Recipe (stated in the design doc as well):
+
+* Q, K, V are i.i.d. N(0, 1) drawn in float32 by ``torch.randn`` from three
+  independent generators seeded ``4*seed + 0/1/2`` (Q, K, V), then rounded to
+  the storage dtype (bf16, fp16 or fp32) with round-to-nearest-even.
+* Long-context K outliers: ``round(frac * N)`` sequence positions chosen by
+  ``torch.randperm`` on a CPU generator seeded ``4*seed + 3`` (the same
+  positions for every batch and head); ``+3.0`` is added to all d entries of K
+  at those positions before the rounding.
+* The named workloads are the shapes the surveyed pages benchmark (LLaMA-13B
+  self-attention, B=4/H=32/D=128 batched attention, a diffusion cross-attention
+  block, 128K long context).  No dataset, weights or benchmark items are used:
+  every tensor is random and only the shapes follow the pages.
+"""
+
+from __future__ import annotations
+
+from dataclasses import dataclass, replace
+
+import torch
+
+BASE_SEED = 20261202
+
+_DTYPES = {"bf16": torch.bfloat16, "fp16": torch.float16, "fp32": torch.float32}
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    H: int
+    Nq: int
+    Nkv: int
+    d: int
+    dtype: str = "bf16"
+    layout: str = "BHND"
+    causal: bool = False
+    seed: int = BASE_SEED
+    k_outlier: float = 0.0
+    outlier_frac: float = 0.0
+
+    @property
+    def flops(self) -> float:
+        """Algorithmic FLOPs: 4*B*H*Nq*Nkv*d, halved when causal."""
+        f = 4.0 * self.B * self.H * self.Nq * self.Nkv * self.d
+        return f / 2 if self.causal else f
+
+    @property
+    def bytes_min(self) -> int:
+        """Compulsory HBM bytes: read Q, K, V once, write O and the fp32 LSE."""
+        es = 4 if self.dtype == "fp32" else 2
+        return (es * self.B * self.H * self.d * (2 * self.Nq + 2 * self.Nkv)
+                + 4 * self.B * self.H * self.Nq)
+
+    def q_shape(self):
+        return (self.B, self.H, self.Nq, self.d) if self.layout == "BHND" else (self.B, self.Nq, self.H, self.d)
+
+    def kv_shape(self):
+        return (self.B, self.H, self.Nkv, self.d) if self.layout == "BHND" else (self.B, self.Nkv, self.H, self.d)
+
+    def with_(self, **kw) -> "Workload":
+        return replace(self, **kw)
+
+
+def _wl(name, idx, **kw):
+    return Workload(name=name, seed=BASE_SEED + idx, **kw)
+
+
+# The five workload families; idx fixes the seed (BASE_SEED + idx).
+WORKLOADS = {
+    "tiny": _wl("tiny", 0, B=1, H=2, Nq=256, Nkv=256, d=64, dtype="fp32", layout="BHND"),
+    "tiny-causal": _wl("tiny-causal", 0, B=1, H=2, Nq=256, Nkv=256, d=64, dtype="fp32", layout="BHND", causal=True),
+    "llama13b-2k": _wl("llama13b-2k", 1, B=1, H=40, Nq=2048, Nkv=2048, d=128, layout="BSND", causal=True),
+    "llama13b-4k": _wl("llama13b-4k", 1, B=1, H=40, Nq=4096, Nkv=4096, d=128, layout="BSND", causal=True),
+    "llama13b-8k": _wl("llama13b-8k", 1, B=1, H=40, Nq=8192, Nkv=8192, d=128, layout="BSND", causal=True),
+    "b4-2k": _wl("b4-2k", 2, B=4, H=32, Nq=2048, Nkv=2048, d=128),
+    "b4-2k-causal": _wl("b4-2k-causal", 2, B=4, H=32, Nq=2048, Nkv=2048, d=128, causal=True),
+    "b4-8k": _wl("b4-8k", 2, B=4, H=32, Nq=8192, Nkv=8192, d=128),
+    "b4-8k-causal": _wl("b4-8k-causal", 2, B=4, H=32, Nq=8192, Nkv=8192, d=128, causal=True),
+    "b4-32k": _wl("b4-32k", 2, B=4, H=32, Nq=32768, Nkv=32768, d=128),
+    "b4-32k-causal": _wl("b4-32k-causal", 2, B=4, H=32, Nq=32768, Nkv=32768, d=128, causal=True),
+    "cross": _wl("cross", 3, B=2, H=8, Nq=4096, Nkv=77, d=64),
+    "long": _wl("long", 4, B=1, H=32, Nq=131072, Nkv=131072, d=128, layout="BSND", causal=True,
+                k_outlier=3.0, outlier_frac=0.01),
+}
+
+
+def _gen(seed: int, device) -> torch.Generator:
+    g = torch.Generator(device=device)
+    g.manual_seed(seed)
+    return g
+
+
+def outlier_positions(wl: Workload) -> torch.Tensor:
+    """Sequence positions of K that receive +k_outlier (sorted, int64, CPU)."""
+    n = int(round(wl.outlier_frac * wl.Nkv))
+    if n == 0:
+        return torch.zeros((0,), dtype=torch.int64)
+    perm = torch.randperm(wl.Nkv, generator=_gen(4 * wl.seed + 3, "cpu"))
+    return torch.sort(perm[:n]).values
+
+
+def make_qkv(wl: Workload, device="cpu"):
+    """Draw (q, k, v) for ``wl`` on ``device`` in its layout and storage dtype."""
+    dev = torch.device(device)
+    dt = _DTYPES[wl.dtype]
+    gdev = "cuda" if dev.type == "cuda" else "cpu"
+    with torch.cuda.device(dev) if dev.type == "cuda" else _null():
+        q = torch.randn(wl.q_shape(), generator=_gen(4 * wl.seed + 0, gdev), device=dev, dtype=torch.float32)
+        q = q.to(dt)
+        k = torch.randn(wl.kv_shape(), generator=_gen(4 * wl.seed + 1, gdev), device=dev, dtype=torch.float32)
+        if wl.k_outlier != 0.0 and wl.outlier_frac > 0.0:
+            pos = outlier_positions(wl).to(dev)
+            axis = 2 if wl.layout == "BHND" else 1
+            k.index_add_(axis, pos, torch.full_like(k.index_select(axis, pos), wl.k_outlier))
+        k = k.to(dt)
+        v = torch.randn(wl.kv_shape(), generator=_gen(4 * wl.seed + 2, gdev), device=dev, dtype=torch.float32)
+        v = v.to(dt)
+    return q, k, v
+
+
+class _null:
+    def __enter__(self):
+        return self
+
+    def __exit__(self, *a):
+        return False
+
+
+def storage_dtype(name: str) -> torch.dtype:
+    return _DTYPES[name]

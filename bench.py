@@ -1,0 +1,358 @@
+"""Benchmark of the B200 fused attention forward.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one call of the whole hot path (fa_fwd: tile scheduling, TMA
+staging, both tcgen05 contractions, online softmax, epilogue) over one batch
+of synthetic input of the named workload (default: the LLaMA-13B-shaped
+self-attention B=1, H=40, N=8192, d=128, bf16, causal, BSND).  Inputs are
+resident in HBM when the timed region starts; two input sets alternate so
+that a step never starts with its own inputs in L2 (each set, 336 MB with O,
+is larger than the 126 MB L2 anyway).
+
+Prints ONE JSON line on rank 0.  With N > 1 (torchrun), every rank runs the
+same workload on its own GPU (independent replicas, weak scaling, no
+collective on the data path); the time is the max over ranks.
+
+``--impl reference`` times the float64 CPU oracle on the host cores instead
+(bounded row samples of the same workload), on rank 0 only.
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd TFLOP/s (and % of B200 dense BF16 peak) and ms/call at 1 GPU"
+UNIT = "TFLOP/s"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return d, "measured"
+    return FALLBACK_PEAKS, "fallback"
+
+
+def dist_env():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+# ------------------------------------------------------------------ clocks
+class ClockSampler:
+    FIELDS = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits", "-lms", "50",
+                 "-i", str(self.gpu), "-f", self.path], stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self, t0: float, t1: float):
+        rows = []
+        if self.path and os.path.exists(self.path):
+            for line in open(self.path):
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) < 10:
+                    continue
+                try:
+                    ts = time.mktime(time.strptime(parts[0].split(".")[0], "%Y/%m/%d %H:%M:%S"))
+                    ts += float("0." + parts[0].split(".")[1]) if "." in parts[0] else 0.0
+                    rows.append((ts, float(parts[2]), float(parts[3]), parts[5:]))
+                except (ValueError, IndexError):
+                    continue
+            os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"], "samples": 0}
+        inside = [r for r in rows if t0 - 0.05 <= r[0] <= t1 + 0.05]
+        use = inside if inside else rows
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in use:
+            for n, v in zip(names, r[3][1:5]):
+                if v.strip().lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(r[1] for r in use), "sm_max_mhz": max(r[2] for r in use),
+                "reasons": sorted(reasons), "samples": len(use), "samples_in_timed_region": len(inside)}
+
+
+# ------------------------------------------------------------------ CPU oracle baseline
+def oracle_sample(wl, rows_budget_s: float = 12.0, seed: int = 0):
+    """Time the float64 oracle (as it stands) on a bounded sample of ``wl``:
+    whole query-row blocks of one head, until about ``rows_budget_s`` seconds of
+    CPU work.  Returns (tflops, sample description, threads)."""
+    import numpy as np
+    import torch
+    from threadpoolctl import threadpool_info
+
+    from oracle import attention
+    from tiled_attention_13_b200.inputs import make_qkv
+
+    one = wl.with_(B=1, H=1)
+    q, k, v = make_qkv(one, device="cpu")
+    if wl.layout == "BSND":
+        q, k, v = q[0, :, 0], k[0, :, 0], v[0, :, 0]
+    else:
+        q, k, v = q[0, 0], k[0, 0], v[0, 0]
+    qn, kn, vn = (t.to(torch.float64).numpy() for t in (q, k, v))
+    block = 512
+    flops = 0.0
+    t0 = time.perf_counter()
+    rows_done = 0
+    # row blocks taken evenly over the sequence so causal work is representative
+    starts = list(range(0, wl.Nq, block))
+    rng = np.random.default_rng(seed)
+    rng.shuffle(starts)
+    for r0 in starts:
+        r1 = min(wl.Nq, r0 + block)
+        attention(qn[r0:r1], kn, vn, causal=wl.causal, row_offset=r0)
+        if wl.causal:
+            flops += 4.0 * wl.d * sum(min(i + 1, wl.Nkv) for i in range(r0, r1))
+        else:
+            flops += 4.0 * wl.d * (r1 - r0) * wl.Nkv
+        rows_done += r1 - r0
+        if time.perf_counter() - t0 > rows_budget_s:
+            break
+    el = time.perf_counter() - t0
+    threads = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+    desc = f"{rows_done} query rows (blocks of {block}) of one head of {wl.name}, float64 numpy oracle"
+    return flops / el / 1e12, desc, threads, el
+
+
+# ------------------------------------------------------------------ main arms
+def run_reference(args, wl):
+    ws, rank, _ = dist_env()
+    if rank != 0:
+        return 0
+    import torch
+    from threadpoolctl import threadpool_info
+
+    torch.set_num_threads(len(os.sched_getaffinity(0)))
+    per_step = []
+    total_flops = 0.0
+    desc = ""
+    threads = 1
+    for i in range(args.warmup + args.steps):
+        tf, desc, threads, el = oracle_sample(wl, rows_budget_s=args.ref_step_s, seed=i)
+        if i >= args.warmup:
+            per_step.append(el)
+            total_flops += tf * el * 1e12
+    el = sum(per_step)
+    value = total_flops / el / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": 1e3 * el / max(1, len(per_step)), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": _config(wl, ws),
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": threads, "kind": "oracle",
+                         "sample": "each step: " + desc},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def _config(wl, ws):
+    return {"workload": wl.name, "B": wl.B, "H": wl.H, "Nq": wl.Nq, "Nkv": wl.Nkv, "d": wl.d,
+            "layout": wl.layout, "causal": wl.causal, "input_dtype": wl.dtype,
+            "parallelism": f"independent replicas x{ws} (no collective)",
+            "l2": "inputs larger than L2; two input sets alternate between steps",
+            "flops_per_step_per_gpu": wl.flops}
+
+
+def run_ours(args, wl):
+    import torch
+    import torch.distributed as dist
+
+    import tiled_attention_13_b200 as fa
+    from tiled_attention_13_b200.inputs import make_qkv
+
+    ws, rank, local = dist_env()
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if ws > 1:
+        import datetime
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+    fa.lib()
+    stream = torch.cuda.current_stream(dev)
+
+    sets = []
+    for s in range(2):
+        q, k, v = make_qkv(wl.with_(seed=wl.seed + 1000 * s * 0 + s), device=dev)
+        o = torch.empty_like(q)
+        lse = torch.empty((wl.B, wl.H, wl.Nq), dtype=torch.float32, device=dev)
+        sets.append((q, k, v, o, lse))
+    torch.cuda.synchronize()
+
+    def step(i):
+        q, k, v, o, lse = sets[i & 1]
+        fa.forward(q, k, v, causal=wl.causal, layout=wl.layout, out=o, lse=lse)
+
+    for i in range(args.warmup):
+        step(i)
+    torch.cuda.synchronize()
+    rc = fa.fa_get_device_status(stream.cuda_stream)
+    if rc != 0:
+        raise RuntimeError(f"device status after warm-up: {fa.fa_status_string(rc)}")
+
+    sampler = ClockSampler(int(os.environ.get("CUDA_VISIBLE_DEVICES", str(local)).split(",")[local])
+                           if "CUDA_VISIBLE_DEVICES" in os.environ else local)
+    if rank == 0:
+        sampler.start()
+        time.sleep(0.3)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    t0 = time.time()
+    start.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        step(i)
+        ev[i][1].record(stream)
+    end.record(stream)
+    torch.cuda.synchronize()
+    t1 = time.time()
+    if ws > 1:
+        dist.barrier()
+    total_ms = start.elapsed_time(end)
+    kern_ms = [a.elapsed_time(b) for a, b in ev]
+    if rank == 0:
+        time.sleep(0.1)
+        sampler.stop()
+    rc = fa.fa_get_device_status(stream.cuda_stream)
+    if rc != 0:
+        raise RuntimeError(f"device status after timing: {fa.fa_status_string(rc)}")
+
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if ws > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    ms_step = t.item() / args.steps
+    value = ws * wl.flops / (ms_step * 1e-3) / 1e12
+
+    # ---- end-to-end through the public API: pinned host in, host out
+    e2e = None
+    if not args.no_e2e:
+        qh, kh, vh = (x.cpu().pin_memory() for x in sets[0][:3])
+        hf = fa.HostForward(qh, kh, vh, causal=wl.causal, layout=wl.layout, device=dev)
+        for _ in range(2):
+            hf(qh, kh, vh)
+        torch.cuda.synchronize()
+        n_e2e = max(3, min(args.steps, 20))
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if ws > 1:
+            dist.barrier()
+        a.record(stream)
+        for _ in range(n_e2e):
+            hf(qh, kh, vh)
+        b.record(stream)
+        torch.cuda.synchronize()
+        te = torch.tensor([a.elapsed_time(b) / n_e2e], dtype=torch.float64, device=dev)
+        if ws > 1:
+            dist.all_reduce(te, op=dist.ReduceOp.MAX)
+        e2e = {"value": ws * wl.flops / (te.item() * 1e-3) / 1e12, "unit": UNIT,
+               "h2d_bytes_per_step": hf.h2d_bytes, "d2h_bytes_per_step": hf.d2h_bytes,
+               "ms_per_step": te.item(), "steps": n_e2e}
+        del hf, qh, kh, vh
+
+    if rank == 0:
+        peaks, src = load_peaks()
+        kmean = sum(kern_ms) / len(kern_ms)
+        achieved = wl.flops / (kmean * 1e-3) / 1e12
+        bound = "tensor" if wl.Nkv >= 512 else "hbm"
+        if bound == "tensor":
+            peak = float(peaks["bf16_tflops"])
+            roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "traffic": args.traffic,
+                    "peak_source": f"{src} bf16_tflops (burst; sustained {peaks.get('bf16_tflops_sustained')})",
+                    "kernel_ms_mean": kmean, "kernel_ms_min": min(kern_ms)}
+        else:
+            gbs = wl.bytes_min / (kmean * 1e-3) / 1e9
+            peak = float(peaks["hbm_gbs"])
+            roof = {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
+                    "traffic": args.traffic, "peak_source": f"{src} hbm_gbs", "kernel_ms_mean": kmean,
+                    "kernel_ms_min": min(kern_ms), "algorithmic_bytes": wl.bytes_min}
+        cpu = None
+        if not args.no_cpu_baseline and ws == 1:
+            tf, desc, threads, el = oracle_sample(wl, rows_budget_s=args.cpu_budget_s)
+            cpu = {"value": tf, "unit": UNIT, "cores": threads, "kind": "oracle",
+                   "sample": desc + f" ({el:.1f} s)"}
+        clocks = sampler.summary(t0, t1)
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16" if wl.dtype == "bf16" else wl.dtype,
+            "data": "synthetic: seeded i.i.d. N(0,1) Q/K/V of the workload's shape",
+            "config": _config(wl, ws), "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
+            "gpu_launches": args.steps, "clocks": clocks,
+            "pct_of_measured_bf16_peak": 100.0 * (value / ws) / float(peaks["bf16_tflops"]),
+        }
+        print(json.dumps(line), flush=True)
+    if ws > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="llama13b-8k")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget-s", type=float, default=12.0)
+    ap.add_argument("--ref-step-s", type=float, default=2.0)
+    ap.add_argument("--traffic", type=float, default=None,
+                    help="DRAM bytes per launch from an ncu capture of the same kernel (else null)")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    from tiled_attention_13_b200.inputs import WORKLOADS
+
+    wl = WORKLOADS[args.workload]
+    if args.impl == "reference":
+        return run_reference(args, wl)
+    return run_ours(args, wl)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

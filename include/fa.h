@@ -1,0 +1,126 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) fused scaled-dot-product attention
+ * forward.
+ *
+ * The operation (page 1, "CANN ops-transformer FlashAttentionScore", section
+ * 平方级显存的精确来源, and page 2, "FlashAttention on Ascend via
+ * ops-transformer", section 标准 vs IO-Aware 实现):
+ *
+ *     S = scale * Q K^T        (masked entries -> -inf when causal)
+ *     P = softmax(S)           (row-wise)
+ *     O = P V
+ *     LSE[i] = log(sum_j exp(S[i, j]))   (natural log of the scaled scores)
+ *
+ * computed tile by tile with the online softmax (page 1, sections 分块 Tiling
+ * 的计算骨架 and 在线 Softmax 的数学原理拆解; page 3, "ops-nn efficient
+ * attention for AIGC", section 2.2), so that the Nq x Nkv score matrix never
+ * reaches device memory.  The argument list follows page 2's
+ * flash_attention_score (scale_value, input_layout in {BSND, ...},
+ * pre_tokens/next_tokens for causal) and page 3's Config (softmax_scale = -1
+ * meaning 1/sqrt(d), causal flag).
+ *
+ * All entry points are plain C: pointers, sizes, ints.  No function throws,
+ * traps or aborts; every failure is a return code.
+ */
+#ifndef FA_B200_H
+#define FA_B200_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Memory layouts of q, k, v and o (page 2: input_layout; page 3: [B, H, N, D]).
+ *   FA_LAYOUT_BHND: element (b, h, n, c) at ((b*H + h)*N + n)*d + c
+ *   FA_LAYOUT_BSND: element (b, n, h, c) at ((b*N + n)*H + h)*d + c
+ * with N = Nq for q and o, N = Nkv for k and v.  Tensors are dense. */
+typedef enum { FA_LAYOUT_BHND = 0, FA_LAYOUT_BSND = 1 } fa_layout_t;
+
+/* Storage type of q, k, v and o.  BF16 and FP16 run on the tcgen05 tensor-core
+ * kernel (fp32 accumulation, P rounded to the input type before P V).  FP32
+ * runs on an exact-fp32 CUDA-core kernel.  LSE is always fp32. */
+typedef enum { FA_DTYPE_BF16 = 0, FA_DTYPE_FP16 = 1, FA_DTYPE_FP32 = 2 } fa_dtype_t;
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1,  /* null pointer, negative size, bad enum, Nkv == 0 with Nq > 0 */
+  FA_ERR_UNSUPPORTED = 2,  /* head dim not in {64, 128}, or a size beyond the index range */
+  FA_ERR_MISALIGNED = 3,   /* q, k, v, o not 16-byte aligned, or lse not 4-byte aligned */
+  FA_ERR_LAUNCH = 4,       /* the CUDA launch or tensor-map creation failed */
+  FA_ERR_TIMEOUT = 5,      /* a bounded device-side wait expired (see fa_get_device_status) */
+  FA_ERR_NO_DEVICE = 6     /* no usable sm_100 device for the current context */
+} fa_status_t;
+
+/*
+ * fa_fwd -- O = softmax(scale * Q K^T [+ causal mask]) V and LSE.
+ *
+ *   q      [B,H,Nq,d] or [B,Nq,H,d] (layout), device memory, read only
+ *   k, v   [B,H,Nkv,d] or [B,Nkv,H,d], device memory, read only
+ *   o      same shape, layout and dtype as q, device memory, written
+ *   lse    [B,H,Nq] fp32 device memory (head-major whatever the layout),
+ *          written; may be NULL, in which case no LSE is written
+ *   d      head dimension, 64 or 128
+ *   scale  softmax scale; scale <= 0 or NaN selects 1/sqrt(d)
+ *   causal 0 or 1.  Causal masking is top-left aligned: query row i sees key j
+ *          iff j <= i (page 3, section 6.1: triu(ones(Nq, Nkv), diagonal=1)
+ *          is masked).  Every row therefore sees key 0.
+ *   layout fa_layout_t, shared by q, k, v and o
+ *   dtype  fa_dtype_t, shared by q, k, v and o
+ *   stream a cudaStream_t (NULL = the legacy default stream)
+ *
+ * Ownership: every buffer belongs to the caller and must stay alive until the
+ * stream has finished the call.  The library keeps no pointer after return and
+ * allocates no device memory (its status word is a static device variable).
+ * The call is asynchronous: it validates, encodes TMA descriptors on the host
+ * and launches one kernel on `stream`.
+ *
+ * Returns FA_OK (also for B*H*Nq == 0, a no-op), or FA_ERR_INVALID_ARG /
+ * FA_ERR_UNSUPPORTED / FA_ERR_MISALIGNED before anything is launched, or
+ * FA_ERR_LAUNCH / FA_ERR_NO_DEVICE.  Device-side failures (a bounded wait that
+ * expired) are reported later by fa_get_device_status().
+ */
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+           int64_t B, int64_t H, int64_t Nq, int64_t Nkv, int64_t d,
+           float scale, int causal, int layout, int dtype, void* stream);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char* fa_status_string(int status);
+
+/*
+ * fa_get_device_status -- synchronise `stream`, then read and clear the
+ * current device's status word.  Returns FA_OK, FA_ERR_TIMEOUT if any kernel
+ * since the last read gave up on a bounded wait (its outputs are then
+ * undefined; the CUDA context stays usable), or FA_ERR_LAUNCH if the stream
+ * itself reported an error.
+ */
+int fa_get_device_status(void* stream);
+
+/*
+ * fa_set_wait_timeout_us -- upper bound, in microseconds, on any single
+ * device-side wait (mbarrier phase) inside the kernels launched afterwards
+ * from this process.  0 restores the default (2,000,000 us).  Returns the
+ * previous value.  Host-side setting; affects later launches only.
+ */
+uint32_t fa_set_wait_timeout_us(uint32_t us);
+
+/*
+ * fa_debug_set_fault -- test hook for failure detection, off by default.
+ *   0: none
+ *   1: the softmax warps of the tensor-core kernel never signal that P is
+ *      ready, so the MMA warp's bounded wait expires; every role then leaves
+ *      its loop, the CTA waits (bounded) for its own TMA copies and MMAs,
+ *      frees its tensor memory and exits, and the status word reads
+ *      FA_ERR_TIMEOUT.  No trap, no fault, no unbounded wait.
+ * Applies to launches made after the call.  Returns the previous mode.
+ */
+int fa_debug_set_fault(int mode);
+
+/* ABI version of this header, (major << 16) | minor. */
+int fa_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H */

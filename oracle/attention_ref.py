@@ -82,8 +82,11 @@ def _as_f64(x) -> np.ndarray:
     return np.asarray(x, dtype=np.float64)
 
 
-def attention(q, k, v, scale=None, causal: bool = False):
+def attention(q, k, v, scale=None, causal: bool = False, row_offset: int = 0):
     """Naive attention for one (batch, head): returns (O [Nq, d], LSE [Nq]).
+
+    ``row_offset`` is the sequence position of q's first row (it only moves the
+    causal mask), so a block of query rows can be evaluated on its own.
 
     Page 1 section 平方级显存的精确来源 and page 2 naive_attention:
       s_ij = scale * sum_c q_ic k_jc            (j in the allowed set A_i)
@@ -108,7 +111,7 @@ def attention(q, k, v, scale=None, causal: bool = False):
         r1 = min(nq, r0 + ROW_BLOCK)
         s = sc * (q[r0:r1] @ k.T)  # [r, Nkv]
         if causal:
-            rows = np.arange(r0, r1)[:, None]
+            rows = np.arange(r0, r1)[:, None] + row_offset
             cols = np.arange(nkv)[None, :]
             s = np.where(cols > rows, -np.inf, s)
         m = s.max(axis=1)

@@ -26,3 +26,12 @@ def pytest_collection_modifyitems(config, items):
     for it in items:
         if "gpu" in it.keywords:
             it.add_marker(skip)
+
+
+@pytest.fixture(scope="session")
+def fa_lib():
+    """The CUDA library, built in-tree if missing or stale (nvcc needs no GPU)."""
+    from tiled_attention_13_b200 import build, lib
+
+    build.build()
+    return lib()

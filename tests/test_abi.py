@@ -1,0 +1,88 @@
+"""C-ABI checks that need no GPU: the library loads, exports every entry point
+declared in include/fa.h, and rejects bad arguments before touching CUDA."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import tiled_attention_13_b200 as fa
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def declared_symbols():
+    text = open(os.path.join(ROOT, "include", "fa.h")).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:const\s+)?[a-z_0-9]+\s*\*?\s*(fa_[a-z_0-9]+)\s*\(", text, flags=re.M)))
+
+
+def test_header_declares_expected_entry_points():
+    assert declared_symbols() == sorted(fa.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(fa_lib):
+    out = subprocess.run(["nm", "-D", "--defined-only", fa.lib_path()], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\s[TW]\s+(\S+)$", out, flags=re.M))
+    for s in declared_symbols():
+        assert s in exported, s
+        assert getattr(fa_lib, s) is not None
+
+
+def test_status_strings_and_version(fa_lib):
+    for code in range(7):
+        assert fa.fa_status_string(code).startswith("FA_")
+    assert fa.fa_status_string(99) == "FA_ERR_UNKNOWN"
+    assert fa.fa_abi_version() == (1 << 16)
+
+
+def test_host_settings_roundtrip(fa_lib):
+    prev = fa.fa_set_wait_timeout_us(12345)
+    assert fa.fa_set_wait_timeout_us(0) == 12345
+    assert fa.fa_set_wait_timeout_us(prev) == 2000000
+    assert fa.fa_debug_set_fault(1) == 0
+    assert fa.fa_debug_set_fault(0) == 1
+
+
+A16 = 1 << 20  # a 16-byte aligned fake address (never dereferenced)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=-1), 1), (dict(H=-2), 1), (dict(Nq=-1), 1), (dict(Nkv=-5), 1), (dict(d=0), 1),
+    (dict(layout=2), 1), (dict(dtype=3), 1), (dict(causal=2), 1),
+    (dict(d=96), 2), (dict(d=256), 2),
+    (dict(Nkv=0), 1),
+    (dict(q=None), 1), (dict(o=None), 1),
+    (dict(q=A16 + 8), 3), (dict(v=A16 + 4), 3), (dict(lse=A16 + 2), 3),
+    (dict(Nq=0, q=None, k=None, v=None, o=None), 0), (dict(B=0), 0), (dict(H=0), 0),
+    (dict(B=1 << 31), 2), (dict(Nq=1 << 31), 2),
+])
+def test_validation_before_any_cuda_call(fa_lib, kw, code):
+    args = dict(q=A16, k=A16, v=A16, o=A16, lse=A16, B=1, H=2, Nq=10, Nkv=10, d=64, scale=-1.0, causal=0,
+                layout=0, dtype=0, stream=None)
+    args.update(kw)
+    rc = fa.fa_fwd(args["q"], args["k"], args["v"], args["o"], args["lse"], args["B"], args["H"], args["Nq"],
+                   args["Nkv"], args["d"], args["scale"], args["causal"], args["layout"], args["dtype"],
+                   args["stream"])
+    assert rc == code, fa.fa_status_string(rc)
+
+
+def test_product_path_has_no_cpu_fallback(monkeypatch, tmp_path):
+    """With the library absent, the binding raises instead of computing."""
+    import importlib
+
+    mod = importlib.reload(fa)
+    monkeypatch.setattr(mod, "lib_path", lambda: str(tmp_path / "missing.so"))
+    mod._LIB = None
+    with pytest.raises(RuntimeError):
+        mod.lib()
+    importlib.reload(fa)
+
+
+def test_binding_does_not_import_oracle():
+    src = open(os.path.join(ROOT, "tiled_attention_13_b200", "__init__.py")).read()
+    for f in os.listdir(os.path.join(ROOT, "tiled_attention_13_b200", "csrc")):
+        src += open(os.path.join(ROOT, "tiled_attention_13_b200", "csrc", f)).read()
+    assert "oracle" not in src

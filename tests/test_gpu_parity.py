@@ -1,0 +1,152 @@
+"""GPU parity: the CUDA path (through the C ABI) against the float64 oracle.
+
+Small ragged problems are compared element by element; they span several
+128-row Q tiles and 128-key KV tiles with ragged tails, both layouts, both
+masks, both head dims and all three input dtypes.  The named full-size
+workloads are run in the launch configuration the bench uses and checked on
+sampled rows (first and last rows, tile boundaries and random rows of a few
+heads) that the oracle evaluates one at a time.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+import tiled_attention_13_b200 as fa
+from tiled_attention_13_b200.inputs import WORKLOADS, Workload, make_qkv
+
+from .parity import compare_full, compare_sampled, half_ulp, run_gpu
+
+pytestmark = pytest.mark.gpu
+
+SHAPES = [  # (B, H, Nq, Nkv)
+    (1, 1, 1, 1),
+    (1, 2, 77, 77),
+    (1, 1, 128, 128),
+    (1, 1, 129, 127),
+    (2, 3, 300, 333),
+    (2, 1, 255, 257),
+    (1, 2, 513, 1000),
+    (1, 1, 384, 40),
+]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _lib(fa_lib):
+    return fa_lib
+
+
+@pytest.mark.parametrize("layout", ["BHND", "BSND"])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("shape", SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_small_bf16(shape, d, causal, layout):
+    B, H, Nq, Nkv = shape
+    wl = Workload("small", B=B, H=H, Nq=Nq, Nkv=Nkv, d=d, dtype="bf16", layout=layout, causal=causal,
+                  seed=sum(shape) + d)
+    compare_full(wl)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("shape", [(2, 3, 300, 333), (1, 2, 513, 1000)], ids=lambda s: "x".join(map(str, s)))
+def test_small_fp16(shape, d, causal):
+    B, H, Nq, Nkv = shape
+    wl = Workload("small16", B=B, H=H, Nq=Nq, Nkv=Nkv, d=d, dtype="fp16", layout="BSND", causal=causal, seed=5)
+    compare_full(wl)
+
+
+@pytest.mark.parametrize("layout", ["BHND", "BSND"])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("shape", [(1, 1, 1, 1), (2, 3, 300, 333), (1, 1, 40, 70)], ids=lambda s: "x".join(map(str, s)))
+def test_small_fp32(shape, d, causal, layout):
+    B, H, Nq, Nkv = shape
+    wl = Workload("small32", B=B, H=H, Nq=Nq, Nkv=Nkv, d=d, dtype="fp32", layout=layout, causal=causal, seed=9)
+    compare_full(wl)
+
+
+def test_explicit_scale_and_regression_inputs():
+    """Explicit scale, and page 1's regression families: all-ones, large random
+    values and alternating extremes (section 数值安全的边界条件)."""
+    wl = Workload("s", B=1, H=2, Nq=200, Nkv=300, d=128, dtype="bf16", layout="BHND", causal=False, seed=3)
+    compare_full(wl, scale=0.05)
+    from oracle import attention_batched
+
+    shape_q, shape_kv = wl.q_shape(), wl.kv_shape()
+    g = torch.Generator().manual_seed(11)
+    cases = {
+        "ones": (torch.ones(shape_q), torch.ones(shape_kv), torch.randn(shape_kv, generator=g)),
+        "large": (torch.randn(shape_q, generator=g) * 8, torch.randn(shape_kv, generator=g) * 8,
+                  torch.randn(shape_kv, generator=g)),
+        "alternating": (torch.ones(shape_q) * 6 * (1 - 2 * (torch.arange(200) % 2)).view(1, 1, -1, 1),
+                        torch.ones(shape_kv) * 6 * (1 - 2 * (torch.arange(300) % 2)).view(1, 1, -1, 1),
+                        torch.randn(shape_kv, generator=g)),
+    }
+    # These inputs are far from N(0, 1): scores spread over hundreds of units,
+    # so P is nearly one-hot and O nearly a single row of V.  The bound follows
+    # from the arithmetic: rounding O to bf16 costs half an ulp of O, rounding
+    # P to bf16 before P V costs at most 2^-9 relative per weight, i.e.
+    # 2^-9 max|V| on O; 1e-3 covers the fp32 accumulation.
+    for name, (q, k, v) in cases.items():
+        q, k, v = (t.to(torch.bfloat16) for t in (q, k, v))
+        vmax = float(v.float().abs().max())
+        for causal in (False, True):
+            o, lse = fa.forward(q.cuda(), k.cuda(), v.cuda(), causal=causal)
+            o_ref, l_ref = attention_batched(q, k, v, causal=causal)
+            err = np.abs(o.double().cpu().numpy() - o_ref)
+            bar = half_ulp(o_ref, "bf16") + 2.0 ** -9 * vmax + 1e-3
+            el = np.abs(lse.double().cpu().numpy() - l_ref).max()
+            assert np.all(err <= bar), (name, causal, err.max())
+            assert el <= 1e-3, (name, causal, el)
+
+
+def test_deterministic_and_lse_optional():
+    wl = Workload("det", B=2, H=4, Nq=700, Nkv=900, d=128, dtype="bf16", layout="BSND", causal=True, seed=21)
+    q, k, v = (t.cuda() for t in make_qkv(wl))
+    o1, l1 = run_gpu(wl, q, k, v)
+    o2, l2 = run_gpu(wl, q, k, v)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    o3 = torch.empty_like(q)
+    rc = fa.fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o3.data_ptr(), None, 2, 4, 700, 900, 128, -1.0, 1,
+                   fa.FA_LAYOUT_BSND, fa.FA_DTYPE_BF16, torch.cuda.current_stream().cuda_stream)
+    assert rc == 0
+    torch.cuda.synchronize()
+    assert torch.equal(o1, o3)
+    assert fa.fa_get_device_status(None) == 0
+
+
+def test_empty_problem_is_a_noop():
+    q = torch.zeros((1, 2, 0, 64), dtype=torch.bfloat16, device="cuda")
+    k = torch.randn((1, 2, 5, 64), device="cuda").to(torch.bfloat16)
+    o, lse = fa.forward(q, k, k)
+    assert o.shape == q.shape and lse.shape == (1, 2, 0)
+
+
+# ----------------------------------------------------------------- named workloads
+def test_tiny_full():
+    for name in ("tiny", "tiny-causal"):
+        compare_full(WORKLOADS[name])
+
+
+def test_cross_attention_full():
+    compare_full(WORKLOADS["cross"])
+
+
+def test_llama13b_2k_full():
+    compare_full(WORKLOADS["llama13b-2k"])
+
+
+@pytest.mark.parametrize("name", ["llama13b-4k", "llama13b-8k", "b4-2k", "b4-2k-causal", "b4-8k",
+                                  "b4-8k-causal", "b4-32k", "b4-32k-causal"])
+def test_named_sampled(name):
+    wl = WORKLOADS[name]
+    heads = [(0, 0), (wl.B - 1, wl.H - 1), (wl.B // 2, wl.H // 2)]
+    compare_sampled(wl, heads, rows_per_head=40)
+
+
+def test_long_context_sampled():
+    wl = WORKLOADS["long"]
+    heads = [(0, 0), (0, wl.H - 1)]
+    compare_sampled(wl, heads, rows_per_head=24)
+    torch.cuda.empty_cache()

@@ -266,6 +266,14 @@ def test_row_blocking_is_invisible():
     assert np.max(np.abs(o - o2)) <= 1e-14 and np.max(np.abs(lse - lse2)) <= 1e-14
 
 
+def test_row_offset_block_equals_full_rows():
+    nq, nkv, d = 50, 60, 4
+    q, k, v = rnd(nq, d), rnd(nkv, d), rnd(nkv, d)
+    o, lse = attention(q, k, v, causal=True)
+    o2, lse2 = attention(q[17:41], k, v, causal=True, row_offset=17)
+    assert np.max(np.abs(o[17:41] - o2)) <= 1e-14 and np.max(np.abs(lse[17:41] - lse2)) <= 1e-14
+
+
 def test_empty_and_invalid():
     o, lse = attention(np.zeros((0, 4)), rnd(3, 4), rnd(3, 4))
     assert o.shape == (0, 4) and lse.shape == (0,)

@@ -1,1 +1,204 @@
-"""B200 (sm_100a) fused scaled-dot-product attention forward."""
+"""B200 (sm_100a) fused scaled-dot-product attention forward.
+
+Python side of the C ABI in ``include/fa.h``: the functions below have the
+same names and arguments as the C entry points and only marshal arguments;
+every step of the computation runs in the CUDA library ``libfa_b200.so``
+(built in-tree by ``python -m tiled_attention_13_b200.build``).  There is no
+CPU path: when the library is missing, every call raises.
+
+``forward(q, k, v, ...)`` is the torch-facing convenience wrapper: it takes
+CUDA tensors, allocates O and LSE with torch (PyTorch is used for device
+memory and streams only) and launches on the current stream.
+``forward_host(...)`` is the end-to-end form: pinned host tensors in, host
+tensors out, with the copies on the same stream.
+"""
+
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+__all__ = [
+    "FA_LAYOUT_BHND", "FA_LAYOUT_BSND", "FA_DTYPE_BF16", "FA_DTYPE_FP16", "FA_DTYPE_FP32",
+    "FaError", "lib", "lib_path", "fa_fwd", "fa_status_string", "fa_get_device_status",
+    "fa_set_wait_timeout_us", "fa_debug_set_fault", "fa_abi_version", "forward", "forward_host",
+    "EXPORTED",
+]
+
+FA_LAYOUT_BHND, FA_LAYOUT_BSND = 0, 1
+FA_DTYPE_BF16, FA_DTYPE_FP16, FA_DTYPE_FP32 = 0, 1, 2
+FA_OK = 0
+
+EXPORTED = ("fa_fwd", "fa_status_string", "fa_get_device_status", "fa_set_wait_timeout_us",
+            "fa_debug_set_fault", "fa_abi_version")
+
+_LIB = None
+
+
+def lib_path() -> str:
+    return os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa_b200.so")
+
+
+class FaError(RuntimeError):
+    def __init__(self, code: int, what: str = ""):
+        self.code = code
+        super().__init__(f"{what}: {fa_status_string(code)} ({code})" if what else fa_status_string(code))
+
+
+def lib() -> ctypes.CDLL:
+    """Load the CUDA library (once).  Raises if it has not been built."""
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    path = lib_path()
+    if not os.path.exists(path):
+        raise RuntimeError(f"{path} is missing: build it with `python -m tiled_attention_13_b200.build`")
+    L = ctypes.CDLL(path)
+    i64, vp = ctypes.c_int64, ctypes.c_void_p
+    L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, ctypes.c_float, ctypes.c_int,
+                         ctypes.c_int, ctypes.c_int, vp]
+    L.fa_fwd.restype = ctypes.c_int
+    L.fa_status_string.argtypes = [ctypes.c_int]
+    L.fa_status_string.restype = ctypes.c_char_p
+    L.fa_get_device_status.argtypes = [vp]
+    L.fa_get_device_status.restype = ctypes.c_int
+    L.fa_set_wait_timeout_us.argtypes = [ctypes.c_uint32]
+    L.fa_set_wait_timeout_us.restype = ctypes.c_uint32
+    L.fa_debug_set_fault.argtypes = [ctypes.c_int]
+    L.fa_debug_set_fault.restype = ctypes.c_int
+    L.fa_abi_version.argtypes = []
+    L.fa_abi_version.restype = ctypes.c_int
+    _LIB = L
+    return L
+
+
+# ------------------------------------------------------------------ C ABI, 1:1
+def fa_fwd(q, k, v, o, lse, B, H, Nq, Nkv, d, scale, causal, layout, dtype, stream) -> int:
+    """int fa_fwd(q, k, v, o, lse, B, H, Nq, Nkv, d, scale, causal, layout, dtype, stream).
+
+    Pointers are integers (device addresses) or None; returns the status code.
+    """
+    return lib().fa_fwd(q, k, v, o, lse, B, H, Nq, Nkv, d, float(scale), int(causal), int(layout),
+                        int(dtype), stream)
+
+
+def fa_status_string(status: int) -> str:
+    return lib().fa_status_string(int(status)).decode()
+
+
+def fa_get_device_status(stream=None) -> int:
+    return lib().fa_get_device_status(stream)
+
+
+def fa_set_wait_timeout_us(us: int) -> int:
+    return lib().fa_set_wait_timeout_us(int(us))
+
+
+def fa_debug_set_fault(mode: int) -> int:
+    return lib().fa_debug_set_fault(int(mode))
+
+
+def fa_abi_version() -> int:
+    return lib().fa_abi_version()
+
+
+# ------------------------------------------------------------------ torch wrappers
+def _dtype_code(t):
+    import torch
+
+    return {torch.bfloat16: FA_DTYPE_BF16, torch.float16: FA_DTYPE_FP16, torch.float32: FA_DTYPE_FP32}[t.dtype]
+
+
+def _dims(q, k, layout):
+    if layout == "BHND":
+        B, H, Nq, d = q.shape
+        Nkv = k.shape[2]
+    elif layout == "BSND":
+        B, Nq, H, d = q.shape
+        Nkv = k.shape[1]
+    else:
+        raise ValueError(f"layout must be 'BHND' or 'BSND', got {layout!r}")
+    return B, H, Nq, Nkv, d
+
+
+def forward(q, k, v, causal: bool = False, scale=None, layout: str = "BHND", out=None, lse=None,
+            stream=None):
+    """O, LSE = softmax(scale Q K^T [+causal]) V on the GPU (returns (o, lse)).
+
+    q: [B,H,Nq,d] (BHND) or [B,Nq,H,d] (BSND); k, v the same with Nkv; all
+    contiguous CUDA tensors of one dtype (bf16, fp16 or fp32); d in {64, 128}.
+    scale None -> 1/sqrt(d).  LSE is fp32 [B, H, Nq].
+    """
+    import torch
+
+    for t in (q, k, v):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v must be contiguous CUDA tensors")
+    if not (q.dtype == k.dtype == v.dtype):
+        raise ValueError("q, k, v must share one dtype")
+    B, H, Nq, Nkv, d = _dims(q, k, layout)
+    if k.shape != v.shape:
+        raise ValueError("k and v must have the same shape")
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    sc = -1.0 if scale is None else float(scale)
+    rc = fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr() if lse.numel() else None,
+                B, H, Nq, Nkv, d, sc, int(bool(causal)), FA_LAYOUT_BHND if layout == "BHND" else FA_LAYOUT_BSND,
+                _dtype_code(q), stream)
+    if rc != FA_OK:
+        raise FaError(rc, "fa_fwd")
+    return out, lse
+
+
+class HostForward:
+    """End-to-end form over pinned host tensors with reusable device buffers.
+
+    Each call copies q, k, v host->device, runs fa_fwd and copies O and LSE
+    device->host, all on one stream; ``__call__`` returns the pinned host
+    outputs (valid after ``torch.cuda.current_stream().synchronize()``).
+    """
+
+    def __init__(self, q_host, k_host, v_host, causal=False, scale=None, layout="BHND", device="cuda"):
+        import torch
+
+        self.causal, self.scale, self.layout = causal, scale, layout
+        self.dev = torch.device(device)
+        self.qd = torch.empty_like(q_host, device=self.dev)
+        self.kd = torch.empty_like(k_host, device=self.dev)
+        self.vd = torch.empty_like(v_host, device=self.dev)
+        self.od = torch.empty_like(self.qd)
+        B, H, Nq, _, _ = _dims(q_host, k_host, layout)
+        self.lsed = torch.empty((B, H, Nq), dtype=torch.float32, device=self.dev)
+        self.o_host = torch.empty_like(q_host).pin_memory()
+        self.lse_host = torch.empty((B, H, Nq), dtype=torch.float32).pin_memory()
+        self.h2d_bytes = sum(t.numel() * t.element_size() for t in (q_host, k_host, v_host))
+        self.d2h_bytes = self.o_host.numel() * self.o_host.element_size() + self.lse_host.numel() * 4
+
+    def __call__(self, q_host, k_host, v_host):
+        self.qd.copy_(q_host, non_blocking=True)
+        self.kd.copy_(k_host, non_blocking=True)
+        self.vd.copy_(v_host, non_blocking=True)
+        forward(self.qd, self.kd, self.vd, causal=self.causal, scale=self.scale, layout=self.layout,
+                out=self.od, lse=self.lsed)
+        self.o_host.copy_(self.od, non_blocking=True)
+        self.lse_host.copy_(self.lsed, non_blocking=True)
+        return self.o_host, self.lse_host
+
+
+def forward_host(q_host, k_host, v_host, causal=False, scale=None, layout="BHND", device="cuda"):
+    """One end-to-end call from host tensors; returns host (o, lse) after syncing."""
+    import torch
+
+    hf = HostForward(q_host, k_host, v_host, causal=causal, scale=scale, layout=layout, device=device)
+    o, lse = hf(q_host, k_host, v_host)
+    torch.cuda.current_stream(hf.dev).synchronize()
+    return o.clone(), lse.clone()
+
+
+def default_scale(d: int) -> float:
+    return 1.0 / math.sqrt(d)

@@ -1,0 +1,237 @@
+// fa_api.cu -- the C ABI declared in include/fa.h: argument validation, TMA
+// descriptor encoding, launch configuration and the device status word.
+//
+// One translation unit holds every kernel so that they share the status word
+// (a static __device__ variable: no device allocation anywhere).
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <atomic>
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+#include <type_traits>
+
+#include "fa.h"
+
+namespace fa {
+// Bit 0: a bounded wait expired.  Written by kernels, read and cleared by
+// fa_get_device_status().
+__device__ unsigned int g_status_word = 0;
+}  // namespace fa
+
+#include "fa_fwd_simt.cuh"
+#include "fa_fwd_tc.cuh"
+
+namespace {
+
+constexpr uint32_t kDefaultTimeoutUs = 2000000u;
+std::atomic<uint32_t> g_timeout_us{kDefaultTimeoutUs};
+std::atomic<int> g_fault_mode{0};
+
+constexpr int kMaxDevices = 64;
+struct DeviceInfo {
+  bool ready = false;
+  bool supported = false;
+  int num_sms = 0;
+  unsigned int* status = nullptr;  // device address of fa::g_status_word
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+EncodeTiledFn g_encode = nullptr;
+
+template <typename K>
+bool set_smem_attr(K kernel, int bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+}
+
+// Per-device one-time set-up with that device current: properties, the
+// status word's device address, kernel shared-memory attributes and the
+// driver's tensor-map encoder.
+int device_setup(int dev, DeviceInfo** out) {
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_NO_DEVICE;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& di = g_dev[dev];
+  if (!di.ready) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return FA_ERR_NO_DEVICE;
+    di.supported = (prop.major == 10 && prop.minor == 0);
+    di.num_sms = prop.multiProcessorCount;
+    if (di.supported) {
+      void* sym = nullptr;
+      if (cudaGetSymbolAddress(&sym, fa::g_status_word) != cudaSuccess) return FA_ERR_LAUNCH;
+      di.status = static_cast<unsigned int*>(sym);
+      bool ok = true;
+      ok &= set_smem_attr(fa::fa_fwd_tc_kernel<64, __nv_bfloat16>, fa::TcCfg<64>::SMEM_BYTES);
+      ok &= set_smem_attr(fa::fa_fwd_tc_kernel<128, __nv_bfloat16>, fa::TcCfg<128>::SMEM_BYTES);
+      ok &= set_smem_attr(fa::fa_fwd_tc_kernel<64, __half>, fa::TcCfg<64>::SMEM_BYTES);
+      ok &= set_smem_attr(fa::fa_fwd_tc_kernel<128, __half>, fa::TcCfg<128>::SMEM_BYTES);
+      ok &= set_smem_attr(fa::fa_fwd_simt_kernel<64>, fa::simt_smem_bytes<64>());
+      ok &= set_smem_attr(fa::fa_fwd_simt_kernel<128>, fa::simt_smem_bytes<128>());
+      if (!ok) return FA_ERR_LAUNCH;
+      if (g_encode == nullptr) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || fn == nullptr)
+          return FA_ERR_LAUNCH;
+        g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+      }
+    }
+    di.ready = true;
+  }
+  if (!di.supported) return FA_ERR_NO_DEVICE;
+  *out = &di;
+  return FA_OK;
+}
+
+// 4-D tensor map over a [B, H, N, D] (BHND) or [B, N, H, D] (BSND) 16-bit
+// tensor, box = 64 columns x 128 rows of one (b, h), 128-byte swizzle,
+// out-of-range rows read as zero.
+bool make_tmap(CUtensorMap* tm, const void* base, bool bf16, bool bsnd, int64_t B, int64_t H, int64_t N,
+               int64_t D) {
+  cuuint64_t dims[4], strides[3];
+  cuuint32_t box[4], estr[4] = {1, 1, 1, 1};
+  const cuuint64_t es = 2;
+  if (!bsnd) {
+    dims[0] = D; dims[1] = N; dims[2] = H; dims[3] = B;
+    strides[0] = D * es; strides[1] = N * D * es; strides[2] = H * N * D * es;
+    box[0] = 64; box[1] = 128; box[2] = 1; box[3] = 1;
+  } else {
+    dims[0] = D; dims[1] = H; dims[2] = N; dims[3] = B;
+    strides[0] = D * es; strides[1] = H * D * es; strides[2] = N * H * D * es;
+    box[0] = 64; box[1] = 1; box[2] = 128; box[3] = 1;
+  }
+  CUresult r = g_encode(tm, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
+                        const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <int D, typename T>
+int launch_tc(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
+              int64_t Nq, int64_t Nkv, float scale, int causal, bool bsnd, cudaStream_t stream,
+              const DeviceInfo& di) {
+  constexpr bool BF16 = std::is_same<T, __nv_bfloat16>::value;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap(&tq, q, BF16, bsnd, B, H, Nq, D) || !make_tmap(&tk, k, BF16, bsnd, B, H, Nkv, D) ||
+      !make_tmap(&tv, v, BF16, bsnd, B, H, Nkv, D))
+    return FA_ERR_LAUNCH;
+  fa::TcParams p;
+  p.o = o;
+  p.lse = lse;
+  p.B = (int)B; p.H = (int)H; p.Nq = (int)Nq; p.Nkv = (int)Nkv;
+  p.bsnd = bsnd ? 1 : 0;
+  p.causal = causal;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const int64_t qtiles = (Nq + fa::TC_BM - 1) / fa::TC_BM;
+  p.n_pairs = (int)((qtiles + 1) / 2);
+  const int64_t units = B * H * (int64_t)p.n_pairs;
+  if (units > INT32_MAX) return FA_ERR_UNSUPPORTED;
+  p.n_units = (int)units;
+  p.timeout_ns = (uint64_t)g_timeout_us.load() * 1000ull;
+  p.fault_mode = g_fault_mode.load();
+  const int grid = (int)(units < di.num_sms ? units : di.num_sms);
+  fa::fa_fwd_tc_kernel<D, T><<<grid, fa::TC_THREADS, fa::TcCfg<D>::SMEM_BYTES, stream>>>(tq, tk, tv, p,
+                                                                                         di.status);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+template <int D>
+int launch_simt(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
+                int64_t Nq, int64_t Nkv, float scale, int causal, bool bsnd, cudaStream_t stream) {
+  fa::SimtParams p;
+  p.q = static_cast<const float*>(q);
+  p.k = static_cast<const float*>(k);
+  p.v = static_cast<const float*>(v);
+  p.o = static_cast<float*>(o);
+  p.lse = lse;
+  p.B = (int)B; p.H = (int)H; p.Nq = (int)Nq; p.Nkv = (int)Nkv;
+  p.bsnd = bsnd ? 1 : 0;
+  p.causal = causal;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.n_qblocks = (int)((Nq + fa::SIMT_ROWS - 1) / fa::SIMT_ROWS);
+  const int64_t blocks = B * H * (int64_t)p.n_qblocks;
+  if (blocks > INT32_MAX) return FA_ERR_UNSUPPORTED;
+  fa::fa_fwd_simt_kernel<D><<<(int)blocks, fa::SIMT_THREADS, fa::simt_smem_bytes<D>(), stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+}  // namespace
+
+extern "C" {
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H, int64_t Nq,
+           int64_t Nkv, int64_t d, float scale, int causal, int layout, int dtype, void* stream) {
+  if (B < 0 || H < 0 || Nq < 0 || Nkv < 0 || d <= 0) return FA_ERR_INVALID_ARG;
+  if (layout != FA_LAYOUT_BHND && layout != FA_LAYOUT_BSND) return FA_ERR_INVALID_ARG;
+  if (dtype != FA_DTYPE_BF16 && dtype != FA_DTYPE_FP16 && dtype != FA_DTYPE_FP32) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0 || Nq == 0) return FA_OK;  // nothing to compute
+  if (Nkv == 0) return FA_ERR_INVALID_ARG;         // softmax over an empty key set
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return FA_ERR_INVALID_ARG;
+  if (B > INT32_MAX || H > INT32_MAX || B * H > INT32_MAX || Nq > INT32_MAX - 256 || Nkv > INT32_MAX - 256)
+    return FA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      (lse != nullptr && !aligned(lse, 4)))
+    return FA_ERR_MISALIGNED;
+  if (!(scale > 0.f) || std::isinf(scale)) scale = 1.0f / std::sqrt((float)d);
+
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_NO_DEVICE;
+  DeviceInfo* di = nullptr;
+  const int st = device_setup(dev, &di);
+  if (st != FA_OK) return st;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool bsnd = layout == FA_LAYOUT_BSND;
+  if (dtype == FA_DTYPE_FP32) {
+    return d == 64 ? launch_simt<64>(q, k, v, o, lse, B, H, Nq, Nkv, scale, causal, bsnd, s)
+                   : launch_simt<128>(q, k, v, o, lse, B, H, Nq, Nkv, scale, causal, bsnd, s);
+  }
+  if (dtype == FA_DTYPE_BF16) {
+    return d == 64 ? launch_tc<64, __nv_bfloat16>(q, k, v, o, lse, B, H, Nq, Nkv, scale, causal, bsnd, s, *di)
+                   : launch_tc<128, __nv_bfloat16>(q, k, v, o, lse, B, H, Nq, Nkv, scale, causal, bsnd, s, *di);
+  }
+  return d == 64 ? launch_tc<64, __half>(q, k, v, o, lse, B, H, Nq, Nkv, scale, causal, bsnd, s, *di)
+                 : launch_tc<128, __half>(q, k, v, o, lse, B, H, Nq, Nkv, scale, causal, bsnd, s, *di);
+}
+
+const char* fa_status_string(int status) {
+  switch (status) {
+    case FA_OK: return "FA_OK";
+    case FA_ERR_INVALID_ARG: return "FA_ERR_INVALID_ARG: invalid argument";
+    case FA_ERR_UNSUPPORTED: return "FA_ERR_UNSUPPORTED: unsupported head dim or size";
+    case FA_ERR_MISALIGNED: return "FA_ERR_MISALIGNED: pointer alignment";
+    case FA_ERR_LAUNCH: return "FA_ERR_LAUNCH: CUDA launch or descriptor failure";
+    case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT: a bounded device wait expired";
+    case FA_ERR_NO_DEVICE: return "FA_ERR_NO_DEVICE: no usable sm_100 device";
+    default: return "FA_ERR_UNKNOWN";
+  }
+}
+
+int fa_get_device_status(void* stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return FA_ERR_LAUNCH;
+  unsigned int w = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&w, fa::g_status_word, sizeof(w)) != cudaSuccess) return FA_ERR_LAUNCH;
+  if (w != 0 && cudaMemcpyToSymbol(fa::g_status_word, &zero, sizeof(zero)) != cudaSuccess) return FA_ERR_LAUNCH;
+  return (w & 1u) ? FA_ERR_TIMEOUT : FA_OK;
+}
+
+uint32_t fa_set_wait_timeout_us(uint32_t us) {
+  return g_timeout_us.exchange(us == 0 ? kDefaultTimeoutUs : us);
+}
+
+int fa_debug_set_fault(int mode) { return g_fault_mode.exchange(mode); }
+
+int fa_abi_version(void) { return (1 << 16) | 0; }
+
+}  // extern "C"

@@ -1,0 +1,456 @@
+// fa_fwd_tc.cuh -- tensor-core (tcgen05 + TMEM + TMA) attention forward for
+// sm_100a, bf16 or fp16 inputs, fp32 accumulation, head dim D in {64, 128}.
+//
+// Method (page 1, "CANN ops-transformer FlashAttentionScore", section 分块
+// Tiling 的计算骨架: every Q tile walks all of its K/V tiles and merges them
+// with the online softmax; page 3, "ops-nn efficient attention for AIGC",
+// section 2.2: unnormalised accumulator o = o * corr + exp(S - m_new) V,
+// divided by l once at the end; section 3.2: causal block skip).
+//
+// B200 mapping (the pages' Cube/Vector/UB design is prior art only):
+//
+//   work unit   one (batch, head, pair of 128-row Q tiles); a persistent grid
+//               of <= #SM CTAs walks the units in a static strided order,
+//               heaviest causal pairs first (longest-processing-time order).
+//   warps 0-3   softmax warpgroup for Q tile 0 of the pair (one thread per
+//               query row = one TMEM lane), then its epilogue
+//   warps 4-7   softmax warpgroup for Q tile 1
+//   warp 8      TMEM allocator and the single MMA-issuing thread
+//   warp 9      TMA producer (Q tiles, K/V ring of KST stages)
+//
+//   TMEM (512 columns x 128 lanes, fp32):  S0 [0,128)  S1 [128,256)
+//   O0 [256, 256+D)  O1 [256+D, 256+2D).  P_i (bf16/fp16 pairs) overwrites
+//   the first 64 columns of S_i once the softmax has read S_i.
+//
+//   MMA order per KV step j (tile i = 0, 1):  O_i += P_i(j-1) V_(j-1), then
+//   S_i(j) = Q_i K_j^T, then commit -> s_full[i].  The tensor pipe executes
+//   a CTA's MMAs in issue order, so S_i(j) overwrites P_i(j-1) only after
+//   the P V product has read it, and when s_full[i] fires O_i is quiescent
+//   (the softmax may rescale it in place).  While the softmax of tile 0 runs,
+//   the tensor pipe works on tile 1 and vice versa.
+//
+//   Online softmax in the exp2 domain: x = s * scale * log2(e).  The running
+//   reference max m is only moved when a tile's max exceeds it by more than
+//   2^8 (then O and l are rescaled by 2^(m_old - m_new)); otherwise P may
+//   reach 2^8, which bf16/fp16 and the fp32 sums hold exactly as well.  The
+//   final O = o / l and LSE = (m + log2 l) ln 2 are the same numbers either
+//   way: the reference max cancels.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include "ptx.cuh"
+
+namespace fa {
+
+constexpr int TC_THREADS = 320;  // 10 warps
+constexpr int TC_BM = 128;       // query rows per Q tile
+constexpr int TC_BN = 128;       // keys per KV tile
+constexpr float TC_RESCALE_THRESHOLD = 8.0f;  // log2 units
+
+template <int D>
+struct TcCfg {
+  static constexpr int TILE_BYTES = TC_BM * D * 2;          // one 128 x D tile of 16-bit values
+  static constexpr int CHUNKS = D / 64;                     // 128-byte-wide column chunks per tile
+  static constexpr int CHUNK_BYTES = TC_BM * 128;           // 128 rows x 128 bytes
+  static constexpr int KST = (D == 128) ? 2 : 4;            // K/V ring depth
+  static constexpr int OFF_Q = 0;                           // Q0, Q1
+  static constexpr int OFF_K = 2 * TILE_BYTES;              // KST K tiles
+  static constexpr int OFF_V = OFF_K + KST * TILE_BYTES;    // KST V tiles
+  static constexpr int OFF_BAR = OFF_V + KST * TILE_BYTES;  // barriers
+  static constexpr int NBAR = 2 + 2 + 4 * KST + 2 + 2 + 2 + 1;
+  static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 /*tmem slot + abort*/ + 1024 /*align slack*/;
+  static constexpr int TMEM_S0 = 0, TMEM_S1 = 128, TMEM_O0 = 256, TMEM_O1 = 256 + D;
+  static constexpr uint32_t TMEM_COLS = 512;
+};
+
+struct TcParams {
+  void* o;
+  float* lse;
+  int B, H, Nq, Nkv;
+  int bsnd;          // 1: [B, N, H, D] rows, 0: [B, H, N, D]
+  int causal;
+  float scale_log2;  // softmax scale * log2(e)
+  int n_pairs;       // ceil(ceil(Nq / 128) / 2)
+  int n_units;       // B * H * n_pairs
+  uint64_t timeout_ns;
+  int fault_mode;
+};
+
+// Per-unit geometry shared by every role (pure integer arithmetic).
+struct Unit {
+  int b, h, qt0;      // qt0 = first Q tile index (even), second = qt0 + 1
+  int active1;        // second Q tile has at least one valid row
+  int n0, n1;         // KV tiles for tile 0 / tile 1 (0 if inactive)
+};
+
+__device__ __forceinline__ int kv_tiles_for(int qt, int Nkv, int causal) {
+  int lim = Nkv;
+  if (causal) {
+    long long e = (long long)(qt + 1) * TC_BM;
+    if (e < lim) lim = (int)e;
+  }
+  return (lim + TC_BN - 1) / TC_BN;
+}
+
+__device__ __forceinline__ Unit decode_unit(int u, const TcParams& p) {
+  Unit w;
+  const int BH = p.B * p.H;
+  const int pair = p.n_pairs - 1 - u / BH;  // heaviest (causal) pairs first
+  const int bh = u % BH;
+  w.b = bh / p.H;
+  w.h = bh % p.H;
+  w.qt0 = 2 * pair;
+  w.active1 = ((long long)(w.qt0 + 1) * TC_BM < (long long)p.Nq) ? 1 : 0;
+  w.n0 = kv_tiles_for(w.qt0, p.Nkv, p.causal);
+  w.n1 = w.active1 ? kv_tiles_for(w.qt0 + 1, p.Nkv, p.causal) : 0;
+  return w;
+}
+
+template <typename T>
+struct Pack;
+template <>
+struct Pack<__nv_bfloat16> {
+  static __device__ __forceinline__ uint32_t two(float lo, float hi) {
+    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  }
+};
+template <>
+struct Pack<__half> {
+  static __device__ __forceinline__ uint32_t two(float lo, float hi) {
+    __half2 v = __floats2half2_rn(lo, hi);
+    return *reinterpret_cast<uint32_t*>(&v);
+  }
+};
+
+template <int D, typename T>
+__global__ void __launch_bounds__(TC_THREADS, 1)
+    fa_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
+                     const __grid_constant__ CUtensorMap tm_v, TcParams p, unsigned int* status_word) {
+  using C = TcCfg<D>;
+  constexpr bool IS_BF16 = std::is_same<T, __nv_bfloat16>::value;
+  extern __shared__ uint8_t smem_raw[];
+  // 1024-byte alignment: the 128-byte swizzle pattern is anchored there.
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  // barrier indices
+  const int B_QFULL = 0, B_QEMPTY = 2, B_KFULL = 4, B_KEMPTY = 4 + C::KST, B_VFULL = 4 + 2 * C::KST,
+            B_VEMPTY = 4 + 3 * C::KST, B_SFULL = 4 + 4 * C::KST, B_PFULL = B_SFULL + 2, B_OFULL = B_PFULL + 2,
+            B_DRAIN = B_OFULL + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  auto bar = [&](int i) { return smem_u32(&bars[i]); };
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(bar(B_QFULL + i), 1);
+      mbar_init(bar(B_QEMPTY + i), 1);
+      mbar_init(bar(B_SFULL + i), 1);
+      mbar_init(bar(B_PFULL + i), 128);
+      mbar_init(bar(B_OFULL + i), 1);
+    }
+    for (int s = 0; s < C::KST; ++s) {
+      mbar_init(bar(B_KFULL + s), 1);
+      mbar_init(bar(B_KEMPTY + s), 1);
+      mbar_init(bar(B_VFULL + s), 1);
+      mbar_init(bar(B_VEMPTY + s), 1);
+    }
+    mbar_init(bar(B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 8) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  if (warp == 9 && lane == 0) {
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_k);
+    prefetch_tmap(&tm_v);
+  }
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  WaitCtx wctx{abort_flag, status_word, p.timeout_ns, 1u};
+
+  if (warp == 9) {
+    // ------------------------------------------------------------ TMA producer
+    if (lane == 0) {
+      const uint64_t pol_q = l2_policy_evict_first();
+      const uint64_t pol_kv = l2_policy_evict_last();
+      uint32_t q_phase[2] = {0, 0};
+      int st = 0;
+      uint32_t kv_phase = 0;
+      // outstanding-load bookkeeping for the drain at exit
+      uint32_t k_issued[C::KST], v_issued[C::KST], q_issued[2];
+      bool k_pend[C::KST], v_pend[C::KST], q_pend[2];
+      for (int s = 0; s < C::KST; ++s) { k_pend[s] = v_pend[s] = false; k_issued[s] = v_issued[s] = 0; }
+      q_pend[0] = q_pend[1] = false; q_issued[0] = q_issued[1] = 0;
+      bool ok = true;
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+        const Unit w = decode_unit(u, p);
+        for (int i = 0; i < 2 && ok; ++i) {
+          if (i == 1 && !w.active1) break;
+          if (!mbar_wait(bar(B_QEMPTY + i), q_phase[i] ^ 1, wctx)) { ok = false; break; }
+          const uint32_t dst = sbase + C::OFF_Q + i * C::TILE_BYTES;
+          mbar_arrive_expect_tx(bar(B_QFULL + i), C::TILE_BYTES);
+          const int row0 = (w.qt0 + i) * TC_BM;
+          for (int c = 0; c < C::CHUNKS; ++c) {
+            if (p.bsnd)
+              tma_load_4d(dst + c * C::CHUNK_BYTES, &tm_q, bar(B_QFULL + i), c * 64, w.h, row0, w.b, pol_q);
+            else
+              tma_load_4d(dst + c * C::CHUNK_BYTES, &tm_q, bar(B_QFULL + i), c * 64, row0, w.h, w.b, pol_q);
+          }
+          q_pend[i] = true; q_issued[i] = q_phase[i];
+          q_phase[i] ^= 1;
+        }
+        const int N = w.n0 > w.n1 ? w.n0 : w.n1;
+        for (int j = 0; j < N && ok; ++j) {
+          const int kv0 = j * TC_BN;
+          if (!mbar_wait(bar(B_KEMPTY + st), kv_phase ^ 1, wctx)) { ok = false; break; }
+          mbar_arrive_expect_tx(bar(B_KFULL + st), C::TILE_BYTES);
+          const uint32_t kdst = sbase + C::OFF_K + st * C::TILE_BYTES;
+          for (int c = 0; c < C::CHUNKS; ++c) {
+            if (p.bsnd)
+              tma_load_4d(kdst + c * C::CHUNK_BYTES, &tm_k, bar(B_KFULL + st), c * 64, w.h, kv0, w.b, pol_kv);
+            else
+              tma_load_4d(kdst + c * C::CHUNK_BYTES, &tm_k, bar(B_KFULL + st), c * 64, kv0, w.h, w.b, pol_kv);
+          }
+          k_pend[st] = true; k_issued[st] = kv_phase;
+          if (!mbar_wait(bar(B_VEMPTY + st), kv_phase ^ 1, wctx)) { ok = false; break; }
+          mbar_arrive_expect_tx(bar(B_VFULL + st), C::TILE_BYTES);
+          const uint32_t vdst = sbase + C::OFF_V + st * C::TILE_BYTES;
+          for (int c = 0; c < C::CHUNKS; ++c) {
+            if (p.bsnd)
+              tma_load_4d(vdst + c * C::CHUNK_BYTES, &tm_v, bar(B_VFULL + st), c * 64, w.h, kv0, w.b, pol_kv);
+            else
+              tma_load_4d(vdst + c * C::CHUNK_BYTES, &tm_v, bar(B_VFULL + st), c * 64, kv0, w.h, w.b, pol_kv);
+          }
+          v_pend[st] = true; v_issued[st] = kv_phase;
+          if (++st == C::KST) { st = 0; kv_phase ^= 1; }
+        }
+      }
+      // Every copy this thread started lands before the CTA may exit (their
+      // barriers complete on their own; the waits are bounded regardless).
+      WaitCtx drain{abort_flag, status_word, p.timeout_ns, 1u};
+      volatile int no_abort = 0;
+      drain.abort_flag = &no_abort;
+      for (int s = 0; s < C::KST; ++s) {
+        if (k_pend[s]) mbar_wait(bar(B_KFULL + s), k_issued[s], drain);
+        if (v_pend[s]) mbar_wait(bar(B_VFULL + s), v_issued[s], drain);
+      }
+      for (int i = 0; i < 2; ++i)
+        if (q_pend[i]) mbar_wait(bar(B_QFULL + i), q_issued[i], drain);
+    }
+    __syncwarp();
+  } else if (warp == 8) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t IDESC_S = idesc_f16(IS_BF16, false, 128, 128);
+      constexpr uint32_t IDESC_PV = idesc_f16(IS_BF16, true, 128, D);
+      uint32_t q_phase[2] = {0, 0}, kv_phase = 0, p_phase[2] = {0, 0};
+      int st = 0;
+      bool ok = true;
+      const uint32_t tS[2] = {tmem + C::TMEM_S0, tmem + C::TMEM_S1};
+      const uint32_t tO[2] = {tmem + C::TMEM_O0, tmem + C::TMEM_O1};
+      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+        const Unit w = decode_unit(u, p);
+        const int n[2] = {w.n0, w.n1};
+        const int N = w.n0 > w.n1 ? w.n0 : w.n1;
+        for (int i = 0; i < 2 && ok; ++i) {
+          if (n[i] == 0) continue;
+          if (!mbar_wait(bar(B_QFULL + i), q_phase[i], wctx)) ok = false;
+          q_phase[i] ^= 1;
+        }
+        int st_prev = 0;
+        uint32_t ph_prev = 0;
+        for (int j = 0; j <= N && ok; ++j) {
+          if (j < N && !mbar_wait(bar(B_KFULL + st), kv_phase, wctx)) { ok = false; break; }
+          if (j > 0 && !mbar_wait(bar(B_VFULL + st_prev), ph_prev, wctx)) { ok = false; break; }
+          tc_fence_after();
+          for (int i = 0; i < 2 && ok; ++i) {
+            if (n[i] == 0) continue;
+            if (j >= 1 && j - 1 < n[i]) {
+              // O_i += P_i(j-1) V_(j-1)
+              if (!mbar_wait(bar(B_PFULL + i), p_phase[i], wctx)) { ok = false; break; }
+              p_phase[i] ^= 1;
+              tc_fence_after();
+              const uint32_t vb = sbase + C::OFF_V + st_prev * C::TILE_BYTES;
+#pragma unroll
+              for (int kk = 0; kk < TC_BN / 16; ++kk) {
+                const uint64_t bdesc = smem_desc_sw128(vb + kk * 16 * 128, C::CHUNK_BYTES, 1024);
+                mma_ts(tO[i], tS[i] + kk * 8, bdesc, IDESC_PV, (j - 1 > 0 || kk > 0) ? 1u : 0u);
+              }
+              if (j - 1 == n[i] - 1) mma_commit(bar(B_OFULL + i));
+            }
+            if (j < n[i]) {
+              // S_i(j) = Q_i K_j^T
+              const uint32_t qb = sbase + C::OFF_Q + i * C::TILE_BYTES;
+              const uint32_t kb = sbase + C::OFF_K + st * C::TILE_BYTES;
+#pragma unroll
+              for (int k = 0; k < D / 16; ++k) {
+                const uint32_t off = (k >> 2) * C::CHUNK_BYTES + (k & 3) * 32;
+                const uint64_t adesc = smem_desc_sw128(qb + off, 16, 1024);
+                const uint64_t bdesc = smem_desc_sw128(kb + off, 16, 1024);
+                mma_ss(tS[i], adesc, bdesc, IDESC_S, k > 0 ? 1u : 0u);
+              }
+              mma_commit(bar(B_SFULL + i));
+              if (j == n[i] - 1) mma_commit(bar(B_QEMPTY + i));
+            }
+          }
+          if (!ok) break;
+          if (j < N) mma_commit(bar(B_KEMPTY + st));
+          if (j > 0) mma_commit(bar(B_VEMPTY + st_prev));
+          st_prev = st;
+          ph_prev = kv_phase;
+          if (j < N) {
+            if (++st == C::KST) { st = 0; kv_phase ^= 1; }
+          }
+        }
+      }
+      // Let every MMA this thread issued finish before the CTA frees TMEM.
+      mma_commit(bar(B_DRAIN));
+      WaitCtx drain{abort_flag, status_word, p.timeout_ns, 1u};
+      volatile int no_abort = 0;
+      drain.abort_flag = &no_abort;
+      mbar_wait(bar(B_DRAIN), 0, drain);
+    }
+    __syncwarp();
+  } else {
+    // ------------------------------------------------------------ softmax + epilogue
+    const int tile = warp >> 2;             // 0: warps 0-3, 1: warps 4-7
+    const int r = (warp & 3) * 32 + lane;   // query row within the Q tile == TMEM lane
+    const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
+    const uint32_t tS = tmem + lane_base + (tile ? C::TMEM_S1 : C::TMEM_S0);
+    const uint32_t tO = tmem + lane_base + (tile ? C::TMEM_O1 : C::TMEM_O0);
+    const float sl2 = p.scale_log2;
+    uint32_t s_phase = 0, o_phase = 0;
+    bool ok = true;
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+      const Unit w = decode_unit(u, p);
+      const int n = tile ? w.n1 : w.n0;
+      if (n == 0) continue;
+      const int qt = w.qt0 + tile;
+      const int row = qt * TC_BM + r;
+      float m_ref = -INFINITY;  // running reference max (log2 domain)
+      float l = 0.f;
+      for (int j = 0; j < n; ++j) {
+        ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SFULL + tile), s_phase, wctx));
+        if (!ok) break;
+        s_phase ^= 1;
+        tc_fence_after();
+        float s[128];
+        tmem_ld128(tS, s);
+        const int col0 = j * TC_BN;
+        const bool need_mask = (col0 + TC_BN > p.Nkv) || (p.causal && col0 + TC_BN - 1 > qt * TC_BM);
+        if (need_mask) {
+          const int lim_c = p.causal ? (row + 1 < p.Nkv ? row + 1 : p.Nkv) : p.Nkv;
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (col0 + c >= lim_c) s[c] = -INFINITY;
+        }
+        float mx[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) mx[t] = s[t];
+#pragma unroll
+        for (int c = 8; c < 128; c += 8)
+#pragma unroll
+          for (int t = 0; t < 8; ++t) mx[t] = fmaxf(mx[t], s[c + t]);
+        float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                         fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+        mt *= sl2;
+        float corr = 1.f;
+        bool moved = false;
+        if (mt > m_ref + TC_RESCALE_THRESHOLD) {
+          corr = ex2(m_ref - mt);  // 0 when m_ref = -inf
+          m_ref = mt;
+          moved = true;
+        }
+        const float mref_use = (m_ref == -INFINITY) ? 0.f : m_ref;
+        float sum[8];
+#pragma unroll
+        for (int t = 0; t < 8; ++t) sum[t] = 0.f;
+        uint32_t pk[64];
+#pragma unroll
+        for (int c = 0; c < 128; c += 2) {
+          const float p0 = ex2(fmaf(s[c], sl2, -mref_use));
+          const float p1 = ex2(fmaf(s[c + 1], sl2, -mref_use));
+          sum[(c >> 1) & 7] += p0 + p1;
+          pk[c >> 1] = Pack<T>::two(p0, p1);
+        }
+        l = l * corr + (((sum[0] + sum[1]) + (sum[2] + sum[3])) + ((sum[4] + sum[5]) + (sum[6] + sum[7])));
+        tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+        tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+        // Rescale O in place when this warp moved any row's reference max
+        // (O is quiescent: its last P V finished before S_i(j) was signalled).
+        if (j > 0 && __any_sync(0xffffffffu, moved)) {
+#pragma unroll 1
+          for (int c = 0; c < D; c += 32) {
+            float ov[32];
+            tmem_ld32(tO + c, ov);
+            uint32_t ow[32];
+#pragma unroll
+            for (int t = 0; t < 32; ++t) ow[t] = __float_as_uint(ov[t] * corr);
+            tmem_st32(tO + c, ow);
+          }
+        }
+        tmem_wait_st();
+        tc_fence_before();
+        if (p.fault_mode != 1) mbar_arrive(bar(B_PFULL + tile));
+      }
+      if (!ok) break;
+      // ---------------------------------------------------------- epilogue
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OFULL + tile), o_phase, wctx));
+      if (!ok) break;
+      o_phase ^= 1;
+      tc_fence_after();
+      const float inv_l = 1.f / l;
+      const bool valid = row < p.Nq;
+      T* orow = nullptr;
+      if (valid) {
+        const long long ridx = p.bsnd ? ((long long)w.b * p.Nq + row) * p.H + w.h
+                                      : ((long long)w.b * p.H + w.h) * p.Nq + row;
+        orow = reinterpret_cast<T*>(p.o) + ridx * D;
+      }
+#pragma unroll 1
+      for (int c = 0; c < D; c += 32) {
+        float ov[32];
+        tmem_ld32(tO + c, ov);
+        if (valid) {
+          uint4* dst = reinterpret_cast<uint4*>(orow + c);
+#pragma unroll
+          for (int q4 = 0; q4 < 4; ++q4) {
+            uint4 pkt;
+            pkt.x = Pack<T>::two(ov[q4 * 8 + 0] * inv_l, ov[q4 * 8 + 1] * inv_l);
+            pkt.y = Pack<T>::two(ov[q4 * 8 + 2] * inv_l, ov[q4 * 8 + 3] * inv_l);
+            pkt.z = Pack<T>::two(ov[q4 * 8 + 4] * inv_l, ov[q4 * 8 + 5] * inv_l);
+            pkt.w = Pack<T>::two(ov[q4 * 8 + 6] * inv_l, ov[q4 * 8 + 7] * inv_l);
+            dst[q4] = pkt;
+          }
+        }
+      }
+      if (valid && p.lse != nullptr) {
+        p.lse[((long long)w.b * p.H + w.h) * p.Nq + row] = (m_ref + __log2f(l)) * 0.69314718055994530942f;
+      }
+    }
+    // Any tcgen05.st of this thread has completed before the CTA frees TMEM.
+    tmem_wait_st();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 8) tmem_dealloc(tmem, C::TMEM_COLS);
+}
+
+}  // namespace fa

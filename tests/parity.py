@@ -16,7 +16,7 @@ import numpy as np
 import torch
 
 from oracle import attention_batched, attention_rows, resolve_scale
-from tiled_attention_13_b200 import forward
+from tiled_attention_13_b200 import fa_get_device_status, forward
 from tiled_attention_13_b200.inputs import Workload, make_qkv
 
 O_TOL = 1e-2
@@ -47,6 +47,8 @@ def o_bar(o_ref: np.ndarray, dtype: str) -> np.ndarray:
 def run_gpu(wl: Workload, q, k, v, scale=None):
     o, lse = forward(q, k, v, causal=wl.causal, scale=scale, layout=wl.layout)
     torch.cuda.synchronize()
+    rc = fa_get_device_status(None)
+    assert rc == 0, f"device status {rc}: a bounded wait expired"
     return o, lse
 
 

@@ -234,4 +234,15 @@ int fa_debug_set_fault(int mode) { return g_fault_mode.exchange(mode); }
 
 int fa_abi_version(void) { return (1 << 16) | 0; }
 
+#ifdef FA_TRACE
+int fa_debug_trace_read(unsigned long long* host, int n) {
+  const int total = fa::TRACE_STREAMS * fa::TRACE_J * fa::TRACE_EV;
+  if (n > total) n = total;
+  if (cudaMemcpyFromSymbol(host, fa::g_trace, n * sizeof(unsigned long long)) != cudaSuccess) return FA_ERR_LAUNCH;
+  static unsigned long long zeros[fa::TRACE_STREAMS * fa::TRACE_J * fa::TRACE_EV];
+  cudaMemcpyToSymbol(fa::g_trace, zeros, sizeof(zeros));
+  return n;
+}
+#endif
+
 }  // extern "C"

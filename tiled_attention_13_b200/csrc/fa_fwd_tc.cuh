@@ -12,22 +12,30 @@
 //   work unit   one (batch, head, pair of 128-row Q tiles); a persistent grid
 //               of <= #SM CTAs walks the units in a static strided order,
 //               heaviest causal pairs first (longest-processing-time order).
-//   warps 0-3   softmax warpgroup for Q tile 0 of the pair (one thread per
-//               query row = one TMEM lane), then its epilogue
-//   warps 4-7   softmax warpgroup for Q tile 1
-//   warp 8      TMEM allocator and the single MMA-issuing thread
-//   warp 9      TMA producer (Q tiles, K/V ring of KST stages)
+//   warps 0-15  four softmax warpgroups: (tile 0, keys 0-63), (tile 0, keys
+//               64-127), (tile 1, keys 0-63), (tile 1, keys 64-127).  A thread
+//               owns one query row (= one TMEM lane) and half of its 128 scores
+//               per KV tile; the two halves swap row maxima through shared
+//               memory each step.  Each warpgroup also writes its half of O.
+//   warp 16     TMEM allocator and the MMA issuer (whole warp, elect.sync)
+//   warp 17     TMA producer (Q tiles, K/V ring of KST stages)
 //
 //   TMEM (512 columns x 128 lanes, fp32):  S0 [0,128)  S1 [128,256)
-//   O0 [256, 256+D)  O1 [256+D, 256+2D).  P_i (bf16/fp16 pairs) overwrites
-//   the first 64 columns of S_i once the softmax has read S_i.
+//   O0 [256, 256+D)  O1 [256+D, 256+2D).  P_i (bf16/fp16 pairs) for keys
+//   0-63 overwrites S_i columns [0,32), for keys 64-127 columns [64,96): each
+//   half writes only columns it has already read.
 //
 //   MMA order per KV step j (tile i = 0, 1):  O_i += P_i(j-1) V_(j-1), then
 //   S_i(j) = Q_i K_j^T, then commit -> s_full[i].  The tensor pipe executes
 //   a CTA's MMAs in issue order, so S_i(j) overwrites P_i(j-1) only after
 //   the P V product has read it, and when s_full[i] fires O_i is quiescent
-//   (the softmax may rescale it in place).  While the softmax of tile 0 runs,
-//   the tensor pipe works on tile 1 and vice versa.
+//   (the softmax may rescale it in place).
+//
+//   Special-function-unit turns: the exp phases of tile 0 and tile 1
+//   alternate (tile 0 step j, tile 1 step j, tile 0 step j+1, ...), so the
+//   SFU serves one tile at a time with two warps per SM sub-partition, and
+//   each tile's exps overlap the other tile's MMAs.  On tiles without masked
+//   scores one exp pair in TC_POLY_EVERY is computed on the FMA pipe.
 //
 //   Online softmax in the exp2 domain: x = s * scale * log2(e).  The running
 //   reference max m is only moved when a tile's max exceeds it by more than
@@ -40,14 +48,41 @@
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
+#include <type_traits>
+
 #include "ptx.cuh"
 
 namespace fa {
 
-constexpr int TC_THREADS = 320;  // 10 warps
-constexpr int TC_BM = 128;       // query rows per Q tile
-constexpr int TC_BN = 128;       // keys per KV tile
+// Optional timeline instrumentation (compile with -DFA_TRACE): SM-clock
+// stamps of each role's phases for the first work unit of CTA 0, readable
+// through fa_debug_trace_read().  Compiles to nothing otherwise.
+#ifdef FA_TRACE
+// [stream][j][event]: streams 0-15 = softmax warps, 16-17 = MMA for tile 0/1
+constexpr int TRACE_J = 64, TRACE_EV = 8, TRACE_STREAMS = 18;
+__device__ unsigned long long g_trace[TRACE_STREAMS * TRACE_J * TRACE_EV];
+#define FA_TR(cond, stream, j, ev)                                                           \
+  do {                                                                                       \
+    if ((cond) && blockIdx.x == 0 && (j) < TRACE_J)                                          \
+      g_trace[((stream) * TRACE_J + (j)) * TRACE_EV + (ev)] = (unsigned long long)clock64(); \
+  } while (0)
+#else
+#define FA_TR(cond, tile, j, ev) \
+  do {                           \
+  } while (0)
+#endif
+
+constexpr int TC_SOFTMAX_WARPS = 16;
+constexpr int WARP_MMA = 16;
+constexpr int WARP_TMA = 17;
+constexpr int TC_THREADS = 32 * 18;
+constexpr int TC_BM = 128;                    // query rows per Q tile
+constexpr int TC_BN = 128;                    // keys per KV tile
 constexpr float TC_RESCALE_THRESHOLD = 8.0f;  // log2 units
+#ifndef FA_POLY_EVERY
+#define FA_POLY_EVERY 4
+#endif
+constexpr int TC_POLY_EVERY = FA_POLY_EVERY;  // one exp pair in TC_POLY_EVERY on the FMA pipe
 
 template <int D>
 struct TcCfg {
@@ -58,8 +93,10 @@ struct TcCfg {
   static constexpr int OFF_Q = 0;                           // Q0, Q1
   static constexpr int OFF_K = 2 * TILE_BYTES;              // KST K tiles
   static constexpr int OFF_V = OFF_K + KST * TILE_BYTES;    // KST V tiles
-  static constexpr int OFF_BAR = OFF_V + KST * TILE_BYTES;  // barriers
-  static constexpr int NBAR = 2 + 2 + 4 * KST + 2 + 2 + 2 + 1;
+  static constexpr int OFF_RED = OFF_V + KST * TILE_BYTES;  // [tile][parity][half][row] fp32 exchange
+  static constexpr int RED_BYTES = 2 * 2 * 2 * TC_BM * 4;
+  static constexpr int OFF_BAR = OFF_RED + RED_BYTES;       // barriers
+  static constexpr int NBAR = 2 + 2 + 4 * KST + 2 + 2 + 2 + 1 + 2 + 2;
   static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 /*tmem slot + abort*/ + 1024 /*align slack*/;
   static constexpr int TMEM_S0 = 0, TMEM_S1 = 128, TMEM_O0 = 256, TMEM_O1 = 256 + D;
   static constexpr uint32_t TMEM_COLS = 512;
@@ -137,10 +174,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   const uint32_t sbase = smem_u32(smem);
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
+  float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
   // barrier indices
   const int B_QFULL = 0, B_QEMPTY = 2, B_KFULL = 4, B_KEMPTY = 4 + C::KST, B_VFULL = 4 + 2 * C::KST,
             B_VEMPTY = 4 + 3 * C::KST, B_SFULL = 4 + 4 * C::KST, B_PFULL = B_SFULL + 2, B_OFULL = B_PFULL + 2,
-            B_DRAIN = B_OFULL + 2;
+            B_DRAIN = B_OFULL + 2, B_TURN0 = B_DRAIN + 1, B_TURN1 = B_DRAIN + 2, B_XCHG = B_DRAIN + 3;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
@@ -153,8 +191,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       mbar_init(bar(B_QFULL + i), 1);
       mbar_init(bar(B_QEMPTY + i), 1);
       mbar_init(bar(B_SFULL + i), 1);
-      mbar_init(bar(B_PFULL + i), 128);
+      mbar_init(bar(B_PFULL + i), 8);  // one arrival per softmax warp of the tile
       mbar_init(bar(B_OFULL + i), 1);
+      mbar_init(bar(B_XCHG + i), 8);
     }
     for (int s = 0; s < C::KST; ++s) {
       mbar_init(bar(B_KFULL + s), 1);
@@ -163,14 +202,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       mbar_init(bar(B_VEMPTY + s), 1);
     }
     mbar_init(bar(B_DRAIN), 1);
+    mbar_init(bar(B_TURN0), 8);
+    mbar_init(bar(B_TURN1), 8);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (warp == 8) {
+  if (warp == WARP_MMA) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
-  if (warp == 9 && lane == 0) {
+  if (warp == WARP_TMA && lane == 0) {
     prefetch_tmap(&tm_q);
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
@@ -183,7 +224,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
   WaitCtx wctx{abort_flag, status_word, p.timeout_ns, 1u};
 
-  if (warp == 9) {
+  if (warp == WARP_TMA) {
     // ------------------------------------------------------------ TMA producer
     if (lane == 0) {
       const uint64_t pol_q = l2_policy_evict_first();
@@ -253,122 +294,160 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (q_pend[i]) mbar_wait(bar(B_QFULL + i), q_issued[i], drain);
     }
     __syncwarp();
-  } else if (warp == 8) {
+  } else if (warp == WARP_MMA) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t IDESC_S = idesc_f16(IS_BF16, false, 128, 128);
-      constexpr uint32_t IDESC_PV = idesc_f16(IS_BF16, true, 128, D);
-      uint32_t q_phase[2] = {0, 0}, kv_phase = 0, p_phase[2] = {0, 0};
-      int st = 0;
-      bool ok = true;
-      const uint32_t tS[2] = {tmem + C::TMEM_S0, tmem + C::TMEM_S1};
-      const uint32_t tO[2] = {tmem + C::TMEM_O0, tmem + C::TMEM_O1};
-      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-        const Unit w = decode_unit(u, p);
-        const int n[2] = {w.n0, w.n1};
-        const int N = w.n0 > w.n1 ? w.n0 : w.n1;
+    // The whole warp runs this role (warp-uniform control flow, descriptors in
+    // uniform registers); elect.sync picks the one lane that issues each
+    // tcgen05 instruction.  Only the start-address field of a descriptor
+    // changes between MMAs, by compile-time offsets.
+    constexpr uint32_t IDESC_S = idesc_f16(IS_BF16, false, 128, 128);
+    constexpr uint32_t IDESC_PV = idesc_f16(IS_BF16, true, 128, D);
+    const uint64_t dQ[2] = {smem_desc_sw128(sbase + C::OFF_Q, 16, 1024),
+                            smem_desc_sw128(sbase + C::OFF_Q + C::TILE_BYTES, 16, 1024)};
+    const uint64_t dK0 = smem_desc_sw128(sbase + C::OFF_K, 16, 1024);
+    const uint64_t dV0 = smem_desc_sw128(sbase + C::OFF_V, C::CHUNK_BYTES, 1024);
+    uint32_t q_phase[2] = {0, 0}, kv_phase = 0, p_phase[2] = {0, 0};
+    int st = 0;
+    bool ok = true;
+    const uint32_t tS[2] = {tmem + C::TMEM_S0, tmem + C::TMEM_S1};
+    const uint32_t tO[2] = {tmem + C::TMEM_O0, tmem + C::TMEM_O1};
+    auto wait_all = [&](int b, uint32_t ph) { return __all_sync(0xffffffffu, mbar_wait(bar(b), ph, wctx)); };
+    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
+      const Unit w = decode_unit(u, p);
+      const int n[2] = {w.n0, w.n1};
+      const int N = w.n0 > w.n1 ? w.n0 : w.n1;
+      for (int i = 0; i < 2 && ok; ++i) {
+        if (n[i] == 0) continue;
+        if (!wait_all(B_QFULL + i, q_phase[i])) ok = false;
+        q_phase[i] ^= 1;
+      }
+      int st_prev = 0;
+      uint32_t ph_prev = 0;
+      for (int j = 0; j <= N && ok; ++j) {
+        if (j < N && !wait_all(B_KFULL + st, kv_phase)) { ok = false; break; }
+        FA_TR(lane == 0 && u == (int)blockIdx.x, 16, j, 0);
+        if (j > 0 && !wait_all(B_VFULL + st_prev, ph_prev)) { ok = false; break; }
+        tc_fence_after();
+        const uint64_t dK = dK0 + (uint64_t)((st * C::TILE_BYTES) >> 4);
+        const uint64_t dV = dV0 + (uint64_t)((st_prev * C::TILE_BYTES) >> 4);
         for (int i = 0; i < 2 && ok; ++i) {
           if (n[i] == 0) continue;
-          if (!mbar_wait(bar(B_QFULL + i), q_phase[i], wctx)) ok = false;
-          q_phase[i] ^= 1;
+          if (j >= 1 && j - 1 < n[i]) {
+            // O_i += P_i(j-1) V_(j-1)
+            if (!wait_all(B_PFULL + i, p_phase[i])) { ok = false; break; }
+            FA_TR(lane == 0 && u == (int)blockIdx.x, 16 + i, j - 1, 1);
+            p_phase[i] ^= 1;
+            tc_fence_after();
+            const uint32_t acc0 = (j - 1 > 0) ? 1u : 0u;
+#pragma unroll
+            for (int kk = 0; kk < TC_BN / 16; ++kk)
+              mma_ts_elect(tO[i], tS[i] + (kk >> 2) * 64 + (kk & 3) * 8, dV + (uint64_t)((kk * 16 * 128) >> 4),
+                           IDESC_PV, kk > 0 ? 1u : acc0);
+            if (j - 1 == n[i] - 1) mma_commit_elect(bar(B_OFULL + i));
+          }
+          if (j < n[i]) {
+            // S_i(j) = Q_i K_j^T
+#pragma unroll
+            for (int k = 0; k < D / 16; ++k) {
+              const uint64_t off = (uint64_t)((((k >> 2) * C::CHUNK_BYTES) + (k & 3) * 32) >> 4);
+              mma_ss_elect(tS[i], dQ[i] + off, dK + off, IDESC_S, k > 0 ? 1u : 0u);
+            }
+            mma_commit_elect(bar(B_SFULL + i));
+            FA_TR(lane == 0 && u == (int)blockIdx.x, 16 + i, j, 2);
+            if (j == n[i] - 1) mma_commit_elect(bar(B_QEMPTY + i));
+          }
         }
-        int st_prev = 0;
-        uint32_t ph_prev = 0;
-        for (int j = 0; j <= N && ok; ++j) {
-          if (j < N && !mbar_wait(bar(B_KFULL + st), kv_phase, wctx)) { ok = false; break; }
-          if (j > 0 && !mbar_wait(bar(B_VFULL + st_prev), ph_prev, wctx)) { ok = false; break; }
-          tc_fence_after();
-          for (int i = 0; i < 2 && ok; ++i) {
-            if (n[i] == 0) continue;
-            if (j >= 1 && j - 1 < n[i]) {
-              // O_i += P_i(j-1) V_(j-1)
-              if (!mbar_wait(bar(B_PFULL + i), p_phase[i], wctx)) { ok = false; break; }
-              p_phase[i] ^= 1;
-              tc_fence_after();
-              const uint32_t vb = sbase + C::OFF_V + st_prev * C::TILE_BYTES;
-#pragma unroll
-              for (int kk = 0; kk < TC_BN / 16; ++kk) {
-                const uint64_t bdesc = smem_desc_sw128(vb + kk * 16 * 128, C::CHUNK_BYTES, 1024);
-                mma_ts(tO[i], tS[i] + kk * 8, bdesc, IDESC_PV, (j - 1 > 0 || kk > 0) ? 1u : 0u);
-              }
-              if (j - 1 == n[i] - 1) mma_commit(bar(B_OFULL + i));
-            }
-            if (j < n[i]) {
-              // S_i(j) = Q_i K_j^T
-              const uint32_t qb = sbase + C::OFF_Q + i * C::TILE_BYTES;
-              const uint32_t kb = sbase + C::OFF_K + st * C::TILE_BYTES;
-#pragma unroll
-              for (int k = 0; k < D / 16; ++k) {
-                const uint32_t off = (k >> 2) * C::CHUNK_BYTES + (k & 3) * 32;
-                const uint64_t adesc = smem_desc_sw128(qb + off, 16, 1024);
-                const uint64_t bdesc = smem_desc_sw128(kb + off, 16, 1024);
-                mma_ss(tS[i], adesc, bdesc, IDESC_S, k > 0 ? 1u : 0u);
-              }
-              mma_commit(bar(B_SFULL + i));
-              if (j == n[i] - 1) mma_commit(bar(B_QEMPTY + i));
-            }
-          }
-          if (!ok) break;
-          if (j < N) mma_commit(bar(B_KEMPTY + st));
-          if (j > 0) mma_commit(bar(B_VEMPTY + st_prev));
-          st_prev = st;
-          ph_prev = kv_phase;
-          if (j < N) {
-            if (++st == C::KST) { st = 0; kv_phase ^= 1; }
-          }
+        if (!ok) break;
+        if (j < N) mma_commit_elect(bar(B_KEMPTY + st));
+        if (j > 0) mma_commit_elect(bar(B_VEMPTY + st_prev));
+        st_prev = st;
+        ph_prev = kv_phase;
+        if (j < N) {
+          if (++st == C::KST) { st = 0; kv_phase ^= 1; }
         }
       }
-      // Let every MMA this thread issued finish before the CTA frees TMEM.
-      mma_commit(bar(B_DRAIN));
+    }
+    // Let every MMA this warp issued finish before the CTA frees TMEM.
+    mma_commit_elect(bar(B_DRAIN));
+    {
       WaitCtx drain{abort_flag, status_word, p.timeout_ns, 1u};
       volatile int no_abort = 0;
       drain.abort_flag = &no_abort;
       mbar_wait(bar(B_DRAIN), 0, drain);
     }
     __syncwarp();
-  } else {
+  } else if (warp < TC_SOFTMAX_WARPS) {
     // ------------------------------------------------------------ softmax + epilogue
-    const int tile = warp >> 2;             // 0: warps 0-3, 1: warps 4-7
+    const int tile = warp >> 3;             // warps 0-7: tile 0, warps 8-15: tile 1
+    const int half = (warp >> 2) & 1;       // keys [64 half, 64 half + 64) of each KV tile
     const int r = (warp & 3) * 32 + lane;   // query row within the Q tile == TMEM lane
     const uint32_t lane_base = (uint32_t)((warp & 3) * 32) << 16;
-    const uint32_t tS = tmem + lane_base + (tile ? C::TMEM_S1 : C::TMEM_S0);
-    const uint32_t tO = tmem + lane_base + (tile ? C::TMEM_O1 : C::TMEM_O0);
+    const uint32_t tS = tmem + lane_base + (tile ? C::TMEM_S1 : C::TMEM_S0) + 64 * half;
+    const uint32_t tO = tmem + lane_base + (tile ? C::TMEM_O1 : C::TMEM_O0) + (D / 2) * half;
+    float* red_t = red + tile * (2 * 2 * TC_BM);  // [parity][half][row]
     const float sl2 = p.scale_log2;
-    uint32_t s_phase = 0, o_phase = 0;
+    uint32_t s_phase = 0, o_phase = 0, t_phase = 0, x_phase = 0;
     bool ok = true;
+    // Swap one float per row with the other half of this tile (bounded wait).
+    auto exchange = [&](float mine, float& theirs) -> bool {
+      red_t[(x_phase * 2 + half) * TC_BM + r] = mine;
+      mbar_arrive_warp(bar(B_XCHG + tile));
+      const bool got = __all_sync(0xffffffffu, mbar_wait(bar(B_XCHG + tile), x_phase, wctx));
+      if (got) theirs = red_t[(x_phase * 2 + (half ^ 1)) * TC_BM + r];
+      x_phase ^= 1;
+      return got;
+    };
     for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
       const Unit w = decode_unit(u, p);
       const int n = tile ? w.n1 : w.n0;
       if (n == 0) continue;
       const int qt = w.qt0 + tile;
       const int row = qt * TC_BM + r;
-      float m_ref = -INFINITY;  // running reference max (log2 domain)
-      float l = 0.f;
+      const bool first_unit = (u == (int)blockIdx.x);
+      (void)first_unit;
+      float m_ref = -INFINITY;  // running reference max (log2 domain), identical in both halves
+      float l = 0.f;            // this half's share of the row sum
       for (int j = 0; j < n; ++j) {
         ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SFULL + tile), s_phase, wctx));
         if (!ok) break;
+        FA_TR(first_unit && lane == 0, warp, j, 0);
         s_phase ^= 1;
         tc_fence_after();
-        float s[128];
-        tmem_ld128(tS, s);
-        const int col0 = j * TC_BN;
-        const bool need_mask = (col0 + TC_BN > p.Nkv) || (p.causal && col0 + TC_BN - 1 > qt * TC_BM);
-        if (need_mask) {
-          const int lim_c = p.causal ? (row + 1 < p.Nkv ? row + 1 : p.Nkv) : p.Nkv;
+        const int col0 = j * TC_BN + 64 * half;
+        const bool need_mask = (j * TC_BN + TC_BN > p.Nkv) || (p.causal && j * TC_BN + TC_BN - 1 > qt * TC_BM);
+        // visible columns of this row: [.., lim_c)
+        const int lim_c = p.causal ? (row + 1 < p.Nkv ? row + 1 : p.Nkv) : p.Nkv;
+        float mt;
+        {
+          // pass 1: this half's row max
+          float s[64];
+          tmem_ld64(tS, s);
+          FA_TR(first_unit && lane == 0, warp, j, 1);
+          if (need_mask) {
 #pragma unroll
-          for (int c = 0; c < 128; ++c)
-            if (col0 + c >= lim_c) s[c] = -INFINITY;
+            for (int c = 0; c < 64; ++c)
+              if (col0 + c >= lim_c) s[c] = -INFINITY;
+          }
+          float mx[4];
+#pragma unroll
+          for (int t = 0; t < 4; ++t) mx[t] = fmaxf(s[t], s[t + 4]);
+#pragma unroll
+          for (int c = 8; c < 64; c += 8)
+#pragma unroll
+            for (int t = 0; t < 4; ++t) mx[t] = fmax3(mx[t], s[c + t], s[c + 4 + t]);
+          mt = fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3]));
         }
-        float mx[8];
-#pragma unroll
-        for (int t = 0; t < 8; ++t) mx[t] = s[t];
-#pragma unroll
-        for (int c = 8; c < 128; c += 8)
-#pragma unroll
-          for (int t = 0; t < 8; ++t) mx[t] = fmaxf(mx[t], s[c + t]);
-        float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                         fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
-        mt *= sl2;
+        // pass 2 re-reads the scores (tensor-memory reads are cheap, registers
+        // are not); the first 32 columns are already in flight during the
+        // row-max exchange and the SFU turn wait.
+        float sa[32], sb[32];
+        tmem_ld32_issue(tS, sa);
+        FA_TR(first_unit && lane == 0, warp, j, 2);
+        float other = -INFINITY;
+        ok = exchange(mt, other);
+        if (!ok) break;
+        FA_TR(first_unit && lane == 0, warp, j, 3);
+        mt = fmaxf(mt, other) * sl2;
         float corr = 1.f;
         bool moved = false;
         if (mt > m_ref + TC_RESCALE_THRESHOLD) {
@@ -377,25 +456,84 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           moved = true;
         }
         const float mref_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-        float sum[8];
-#pragma unroll
-        for (int t = 0; t < 8; ++t) sum[t] = 0.f;
-        uint32_t pk[64];
-#pragma unroll
-        for (int c = 0; c < 128; c += 2) {
-          const float p0 = ex2(fmaf(s[c], sl2, -mref_use));
-          const float p1 = ex2(fmaf(s[c + 1], sl2, -mref_use));
-          sum[(c >> 1) & 7] += p0 + p1;
-          pk[c >> 1] = Pack<T>::two(p0, p1);
+        // SFU turn: tile 0 step j, tile 1 step j, tile 0 step j + 1, ...
+        if (tile == 0) {
+          if (j >= 1 && w.active1) {
+            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_TURN0), t_phase, wctx));
+            t_phase ^= 1;
+          }
+        } else if (j < w.n0) {
+          ok = __all_sync(0xffffffffu, mbar_wait(bar(B_TURN1), t_phase, wctx));
+          t_phase ^= 1;
         }
-        l = l * corr + (((sum[0] + sum[1]) + (sum[2] + sum[3])) + ((sum[4] + sum[5]) + (sum[6] + sum[7])));
-        tmem_st32(tS, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
-        tmem_st32(tS + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
-        // Rescale O in place when this warp moved any row's reference max
-        // (O is quiescent: its last P V finished before S_i(j) was signalled).
+        if (!ok) break;
+        FA_TR(first_unit && lane == 0, warp, j, 4);
+        const uint64_t scale2 = f2_pack(sl2, sl2);
+        const uint64_t negm2 = f2_pack(-mref_use, -mref_use);
+        uint64_t acc2[2] = {0ull, 0ull};
+        // 16 scores -> 8 packed P columns, written over this half's first 32
+        // S columns (already read).  On tiles without masked scores one pair
+        // in TC_POLY_EVERY takes 2^x on the FMA pipe.
+        auto exp_chunks = [&](auto use_poly) {
+          auto sub = [&](const float* sc, int cbase) {
+            uint32_t pk[8];
+#pragma unroll
+            for (int t = 0; t < 8; ++t) {
+              const uint64_t x2 = f2_fma(f2_pack(sc[2 * t], sc[2 * t + 1]), scale2, negm2);
+              float p0, p1;
+              if (decltype(use_poly)::value && (t % TC_POLY_EVERY) == TC_POLY_EVERY - 1) {
+                exp2_poly_x2(x2, p0, p1);
+              } else {
+                float x0, x1;
+                f2_unpack(x2, x0, x1);
+                p0 = ex2(x0);
+                p1 = ex2(x1);
+              }
+              acc2[t & 1] = f2_add(acc2[t & 1], f2_pack(p0, p1));
+              pk[t] = Pack<T>::two(p0, p1);
+            }
+            tmem_st8(tS + cbase / 2, pk);
+          };
+          auto mask32 = [&](float(&sc)[32], int cbase) {
+            if (!decltype(use_poly)::value && need_mask) {
+#pragma unroll
+              for (int c = 0; c < 32; ++c)
+                if (col0 + cbase + c >= lim_c) sc[c] = -INFINITY;
+            }
+          };
+          tmem_ld_wait32(sa);
+          mask32(sa, 0);
+          sub(sa, 0);
+          tmem_ld32_issue(tS + 32, sb);  // columns 32-63 load while 16-31 are processed
+          sub(sa + 16, 16);
+          tmem_ld_wait32(sb);
+          mask32(sb, 32);
+          sub(sb, 32);
+          sub(sb + 16, 48);
+        };
+        if (need_mask)
+          exp_chunks(std::false_type{});
+        else
+          exp_chunks(std::true_type{});
+        FA_TR(first_unit && lane == 0, warp, j, 5);
+        if (tile == 0) {
+          if (w.active1) mbar_arrive_warp(bar(B_TURN1));
+        } else if (j + 1 < w.n0) {
+          mbar_arrive_warp(bar(B_TURN0));
+        }
+        float sum;
+        {
+          float a0, a1;
+          f2_unpack(f2_add(acc2[0], acc2[1]), a0, a1);
+          sum = a0 + a1;
+        }
+        l = l * corr + sum;
+        // Rescale this half of O in place when this warp moved any row's
+        // reference max (O is quiescent: its last P V finished before S_i(j)
+        // was signalled).
         if (j > 0 && __any_sync(0xffffffffu, moved)) {
 #pragma unroll 1
-          for (int c = 0; c < D; c += 32) {
+          for (int c = 0; c < D / 2; c += 32) {
             float ov[32];
             tmem_ld32(tO + c, ov);
             uint32_t ow[32];
@@ -406,10 +544,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         tmem_wait_st();
         tc_fence_before();
-        if (p.fault_mode != 1) mbar_arrive(bar(B_PFULL + tile));
+        if (p.fault_mode != 1) mbar_arrive_warp(bar(B_PFULL + tile));
+        FA_TR(first_unit && lane == 0, warp, j, 6);
       }
       if (!ok) break;
       // ---------------------------------------------------------- epilogue
+      float l_other = 0.f;
+      ok = exchange(l, l_other);
+      if (!ok) break;
+      l += l_other;
       ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OFULL + tile), o_phase, wctx));
       if (!ok) break;
       o_phase ^= 1;
@@ -420,10 +563,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       if (valid) {
         const long long ridx = p.bsnd ? ((long long)w.b * p.Nq + row) * p.H + w.h
                                       : ((long long)w.b * p.H + w.h) * p.Nq + row;
-        orow = reinterpret_cast<T*>(p.o) + ridx * D;
+        orow = reinterpret_cast<T*>(p.o) + ridx * D + (D / 2) * half;
       }
 #pragma unroll 1
-      for (int c = 0; c < D; c += 32) {
+      for (int c = 0; c < D / 2; c += 32) {
         float ov[32];
         tmem_ld32(tO + c, ov);
         if (valid) {
@@ -439,7 +582,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           }
         }
       }
-      if (valid && p.lse != nullptr) {
+      if (valid && half == 0 && p.lse != nullptr) {
         p.lse[((long long)w.b * p.H + w.h) * p.Nq + row] = (m_ref + __log2f(l)) * 0.69314718055994530942f;
       }
     }
@@ -450,7 +593,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 8) tmem_dealloc(tmem, C::TMEM_COLS);
+  if (warp == WARP_MMA) tmem_dealloc(tmem, C::TMEM_COLS);
 }
 
 }  // namespace fa

@@ -45,6 +45,18 @@ def load_peaks():
     return FALLBACK_PEAKS, "fallback"
 
 
+def max_over_ranks(x: float, device=None) -> float:
+    """Max of a per-rank float over all ranks (identity without a process group)."""
+    import torch
+    import torch.distributed as dist
+
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device if device is not None else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -260,10 +272,7 @@ def run_ours(args, wl):
     if rc != 0:
         raise RuntimeError(f"device status after timing: {fa.fa_status_string(rc)}")
 
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if ws > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    ms_step = t.item() / args.steps
+    ms_step = max_over_ranks(total_ms, dev) / args.steps
     value = ws * wl.flops / (ms_step * 1e-3) / 1e12
 
     # ---- end-to-end through the public API: pinned host in, host out
@@ -283,12 +292,10 @@ def run_ours(args, wl):
             hf(qh, kh, vh)
         b.record(stream)
         torch.cuda.synchronize()
-        te = torch.tensor([a.elapsed_time(b) / n_e2e], dtype=torch.float64, device=dev)
-        if ws > 1:
-            dist.all_reduce(te, op=dist.ReduceOp.MAX)
-        e2e = {"value": ws * wl.flops / (te.item() * 1e-3) / 1e12, "unit": UNIT,
+        te = max_over_ranks(a.elapsed_time(b) / n_e2e, dev)
+        e2e = {"value": ws * wl.flops / (te * 1e-3) / 1e12, "unit": UNIT,
                "h2d_bytes_per_step": hf.h2d_bytes, "d2h_bytes_per_step": hf.d2h_bytes,
-               "ms_per_step": te.item(), "steps": n_e2e}
+               "ms_per_step": te, "steps": n_e2e}
         del hf, qh, kh, vh
 
     if rank == 0:

@@ -70,10 +70,12 @@ typedef enum {
  *   stream a cudaStream_t (NULL = the legacy default stream)
  *
  * Ownership: every buffer belongs to the caller and must stay alive until the
- * stream has finished the call.  The library keeps no pointer after return and
- * allocates no device memory (its status word is a static device variable).
- * The call is asynchronous: it validates, encodes TMA descriptors on the host
- * and launches one kernel on `stream`.
+ * stream has finished the call.  The library keeps no pointer after return.
+ * On its first call on a device it allocates 8 KB of device memory for the
+ * tile scheduler's per-launch work counters (kept until the process exits;
+ * make that first call outside any stream capture); later calls allocate
+ * nothing.  The call is asynchronous: it validates, encodes TMA descriptors
+ * on the host and launches one kernel on `stream`.
  *
  * Returns FA_OK (also for B*H*Nq == 0, a no-op), or FA_ERR_INVALID_ARG /
  * FA_ERR_UNSUPPORTED / FA_ERR_MISALIGNED before anything is launched, or

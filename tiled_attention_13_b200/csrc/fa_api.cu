@@ -30,11 +30,15 @@ std::atomic<uint32_t> g_timeout_us{kDefaultTimeoutUs};
 std::atomic<int> g_fault_mode{0};
 
 constexpr int kMaxDevices = 64;
+constexpr int kSchedSlots = 1024;  // per-device ring of per-launch ticket counters
+
 struct DeviceInfo {
   bool ready = false;
   bool supported = false;
   int num_sms = 0;
-  unsigned int* status = nullptr;  // device address of fa::g_status_word
+  unsigned int* status = nullptr;      // device address of fa::g_status_word
+  fa::SchedSlot* sched = nullptr;      // kSchedSlots counters, allocated once
+  std::atomic<uint64_t> launches{0};   // picks the counter slot of a launch
 };
 DeviceInfo g_dev[kMaxDevices];
 std::mutex g_dev_mu;
@@ -73,6 +77,16 @@ int device_setup(int dev, DeviceInfo** out) {
       ok &= set_smem_attr(fa::fa_fwd_simt_kernel<64>, fa::simt_smem_bytes<64>());
       ok &= set_smem_attr(fa::fa_fwd_simt_kernel<128>, fa::simt_smem_bytes<128>());
       if (!ok) return FA_ERR_LAUNCH;
+      // The tile scheduler's ticket counters: one slot per launch in flight,
+      // each put back to zero by the last CTA of its launch.
+      void* sp = nullptr;
+      if (cudaMalloc(&sp, kSchedSlots * sizeof(fa::SchedSlot)) != cudaSuccess) return FA_ERR_LAUNCH;
+      if (cudaMemset(sp, 0, kSchedSlots * sizeof(fa::SchedSlot)) != cudaSuccess ||
+          cudaDeviceSynchronize() != cudaSuccess) {
+        cudaFree(sp);
+        return FA_ERR_LAUNCH;
+      }
+      di.sched = static_cast<fa::SchedSlot*>(sp);
       if (g_encode == nullptr) {
         void* fn = nullptr;
         cudaDriverEntryPointQueryResult q;
@@ -113,10 +127,22 @@ bool make_tmap(CUtensorMap* tm, const void* base, bool bf16, bool bsnd, int64_t 
   return r == CUDA_SUCCESS;
 }
 
+// (batch, head) pairs per scheduling chunk: enough that the chunk's K and V
+// (2 * Nkv * D * 2 bytes per head) stay within a comfortable share of the
+// 126 MB L2 while every CTA works on the chunk.
+int chunk_heads_for(int64_t BH, int64_t Nkv, int64_t D) {
+  const double kv_head = 4.0 * (double)Nkv * (double)D;
+  const double budget = 40.0 * 1024 * 1024;
+  int64_t g = (int64_t)(budget / kv_head);
+  if (g < 1) g = 1;
+  if (g > BH) g = BH;
+  return (int)g;
+}
+
 template <int D, typename T>
 int launch_tc(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
               int64_t Nq, int64_t Nkv, float scale, int causal, bool bsnd, cudaStream_t stream,
-              const DeviceInfo& di) {
+              DeviceInfo& di) {
   constexpr bool BF16 = std::is_same<T, __nv_bfloat16>::value;
   CUtensorMap tq, tk, tv;
   if (!make_tmap(&tq, q, BF16, bsnd, B, H, Nq, D) || !make_tmap(&tk, k, BF16, bsnd, B, H, Nkv, D) ||
@@ -134,6 +160,8 @@ int launch_tc(const void* q, const void* k, const void* v, void* o, float* lse, 
   const int64_t units = B * H * (int64_t)p.n_pairs;
   if (units > INT32_MAX) return FA_ERR_UNSUPPORTED;
   p.n_units = (int)units;
+  p.chunk_heads = chunk_heads_for(B * H, Nkv, D);
+  p.sched = di.sched + (di.launches.fetch_add(1) % kSchedSlots);
   p.timeout_ns = (uint64_t)g_timeout_us.load() * 1000ull;
   p.fault_mode = g_fault_mode.load();
   const int grid = (int)(units < di.num_sms ? units : di.num_sms);

@@ -15,8 +15,9 @@
 //   warps 0-15  four softmax warpgroups: (tile 0, keys 0-63), (tile 0, keys
 //               64-127), (tile 1, keys 0-63), (tile 1, keys 64-127).  A thread
 //               owns one query row (= one TMEM lane) and half of its 128 scores
-//               per KV tile; the two halves swap row maxima through shared
-//               memory each step.  Each warpgroup also writes its half of O.
+//               per KV tile; the two halves of a row agree on the reference max
+//               through shared memory (lazily, see below).  Each warpgroup also
+//               writes its half of O.
 //   warp 16     TMEM allocator and the MMA issuer (whole warp, elect.sync)
 //   warp 17     TMA producer (Q tiles, K/V ring of KST stages)
 //
@@ -31,11 +32,10 @@
 //   the P V product has read it, and when s_full[i] fires O_i is quiescent
 //   (the softmax may rescale it in place).
 //
-//   Special-function-unit turns: the exp phases of tile 0 and tile 1
-//   alternate (tile 0 step j, tile 1 step j, tile 0 step j+1, ...), so the
-//   SFU serves one tile at a time with two warps per SM sub-partition, and
-//   each tile's exps overlap the other tile's MMAs.  On tiles without masked
-//   scores one exp pair in TC_POLY_EVERY is computed on the FMA pipe.
+//   The two tiles run half a step apart (the MMA issue order staggers them):
+//   one tile's exps, on two warps per SM sub-partition, overlap the other
+//   tile's MMAs.  On tiles without masked scores one exp pair in
+//   TC_POLY_EVERY is computed on the FMA pipe instead of the SFU.
 //
 //   Online softmax in the exp2 domain: x = s * scale * log2(e).  The running
 //   reference max m is only moved when a tile's max exceeds it by more than
@@ -95,11 +95,21 @@ struct TcCfg {
   static constexpr int OFF_V = OFF_K + KST * TILE_BYTES;    // KST V tiles
   static constexpr int OFF_RED = OFF_V + KST * TILE_BYTES;  // [tile][parity][half][row] fp32 exchange
   static constexpr int RED_BYTES = 2 * 2 * 2 * TC_BM * 4;
-  static constexpr int OFF_BAR = OFF_RED + RED_BYTES;       // barriers
-  static constexpr int NBAR = 2 + 2 + 4 * KST + 2 + 2 + 2 + 1 + 2 + 2;
+  static constexpr int OFF_UNIT = OFF_RED + RED_BYTES;      // unit-ticket ring (UNIT_SLOTS ints)
+  static constexpr int UNIT_SLOTS = 4;
+  static constexpr int OFF_BAR = OFF_UNIT + 16 * UNIT_SLOTS;  // barriers
+  static constexpr int NBAR = 2 + 2 + 4 * KST + 2 + 2 + 2 + 1 + 2 + 2 * UNIT_SLOTS;
   static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 /*tmem slot + abort*/ + 1024 /*align slack*/;
   static constexpr int TMEM_S0 = 0, TMEM_S1 = 128, TMEM_O0 = 256, TMEM_O1 = 256 + D;
   static constexpr uint32_t TMEM_COLS = 512;
+};
+
+// Work-ticket counter of one launch.  `next` hands out tickets; the last CTA
+// to finish (counted by `done`) puts both back to zero for the launch that
+// reuses the slot.
+struct SchedSlot {
+  unsigned int next;
+  unsigned int done;
 };
 
 struct TcParams {
@@ -111,6 +121,8 @@ struct TcParams {
   float scale_log2;  // softmax scale * log2(e)
   int n_pairs;       // ceil(ceil(Nq / 128) / 2)
   int n_units;       // B * H * n_pairs
+  int chunk_heads;   // (batch, head) pairs per scheduling chunk (L2 working set)
+  SchedSlot* sched;  // this launch's work-ticket counter
   uint64_t timeout_ns;
   int fault_mode;
 };
@@ -131,11 +143,20 @@ __device__ __forceinline__ int kv_tiles_for(int qt, int Nkv, int causal) {
   return (lim + TC_BN - 1) / TC_BN;
 }
 
-__device__ __forceinline__ Unit decode_unit(int u, const TcParams& p) {
+// Ticket t -> unit.  Tickets walk the (batch, head) pairs in chunks of
+// chunk_heads, so the K/V of the heads in flight stay in L2; inside a chunk
+// the heaviest causal Q-tile pairs come first (longest-processing-time order)
+// and the heads of one pair are adjacent.
+__device__ __forceinline__ Unit decode_unit(int t, const TcParams& p) {
   Unit w;
   const int BH = p.B * p.H;
-  const int pair = p.n_pairs - 1 - u / BH;  // heaviest (causal) pairs first
-  const int bh = u % BH;
+  const long long per_chunk = (long long)p.chunk_heads * p.n_pairs;
+  const int chunk = (int)(t / per_chunk);
+  const int idx = (int)(t - chunk * per_chunk);
+  const int h0 = chunk * p.chunk_heads;
+  const int g = (BH - h0 < p.chunk_heads) ? (BH - h0) : p.chunk_heads;
+  const int pair = p.n_pairs - 1 - idx / g;
+  const int bh = h0 + idx % g;
   w.b = bh / p.H;
   w.h = bh % p.H;
   w.qt0 = 2 * pair;
@@ -153,12 +174,18 @@ struct Pack<__nv_bfloat16> {
     __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
   }
+  static __device__ __forceinline__ float2 unpack(uint32_t w) {
+    return make_float2(__uint_as_float(w << 16), __uint_as_float(w & 0xffff0000u));
+  }
 };
 template <>
 struct Pack<__half> {
   static __device__ __forceinline__ uint32_t two(float lo, float hi) {
     __half2 v = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
+  }
+  static __device__ __forceinline__ float2 unpack(uint32_t w) {
+    return __half22float2(*reinterpret_cast<const __half2*>(&w));
   }
 };
 
@@ -175,10 +202,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   float* red = reinterpret_cast<float*>(smem + C::OFF_RED);
+  volatile int* unit_ring = reinterpret_cast<volatile int*>(smem + C::OFF_UNIT);
   // barrier indices
   const int B_QFULL = 0, B_QEMPTY = 2, B_KFULL = 4, B_KEMPTY = 4 + C::KST, B_VFULL = 4 + 2 * C::KST,
             B_VEMPTY = 4 + 3 * C::KST, B_SFULL = 4 + 4 * C::KST, B_PFULL = B_SFULL + 2, B_OFULL = B_PFULL + 2,
-            B_DRAIN = B_OFULL + 2, B_TURN0 = B_DRAIN + 1, B_TURN1 = B_DRAIN + 2, B_XCHG = B_DRAIN + 3;
+            B_DRAIN = B_OFULL + 2, B_XCHG = B_DRAIN + 1, B_UFULL = B_XCHG + 2,
+            B_UEMPTY = B_UFULL + C::UNIT_SLOTS;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
@@ -202,8 +231,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       mbar_init(bar(B_VEMPTY + s), 1);
     }
     mbar_init(bar(B_DRAIN), 1);
-    mbar_init(bar(B_TURN0), 8);
-    mbar_init(bar(B_TURN1), 8);
+    for (int i = 0; i < C::UNIT_SLOTS; ++i) {
+      mbar_init(bar(B_UFULL + i), 1);
+      mbar_init(bar(B_UEMPTY + i), 1 + TC_SOFTMAX_WARPS);  // MMA warp + softmax warps
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -238,8 +269,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       for (int s = 0; s < C::KST; ++s) { k_pend[s] = v_pend[s] = false; k_issued[s] = v_issued[s] = 0; }
       q_pend[0] = q_pend[1] = false; q_issued[0] = q_issued[1] = 0;
       bool ok = true;
-      for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-        const Unit w = decode_unit(u, p);
+      int uslot = 0;
+      uint32_t uphase = 0;
+      while (ok) {
+        // claim the next ticket and hand it to the other roles
+        const unsigned int t = atomicAdd(&p.sched->next, 1u);
+        const int tk = (t < (unsigned int)p.n_units) ? (int)t : -1;
+        if (!mbar_wait(bar(B_UEMPTY + uslot), uphase ^ 1, wctx)) break;
+        unit_ring[uslot] = tk;
+        mbar_arrive(bar(B_UFULL + uslot));
+        if (++uslot == C::UNIT_SLOTS) { uslot = 0; uphase ^= 1; }
+        if (tk < 0) break;
+        const Unit w = decode_unit(tk, p);
         for (int i = 0; i < 2 && ok; ++i) {
           if (i == 1 && !w.active1) break;
           if (!mbar_wait(bar(B_QEMPTY + i), q_phase[i] ^ 1, wctx)) { ok = false; break; }
@@ -312,8 +353,19 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const uint32_t tS[2] = {tmem + C::TMEM_S0, tmem + C::TMEM_S1};
     const uint32_t tO[2] = {tmem + C::TMEM_O0, tmem + C::TMEM_O1};
     auto wait_all = [&](int b, uint32_t ph) { return __all_sync(0xffffffffu, mbar_wait(bar(b), ph, wctx)); };
-    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-      const Unit w = decode_unit(u, p);
+    int uslot = 0;
+    uint32_t uphase = 0;
+    bool first_unit_m = true;
+    while (ok) {
+      if (!wait_all(B_UFULL + uslot, uphase)) break;
+      const int tk = unit_ring[uslot];
+      mbar_arrive_warp(bar(B_UEMPTY + uslot));
+      if (++uslot == C::UNIT_SLOTS) { uslot = 0; uphase ^= 1; }
+      if (tk < 0) break;
+      const bool u_first = first_unit_m;
+      first_unit_m = false;
+      (void)u_first;
+      const Unit w = decode_unit(tk, p);
       const int n[2] = {w.n0, w.n1};
       const int N = w.n0 > w.n1 ? w.n0 : w.n1;
       for (int i = 0; i < 2 && ok; ++i) {
@@ -325,7 +377,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       uint32_t ph_prev = 0;
       for (int j = 0; j <= N && ok; ++j) {
         if (j < N && !wait_all(B_KFULL + st, kv_phase)) { ok = false; break; }
-        FA_TR(lane == 0 && u == (int)blockIdx.x, 16, j, 0);
+        FA_TR(lane == 0 && u_first, 16, j, 0);
         if (j > 0 && !wait_all(B_VFULL + st_prev, ph_prev)) { ok = false; break; }
         tc_fence_after();
         const uint64_t dK = dK0 + (uint64_t)((st * C::TILE_BYTES) >> 4);
@@ -335,7 +387,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           if (j >= 1 && j - 1 < n[i]) {
             // O_i += P_i(j-1) V_(j-1)
             if (!wait_all(B_PFULL + i, p_phase[i])) { ok = false; break; }
-            FA_TR(lane == 0 && u == (int)blockIdx.x, 16 + i, j - 1, 1);
+            FA_TR(lane == 0 && u_first, 16 + i, j - 1, 1);
             p_phase[i] ^= 1;
             tc_fence_after();
             const uint32_t acc0 = (j - 1 > 0) ? 1u : 0u;
@@ -353,7 +405,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               mma_ss_elect(tS[i], dQ[i] + off, dK + off, IDESC_S, k > 0 ? 1u : 0u);
             }
             mma_commit_elect(bar(B_SFULL + i));
-            FA_TR(lane == 0 && u == (int)blockIdx.x, 16 + i, j, 2);
+            FA_TR(lane == 0 && u_first, 16 + i, j, 2);
             if (j == n[i] - 1) mma_commit_elect(bar(B_QEMPTY + i));
           }
         }
@@ -386,31 +438,45 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     const uint32_t tO = tmem + lane_base + (tile ? C::TMEM_O1 : C::TMEM_O0) + (D / 2) * half;
     float* red_t = red + tile * (2 * 2 * TC_BM);  // [parity][half][row]
     const float sl2 = p.scale_log2;
-    uint32_t s_phase = 0, o_phase = 0, t_phase = 0, x_phase = 0;
+    uint32_t s_phase = 0, o_phase = 0, x_phase = 0;
     bool ok = true;
-    // Swap one float per row with the other half of this tile (bounded wait).
-    auto exchange = [&](float mine, float& theirs) -> bool {
+    // One float per row is swapped with the other half of this tile through
+    // shared memory (double-buffered by phase parity): publish() writes and
+    // arrives, collect() waits (bounded) and reads the partner's value.
+    auto publish = [&](float mine) {
       red_t[(x_phase * 2 + half) * TC_BM + r] = mine;
       mbar_arrive_warp(bar(B_XCHG + tile));
+    };
+    auto collect = [&](float& theirs) -> bool {
       const bool got = __all_sync(0xffffffffu, mbar_wait(bar(B_XCHG + tile), x_phase, wctx));
       if (got) theirs = red_t[(x_phase * 2 + (half ^ 1)) * TC_BM + r];
       x_phase ^= 1;
       return got;
     };
-    for (int u = blockIdx.x; u < p.n_units && ok; u += gridDim.x) {
-      const Unit w = decode_unit(u, p);
+    int uslot = 0;
+    uint32_t uphase = 0;
+    bool first_unit = true;
+    while (ok) {
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_UFULL + uslot), uphase, wctx));
+      if (!ok) break;
+      const int tk = unit_ring[uslot];
+      mbar_arrive_warp(bar(B_UEMPTY + uslot));
+      if (++uslot == C::UNIT_SLOTS) { uslot = 0; uphase ^= 1; }
+      if (tk < 0) break;
+      const Unit w = decode_unit(tk, p);
       const int n = tile ? w.n1 : w.n0;
+      const bool this_first = first_unit;
+      first_unit = false;
       if (n == 0) continue;
       const int qt = w.qt0 + tile;
       const int row = qt * TC_BM + r;
-      const bool first_unit = (u == (int)blockIdx.x);
-      (void)first_unit;
+      (void)this_first;
       float m_ref = -INFINITY;  // running reference max (log2 domain), identical in both halves
       float l = 0.f;            // this half's share of the row sum
       for (int j = 0; j < n; ++j) {
         ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SFULL + tile), s_phase, wctx));
         if (!ok) break;
-        FA_TR(first_unit && lane == 0, warp, j, 0);
+        FA_TR(this_first && lane == 0, warp, j, 0);
         s_phase ^= 1;
         tc_fence_after();
         const int col0 = j * TC_BN + 64 * half;
@@ -422,7 +488,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           // pass 1: this half's row max
           float s[64];
           tmem_ld64(tS, s);
-          FA_TR(first_unit && lane == 0, warp, j, 1);
+          FA_TR(this_first && lane == 0, warp, j, 1);
           if (need_mask) {
 #pragma unroll
             for (int c = 0; c < 64; ++c)
@@ -442,32 +508,31 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         // row-max exchange and the SFU turn wait.
         float sa[32], sb[32];
         tmem_ld32_issue(tS, sa);
-        FA_TR(first_unit && lane == 0, warp, j, 2);
-        float other = -INFINITY;
-        ok = exchange(mt, other);
-        if (!ok) break;
-        FA_TR(first_unit && lane == 0, warp, j, 3);
-        mt = fmaxf(mt, other) * sl2;
-        float corr = 1.f;
+        FA_TR(this_first && lane == 0, warp, j, 2);
+        // Reference max (log2 domain).  A warp waits for the other half's
+        // candidate now only when one of its rows must move the reference;
+        // otherwise it goes ahead with m_ref and checks the partner's
+        // candidate after its exps (published long before).  The reference is
+        // the exact max when it moves, so the largest P of that step is
+        // exactly 1 (no rounding on the dominant weight).
+        const float cand = mt * sl2;
+        publish(cand);
+        const bool waited = __any_sync(0xffffffffu, cand > m_ref + TC_RESCALE_THRESHOLD);
+        float m_new = m_ref, m_use = m_ref;
         bool moved = false;
-        if (mt > m_ref + TC_RESCALE_THRESHOLD) {
-          corr = ex2(m_ref - mt);  // 0 when m_ref = -inf
-          m_ref = mt;
-          moved = true;
-        }
-        const float mref_use = (m_ref == -INFINITY) ? 0.f : m_ref;
-        // SFU turn: tile 0 step j, tile 1 step j, tile 0 step j + 1, ...
-        if (tile == 0) {
-          if (j >= 1 && w.active1) {
-            ok = __all_sync(0xffffffffu, mbar_wait(bar(B_TURN0), t_phase, wctx));
-            t_phase ^= 1;
+        if (waited) {
+          float other = -INFINITY;
+          ok = collect(other);
+          if (!ok) break;
+          const float mx2 = fmaxf(cand, other);
+          if (mx2 > m_ref + TC_RESCALE_THRESHOLD) {
+            moved = true;
+            m_new = m_use = mx2;
           }
-        } else if (j < w.n0) {
-          ok = __all_sync(0xffffffffu, mbar_wait(bar(B_TURN1), t_phase, wctx));
-          t_phase ^= 1;
         }
-        if (!ok) break;
-        FA_TR(first_unit && lane == 0, warp, j, 4);
+        FA_TR(this_first && lane == 0, warp, j, 3);
+        FA_TR(this_first && lane == 0, warp, j, 4);
+        const float mref_use = (m_use == -INFINITY) ? 0.f : m_use;
         const uint64_t scale2 = f2_pack(sl2, sl2);
         const uint64_t negm2 = f2_pack(-mref_use, -mref_use);
         uint64_t acc2[2] = {0ull, 0ull};
@@ -515,19 +580,42 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           exp_chunks(std::false_type{});
         else
           exp_chunks(std::true_type{});
-        FA_TR(first_unit && lane == 0, warp, j, 5);
-        if (tile == 0) {
-          if (w.active1) mbar_arrive_warp(bar(B_TURN1));
-        } else if (j + 1 < w.n0) {
-          mbar_arrive_warp(bar(B_TURN0));
-        }
+        FA_TR(this_first && lane == 0, warp, j, 5);
         float sum;
         {
           float a0, a1;
           f2_unpack(f2_add(acc2[0], acc2[1]), a0, a1);
           sum = a0 + a1;
         }
-        l = l * corr + sum;
+        bool redo = false;
+        if (!waited) {
+          float other = -INFINITY;
+          ok = collect(other);
+          if (!ok) break;
+          const float mx2 = fmaxf(cand, other);
+          if (mx2 > m_ref + TC_RESCALE_THRESHOLD) {
+            moved = redo = true;
+            m_new = mx2;
+          }
+        }
+        // The other half moved the reference after this half had computed P
+        // against m_ref: scale this half's P and row sum by 2^(m_ref - m_new)
+        // (rare; one extra rounding of that step's P).
+        if (__any_sync(0xffffffffu, redo)) {
+          const float f = redo ? ex2(m_ref - m_new) : 1.f;
+          float pv[32];
+          tmem_ld32(tS, pv);
+          uint32_t pw[32];
+#pragma unroll
+          for (int t = 0; t < 32; ++t) {
+            const float2 q2 = Pack<T>::unpack(__float_as_uint(pv[t]));
+            pw[t] = Pack<T>::two(q2.x * f, q2.y * f);
+          }
+          tmem_st32(tS, pw);
+          sum *= f;
+        }
+        FA_TR(this_first && lane == 0, warp, j, 7);
+        const float corr = moved ? ex2(m_ref - m_new) : 1.f;  // 0 when m_ref = -inf
         // Rescale this half of O in place when this warp moved any row's
         // reference max (O is quiescent: its last P V finished before S_i(j)
         // was signalled).
@@ -545,12 +633,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         tmem_wait_st();
         tc_fence_before();
         if (p.fault_mode != 1) mbar_arrive_warp(bar(B_PFULL + tile));
-        FA_TR(first_unit && lane == 0, warp, j, 6);
+        m_ref = m_new;
+        l = l * corr + sum;
+        FA_TR(this_first && lane == 0, warp, j, 6);
       }
       if (!ok) break;
       // ---------------------------------------------------------- epilogue
       float l_other = 0.f;
-      ok = exchange(l, l_other);
+      publish(l);
+      ok = collect(l_other);
       if (!ok) break;
       l += l_other;
       ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OFULL + tile), o_phase, wctx));
@@ -594,6 +685,14 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == WARP_MMA) tmem_dealloc(tmem, C::TMEM_COLS);
+  if (threadIdx.x == 0) {
+    // The last CTA out returns this launch's ticket counter to zero.
+    __threadfence();
+    if (atomicAdd(&p.sched->done, 1u) == gridDim.x - 1) {
+      atomicExch(&p.sched->next, 0u);
+      atomicExch(&p.sched->done, 0u);
+    }
+  }
 }
 
 }  // namespace fa

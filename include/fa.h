@@ -49,7 +49,8 @@ typedef enum {
   FA_ERR_MISALIGNED = 3,   /* q, k, v, o not 16-byte aligned, or lse not 4-byte aligned */
   FA_ERR_LAUNCH = 4,       /* the CUDA launch or tensor-map creation failed */
   FA_ERR_TIMEOUT = 5,      /* a bounded device-side wait expired (see fa_get_device_status) */
-  FA_ERR_NO_DEVICE = 6     /* no usable sm_100 device for the current context */
+  FA_ERR_NO_DEVICE = 6,    /* no usable sm_100 device for the current context */
+  FA_ERR_TOO_LARGE = 7     /* fa_fwd_noalloc only: the call needs more than its fixed scratch */
 } fa_status_t;
 
 /*
@@ -85,6 +86,39 @@ typedef enum {
 int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
            int64_t B, int64_t H, int64_t Nq, int64_t Nkv, int64_t d,
            float scale, int causal, int layout, int dtype, void* stream);
+
+/*
+ * fa_fwd_noalloc -- the same computation, arguments and results as fa_fwd,
+ * for callers that must never allocate device memory: code that runs inside
+ * a memory pool or arena it does not own, real-time or embedded services that
+ * reserve all device memory when they start, or hosts that forbid cudaMalloc
+ * after start-up.  (The surveyed pages have no counterpart: this is a property
+ * of the library, not of the method.)
+ *
+ * fa_fwd's tile scheduler keeps its per-launch work counters in 8 KB that it
+ * allocates on its first call on a device.  This entry point keeps its single
+ * counter in a fixed 256-byte static device array instead, which every GPU
+ * that loads the library holds until the process exits; no call allocates
+ * or frees anything.  The counter is cleared (cudaMemsetAsync on `stream`)
+ * before each launch.
+ *
+ *   - The first call on a device looks up the array's device address
+ *     (cudaGetSymbolAddress) and sets kernel attributes; make that first call
+ *     before any stream capture.
+ *   - Every call on a device shares the array and it keeps the last call's
+ *     contents: calls that overlap on the GPU (other streams, other threads)
+ *     race on the counter and may compute wrong results.  Serialise them.
+ *   - Limit: the scratch holds one 32-bit work-ticket counter, so a bf16/fp16
+ *     call may have at most 2^31 - 1025 work units (a unit is a pair of
+ *     128-row query tiles of one batch and head); larger calls return
+ *     FA_ERR_TOO_LARGE before anything is launched.  fp32 inputs use no
+ *     scratch.
+ *
+ * Other arguments, ownership and errors are as for fa_fwd.
+ */
+int fa_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse,
+                   int64_t B, int64_t H, int64_t Nq, int64_t Nkv, int64_t d,
+                   float scale, int causal, int layout, int dtype, void* stream);
 
 /* Human-readable name of a status code (static string, never NULL). */
 const char* fa_status_string(int status);

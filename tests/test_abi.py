@@ -32,7 +32,7 @@ def test_library_exports_every_declared_symbol(fa_lib):
 
 
 def test_status_strings_and_version(fa_lib):
-    for code in range(7):
+    for code in range(8):
         assert fa.fa_status_string(code).startswith("FA_")
     assert fa.fa_status_string(99) == "FA_ERR_UNKNOWN"
     assert fa.fa_abi_version() == (1 << 16)

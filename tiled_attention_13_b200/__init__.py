@@ -21,7 +21,7 @@ import os
 
 __all__ = [
     "FA_LAYOUT_BHND", "FA_LAYOUT_BSND", "FA_DTYPE_BF16", "FA_DTYPE_FP16", "FA_DTYPE_FP32",
-    "FaError", "lib", "lib_path", "fa_fwd", "fa_status_string", "fa_get_device_status",
+    "FaError", "lib", "lib_path", "fa_fwd", "fa_fwd_noalloc", "fa_status_string", "fa_get_device_status",
     "fa_set_wait_timeout_us", "fa_debug_set_fault", "fa_abi_version", "forward", "forward_host",
     "EXPORTED",
 ]
@@ -30,7 +30,7 @@ FA_LAYOUT_BHND, FA_LAYOUT_BSND = 0, 1
 FA_DTYPE_BF16, FA_DTYPE_FP16, FA_DTYPE_FP32 = 0, 1, 2
 FA_OK = 0
 
-EXPORTED = ("fa_fwd", "fa_status_string", "fa_get_device_status", "fa_set_wait_timeout_us",
+EXPORTED = ("fa_fwd", "fa_fwd_noalloc", "fa_status_string", "fa_get_device_status", "fa_set_wait_timeout_us",
             "fa_debug_set_fault", "fa_abi_version")
 
 _LIB = None
@@ -59,6 +59,8 @@ def lib() -> ctypes.CDLL:
     L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, ctypes.c_float, ctypes.c_int,
                          ctypes.c_int, ctypes.c_int, vp]
     L.fa_fwd.restype = ctypes.c_int
+    L.fa_fwd_noalloc.argtypes = L.fa_fwd.argtypes
+    L.fa_fwd_noalloc.restype = ctypes.c_int
     L.fa_status_string.argtypes = [ctypes.c_int]
     L.fa_status_string.restype = ctypes.c_char_p
     L.fa_get_device_status.argtypes = [vp]
@@ -81,6 +83,13 @@ def fa_fwd(q, k, v, o, lse, B, H, Nq, Nkv, d, scale, causal, layout, dtype, stre
     """
     return lib().fa_fwd(q, k, v, o, lse, B, H, Nq, Nkv, d, float(scale), int(causal), int(layout),
                         int(dtype), stream)
+
+
+def fa_fwd_noalloc(q, k, v, o, lse, B, H, Nq, Nkv, d, scale, causal, layout, dtype, stream) -> int:
+    """int fa_fwd_noalloc(...): fa_fwd for callers that must not allocate device
+    memory (fixed static scratch; calls must not overlap on the GPU)."""
+    return lib().fa_fwd_noalloc(q, k, v, o, lse, B, H, Nq, Nkv, d, float(scale), int(causal), int(layout),
+                                int(dtype), stream)
 
 
 def fa_status_string(status: int) -> str:

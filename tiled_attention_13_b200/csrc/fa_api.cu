@@ -242,6 +242,7 @@ const char* fa_status_string(int status) {
     case FA_ERR_LAUNCH: return "FA_ERR_LAUNCH: CUDA launch or descriptor failure";
     case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT: a bounded device wait expired";
     case FA_ERR_NO_DEVICE: return "FA_ERR_NO_DEVICE: no usable sm_100 device";
+    case FA_ERR_TOO_LARGE: return "FA_ERR_TOO_LARGE: the problem needs more than fa_fwd_noalloc's fixed scratch";
     default: return "FA_ERR_UNKNOWN";
   }
 }
@@ -274,3 +275,154 @@ int fa_debug_trace_read(unsigned long long* host, int n) {
 #endif
 
 }  // extern "C"
+
+// ---------------------------------------------------------------- fa_fwd_noalloc
+// An entry point for callers that must not allocate device memory at all:
+// code running inside a memory pool or arena it does not own, real-time or
+// embedded services that reserve all device memory up front, or hosts that
+// forbid cudaMalloc after start-up.  fa_fwd's tile scheduler keeps its work
+// counters in an 8 KB buffer that it allocates on its first call on a device;
+// this variant keeps the counter in a fixed static device array instead, so
+// none of its calls allocates anything.
+namespace fa {
+constexpr int kNoAllocScratchBytes = 256;
+constexpr int kNoAllocScratchSlots = kNoAllocScratchBytes / (int)sizeof(SchedSlot);
+// One copy per device that loads the library, held until the process exits.
+// Every call of fa_fwd_noalloc on a device uses slot 0; see the header for why
+// overlapping calls race.
+static __device__ __align__(256) SchedSlot g_noalloc_scratch[kNoAllocScratchSlots];
+}  // namespace fa
+
+namespace {
+
+struct NoAllocDevice {
+  bool ready = false;
+  bool supported = false;
+  int num_sms = 0;
+  unsigned int* status = nullptr;       // device address of fa::g_status_word
+  fa::SchedSlot* scratch = nullptr;     // device address of fa::g_noalloc_scratch
+};
+NoAllocDevice g_noalloc_dev[kMaxDevices];
+
+// Once per device, with that device current.  Host code only holds a stand-in
+// for a __device__ variable's name, so the device address of the scratch
+// array comes from cudaGetSymbolAddress.  Nothing here allocates memory.
+int noalloc_setup(int dev, NoAllocDevice** out) {
+  if (dev < 0 || dev >= kMaxDevices) return FA_ERR_NO_DEVICE;
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  NoAllocDevice& nd = g_noalloc_dev[dev];
+  if (!nd.ready) {
+    cudaDeviceProp prop;
+    if (cudaGetDeviceProperties(&prop, dev) != cudaSuccess) return FA_ERR_NO_DEVICE;
+    nd.supported = (prop.major == 10 && prop.minor == 0);
+    nd.num_sms = prop.multiProcessorCount;
+    if (nd.supported) {
+      void* sym = nullptr;
+      if (cudaGetSymbolAddress(&sym, fa::g_status_word) != cudaSuccess) return FA_ERR_LAUNCH;
+      nd.status = static_cast<unsigned int*>(sym);
+      void* scr = nullptr;
+      if (cudaGetSymbolAddress(&scr, fa::g_noalloc_scratch) != cudaSuccess || scr == nullptr)
+        return FA_ERR_LAUNCH;
+      nd.scratch = static_cast<fa::SchedSlot*>(scr);
+      bool ok = true;
+      ok &= set_smem_attr(fa::fa_fwd_tc_kernel<64, __nv_bfloat16>, fa::TcCfg<64>::SMEM_BYTES);
+      ok &= set_smem_attr(fa::fa_fwd_tc_kernel<128, __nv_bfloat16>, fa::TcCfg<128>::SMEM_BYTES);
+      ok &= set_smem_attr(fa::fa_fwd_tc_kernel<64, __half>, fa::TcCfg<64>::SMEM_BYTES);
+      ok &= set_smem_attr(fa::fa_fwd_tc_kernel<128, __half>, fa::TcCfg<128>::SMEM_BYTES);
+      ok &= set_smem_attr(fa::fa_fwd_simt_kernel<64>, fa::simt_smem_bytes<64>());
+      ok &= set_smem_attr(fa::fa_fwd_simt_kernel<128>, fa::simt_smem_bytes<128>());
+      if (!ok) return FA_ERR_LAUNCH;
+      if (g_encode == nullptr) {
+        void* fn = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &fn, cudaEnableDefault, &q) != cudaSuccess ||
+            q != cudaDriverEntryPointSuccess || fn == nullptr)
+          return FA_ERR_LAUNCH;
+        g_encode = reinterpret_cast<EncodeTiledFn>(fn);
+      }
+    }
+    nd.ready = true;
+  }
+  if (!nd.supported) return FA_ERR_NO_DEVICE;
+  *out = &nd;
+  return FA_OK;
+}
+
+template <int D, typename T>
+int launch_tc_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
+                      int64_t Nq, int64_t Nkv, float scale, int causal, bool bsnd, cudaStream_t stream,
+                      const NoAllocDevice& nd) {
+  constexpr bool BF16 = std::is_same<T, __nv_bfloat16>::value;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap(&tq, q, BF16, bsnd, B, H, Nq, D) || !make_tmap(&tk, k, BF16, bsnd, B, H, Nkv, D) ||
+      !make_tmap(&tv, v, BF16, bsnd, B, H, Nkv, D))
+    return FA_ERR_LAUNCH;
+  fa::TcParams p;
+  p.o = o;
+  p.lse = lse;
+  p.B = (int)B; p.H = (int)H; p.Nq = (int)Nq; p.Nkv = (int)Nkv;
+  p.bsnd = bsnd ? 1 : 0;
+  p.causal = causal;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const int64_t qtiles = (Nq + fa::TC_BM - 1) / fa::TC_BM;
+  p.n_pairs = (int)((qtiles + 1) / 2);
+  p.n_units = (int)(B * H * (int64_t)p.n_pairs);
+  p.chunk_heads = chunk_heads_for(B * H, Nkv, D);
+  p.sched = nd.scratch;  // slot 0 of the static array
+  p.timeout_ns = (uint64_t)g_timeout_us.load() * 1000ull;
+  p.fault_mode = g_fault_mode.load();
+  const int grid = (int)(p.n_units < nd.num_sms ? p.n_units : nd.num_sms);
+  // The counter must start at zero: the previous call's last CTA normally
+  // leaves it so, but clear it in stream order anyway (no allocation).
+  if (cudaMemsetAsync(nd.scratch, 0, sizeof(fa::SchedSlot), stream) != cudaSuccess) return FA_ERR_LAUNCH;
+  fa::fa_fwd_tc_kernel<D, T><<<grid, fa::TC_THREADS, fa::TcCfg<D>::SMEM_BYTES, stream>>>(tq, tk, tv, p,
+                                                                                         nd.status);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+}  // namespace
+
+extern "C" int fa_fwd_noalloc(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B,
+                              int64_t H, int64_t Nq, int64_t Nkv, int64_t d, float scale, int causal, int layout,
+                              int dtype, void* stream) {
+  if (B < 0 || H < 0 || Nq < 0 || Nkv < 0 || d <= 0) return FA_ERR_INVALID_ARG;
+  if (layout != FA_LAYOUT_BHND && layout != FA_LAYOUT_BSND) return FA_ERR_INVALID_ARG;
+  if (dtype != FA_DTYPE_BF16 && dtype != FA_DTYPE_FP16 && dtype != FA_DTYPE_FP32) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (B == 0 || H == 0 || Nq == 0) return FA_OK;
+  if (Nkv == 0) return FA_ERR_INVALID_ARG;
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return FA_ERR_INVALID_ARG;
+  if (B > INT32_MAX || H > INT32_MAX || B * H > INT32_MAX || Nq > INT32_MAX - 256 || Nkv > INT32_MAX - 256)
+    return FA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      (lse != nullptr && !aligned(lse, 4)))
+    return FA_ERR_MISALIGNED;
+  // The fixed scratch holds one 32-bit work-ticket counter: a call fits when
+  // the counter can number all its work units (pairs of 128-row query tiles
+  // over every batch and head) plus one closing ticket per CTA.
+  if ((int)sizeof(fa::SchedSlot) > fa::kNoAllocScratchBytes) return FA_ERR_TOO_LARGE;
+  const int64_t units = B * H * (((Nq + fa::TC_BM - 1) / fa::TC_BM + 1) / 2);
+  if (dtype != FA_DTYPE_FP32 && units > (int64_t)INT32_MAX - 1024) return FA_ERR_TOO_LARGE;
+  if (!(scale > 0.f) || std::isinf(scale)) scale = 1.0f / std::sqrt((float)d);
+
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_NO_DEVICE;
+  NoAllocDevice* nd = nullptr;
+  const int st = noalloc_setup(dev, &nd);
+  if (st != FA_OK) return st;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool bsnd = layout == FA_LAYOUT_BSND;
+  if (dtype == FA_DTYPE_FP32) {  // this kernel uses no scratch at all
+    return d == 64 ? launch_simt<64>(q, k, v, o, lse, B, H, Nq, Nkv, scale, causal, bsnd, s)
+                   : launch_simt<128>(q, k, v, o, lse, B, H, Nq, Nkv, scale, causal, bsnd, s);
+  }
+  if (dtype == FA_DTYPE_BF16) {
+    return d == 64 ? launch_tc_noalloc<64, __nv_bfloat16>(q, k, v, o, lse, B, H, Nq, Nkv, scale, causal, bsnd, s, *nd)
+                   : launch_tc_noalloc<128, __nv_bfloat16>(q, k, v, o, lse, B, H, Nq, Nkv, scale, causal, bsnd, s,
+                                                           *nd);
+  }
+  return d == 64 ? launch_tc_noalloc<64, __half>(q, k, v, o, lse, B, H, Nq, Nkv, scale, causal, bsnd, s, *nd)
+                 : launch_tc_noalloc<128, __half>(q, k, v, o, lse, B, H, Nq, Nkv, scale, causal, bsnd, s, *nd);
+}

@@ -57,6 +57,24 @@ def max_over_ranks(x: float, device=None) -> float:
     return float(t.item())
 
 
+def captured_traffic(workload: str):
+    """DRAM bytes per launch from the committed ncu capture of this workload's
+    kernel (profiles/fa_fwd_tc_<workload>.json), or None when there is none or
+    the kernel source has changed since the counters were taken."""
+    import hashlib
+
+    path = os.path.join(ROOT, "profiles", f"fa_fwd_tc_{workload.replace('-', '_')}.json")
+    if not os.path.exists(path):
+        return None
+    rec = json.load(open(path))
+    csrc = os.path.join(ROOT, "tiled_attention_13_b200", "csrc")
+    sha = hashlib.sha256(b"".join(open(os.path.join(csrc, f), "rb").read()
+                                  for f in ("fa_fwd_tc.cuh", "ptx.cuh"))).hexdigest()
+    if rec.get("kernel_source_sha256") != sha or rec.get("workload") != workload:
+        return None
+    return float(rec["dram_bytes_per_launch"])
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -301,19 +319,20 @@ def run_ours(args, wl):
     if rank == 0:
         peaks, src = load_peaks()
         kmean = sum(kern_ms) / len(kern_ms)
+        traffic = args.traffic if args.traffic is not None else captured_traffic(wl.name)
         achieved = wl.flops / (kmean * 1e-3) / 1e12
         bound = "tensor" if wl.Nkv >= 512 else "hbm"
         if bound == "tensor":
             peak = float(peaks["bf16_tflops"])
             roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                    "frac": achieved / peak, "traffic": args.traffic,
+                    "frac": achieved / peak, "traffic": traffic,
                     "peak_source": f"{src} bf16_tflops (burst; sustained {peaks.get('bf16_tflops_sustained')})",
                     "kernel_ms_mean": kmean, "kernel_ms_min": min(kern_ms)}
         else:
             gbs = wl.bytes_min / (kmean * 1e-3) / 1e9
             peak = float(peaks["hbm_gbs"])
             roof = {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
-                    "traffic": args.traffic, "peak_source": f"{src} hbm_gbs", "kernel_ms_mean": kmean,
+                    "traffic": traffic, "peak_source": f"{src} hbm_gbs", "kernel_ms_mean": kmean,
                     "kernel_ms_min": min(kern_ms), "algorithmic_bytes": wl.bytes_min}
         cpu = None
         if not args.no_cpu_baseline and ws == 1:

@@ -37,7 +37,8 @@ _LIB = None
 
 
 def lib_path() -> str:
-    return os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa_b200.so")
+    """The in-tree library, or another build named by $FA_B200_LIB."""
+    return os.environ.get("FA_B200_LIB") or os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa_b200.so")
 
 
 class FaError(RuntimeError):

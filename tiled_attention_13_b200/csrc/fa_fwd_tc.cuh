@@ -82,6 +82,9 @@ constexpr float TC_RESCALE_THRESHOLD = 8.0f;  // log2 units
 #ifndef FA_POLY_EVERY
 #define FA_POLY_EVERY 4
 #endif
+#ifndef FA_POLY_MODE
+#define FA_POLY_MODE 0  // 0: one pair in FA_POLY_EVERY per sub-chunk; 1: one whole sub-chunk per half, staggered
+#endif
 constexpr int TC_POLY_EVERY = FA_POLY_EVERY;  // one exp pair in TC_POLY_EVERY on the FMA pipe
 
 template <int D>
@@ -540,13 +543,19 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         // S columns (already read).  On tiles without masked scores one pair
         // in TC_POLY_EVERY takes 2^x on the FMA pipe.
         auto exp_chunks = [&](auto use_poly) {
-          auto sub = [&](const float* sc, int cbase) {
+          // 8 pairs -> 8 packed P columns; POLY selects the FMA-pipe exp2
+          // for the whole sub-chunk (interleaved mode: one pair in
+          // TC_POLY_EVERY instead).
+          auto sub = [&](const float* sc, int cbase, auto poly_all) {
             uint32_t pk[8];
 #pragma unroll
             for (int t = 0; t < 8; ++t) {
               const uint64_t x2 = f2_fma(f2_pack(sc[2 * t], sc[2 * t + 1]), scale2, negm2);
               float p0, p1;
-              if (decltype(use_poly)::value && (t % TC_POLY_EVERY) == TC_POLY_EVERY - 1) {
+              constexpr bool kPolyAll = decltype(poly_all)::value;
+              const bool poly = decltype(use_poly)::value &&
+                                (FA_POLY_MODE == 1 ? kPolyAll : ((t % TC_POLY_EVERY) == TC_POLY_EVERY - 1));
+              if (poly) {
                 exp2_poly_x2(x2, p0, p1);
               } else {
                 float x0, x1;
@@ -566,15 +575,17 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                 if (col0 + cbase + c >= lim_c) sc[c] = -INFINITY;
             }
           };
+          using PY = std::true_type;
+          using PN = std::false_type;
           tmem_ld_wait32(sa);
           mask32(sa, 0);
-          sub(sa, 0);
+          if (FA_POLY_MODE == 1 && half == 1) sub(sa, 0, PY{}); else sub(sa, 0, PN{});
           tmem_ld32_issue(tS + 32, sb);  // columns 32-63 load while 16-31 are processed
-          sub(sa + 16, 16);
+          sub(sa + 16, 16, PN{});
           tmem_ld_wait32(sb);
           mask32(sb, 32);
-          sub(sb, 32);
-          sub(sb + 16, 48);
+          sub(sb, 32, PN{});
+          if (FA_POLY_MODE == 1 && half == 0) sub(sb + 16, 48, PY{}); else sub(sb + 16, 48, PN{});
         };
         if (need_mask)
           exp_chunks(std::false_type{});

@@ -26,11 +26,12 @@
 //   0-63 overwrites S_i columns [0,32), for keys 64-127 columns [64,96): each
 //   half writes only columns it has already read.
 //
-//   MMA order per KV step j (tile i = 0, 1):  O_i += P_i(j-1) V_(j-1), then
-//   S_i(j) = Q_i K_j^T, then commit -> s_full[i].  The tensor pipe executes
-//   a CTA's MMAs in issue order, so S_i(j) overwrites P_i(j-1) only after
-//   the P V product has read it, and when s_full[i] fires O_i is quiescent
-//   (the softmax may rescale it in place).
+//   MMA order per KV step j (tile i = 0, 1):  O_i += P_i(j-1) V_(j-1) in two
+//   parts as the softmax hands them over (keys 0-31 of each half, then keys
+//   32-63), then S_i(j) = Q_i K_j^T, then commit -> s_full[i].  The tensor
+//   pipe executes a CTA's MMAs in issue order, so S_i(j) overwrites P_i(j-1)
+//   only after the P V product has read it, and when s_full[i] fires O_i is
+//   quiescent (the softmax may rescale it in place).
 //
 //   The two tiles run half a step apart (the MMA issue order staggers them):
 //   one tile's exps, on two warps per SM sub-partition, overlap the other
@@ -82,10 +83,8 @@ constexpr float TC_RESCALE_THRESHOLD = 8.0f;  // log2 units
 #ifndef FA_POLY_EVERY
 #define FA_POLY_EVERY 4
 #endif
-#ifndef FA_POLY_MODE
-#define FA_POLY_MODE 0  // 0: one pair in FA_POLY_EVERY per sub-chunk; 1: one whole sub-chunk per half, staggered
-#endif
 constexpr int TC_POLY_EVERY = FA_POLY_EVERY;  // one exp pair in TC_POLY_EVERY on the FMA pipe
+
 
 template <int D>
 struct TcCfg {
@@ -101,7 +100,7 @@ struct TcCfg {
   static constexpr int OFF_UNIT = OFF_RED + RED_BYTES;      // unit-ticket ring (UNIT_SLOTS ints)
   static constexpr int UNIT_SLOTS = 4;
   static constexpr int OFF_BAR = OFF_UNIT + 16 * UNIT_SLOTS;  // barriers
-  static constexpr int NBAR = 2 + 2 + 4 * KST + 2 + 2 + 2 + 1 + 2 + 2 * UNIT_SLOTS;
+  static constexpr int NBAR = 2 + 2 + 4 * KST + 2 + 4 + 2 + 1 + 2 + 2 * UNIT_SLOTS;
   static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 /*tmem slot + abort*/ + 1024 /*align slack*/;
   static constexpr int TMEM_S0 = 0, TMEM_S1 = 128, TMEM_O0 = 256, TMEM_O1 = 256 + D;
   static constexpr uint32_t TMEM_COLS = 512;
@@ -208,7 +207,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   volatile int* unit_ring = reinterpret_cast<volatile int*>(smem + C::OFF_UNIT);
   // barrier indices
   const int B_QFULL = 0, B_QEMPTY = 2, B_KFULL = 4, B_KEMPTY = 4 + C::KST, B_VFULL = 4 + 2 * C::KST,
-            B_VEMPTY = 4 + 3 * C::KST, B_SFULL = 4 + 4 * C::KST, B_PFULL = B_SFULL + 2, B_OFULL = B_PFULL + 2,
+            B_VEMPTY = 4 + 3 * C::KST, B_SFULL = 4 + 4 * C::KST, B_PFULL = B_SFULL + 2, B_OFULL = B_PFULL + 4,
             B_DRAIN = B_OFULL + 2, B_XCHG = B_DRAIN + 1, B_UFULL = B_XCHG + 2,
             B_UEMPTY = B_UFULL + C::UNIT_SLOTS;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
@@ -223,7 +222,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       mbar_init(bar(B_QFULL + i), 1);
       mbar_init(bar(B_QEMPTY + i), 1);
       mbar_init(bar(B_SFULL + i), 1);
-      mbar_init(bar(B_PFULL + i), 8);  // one arrival per softmax warp of the tile
+      mbar_init(bar(B_PFULL + 2 * i), 8);      // P keys 0-31 and 64-95: one arrival per warp of the tile
+      mbar_init(bar(B_PFULL + 2 * i + 1), 8);  // P keys 32-63 and 96-127
       mbar_init(bar(B_OFULL + i), 1);
       mbar_init(bar(B_XCHG + i), 8);
     }
@@ -350,7 +350,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
                             smem_desc_sw128(sbase + C::OFF_Q + C::TILE_BYTES, 16, 1024)};
     const uint64_t dK0 = smem_desc_sw128(sbase + C::OFF_K, 16, 1024);
     const uint64_t dV0 = smem_desc_sw128(sbase + C::OFF_V, C::CHUNK_BYTES, 1024);
-    uint32_t q_phase[2] = {0, 0}, kv_phase = 0, p_phase[2] = {0, 0};
+    uint32_t q_phase[2] = {0, 0}, kv_phase = 0, p_phase[4] = {0, 0, 0, 0};
     int st = 0;
     bool ok = true;
     const uint32_t tS[2] = {tmem + C::TMEM_S0, tmem + C::TMEM_S1};
@@ -379,28 +379,46 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       int st_prev = 0;
       uint32_t ph_prev = 0;
       for (int j = 0; j <= N && ok; ++j) {
-        if (j < N && !wait_all(B_KFULL + st, kv_phase)) { ok = false; break; }
+        // K_j is needed only by this iteration's S MMAs (waited for just
+        // before the first of them), V_(j-1) by its P V.
+        bool k_ready = false;
         FA_TR(lane == 0 && u_first, 16, j, 0);
         if (j > 0 && !wait_all(B_VFULL + st_prev, ph_prev)) { ok = false; break; }
+        FA_TR(lane == 0 && u_first, 17, j, 0);
         tc_fence_after();
         const uint64_t dK = dK0 + (uint64_t)((st * C::TILE_BYTES) >> 4);
         const uint64_t dV = dV0 + (uint64_t)((st_prev * C::TILE_BYTES) >> 4);
         for (int i = 0; i < 2 && ok; ++i) {
           if (n[i] == 0) continue;
           if (j >= 1 && j - 1 < n[i]) {
-            // O_i += P_i(j-1) V_(j-1)
-            if (!wait_all(B_PFULL + i, p_phase[i])) { ok = false; break; }
-            FA_TR(lane == 0 && u_first, 16 + i, j - 1, 1);
-            p_phase[i] ^= 1;
-            tc_fence_after();
+            // O_i += P_i(j-1) V_(j-1), in two parts as the softmax hands them
+            // over: part q holds keys [32q, 32q+32) of both key halves, i.e.
+            // k-steps {2q, 2q+1, 4+2q, 5+2q}.
             const uint32_t acc0 = (j - 1 > 0) ? 1u : 0u;
 #pragma unroll
-            for (int kk = 0; kk < TC_BN / 16; ++kk)
-              mma_ts_elect(tO[i], tS[i] + (kk >> 2) * 64 + (kk & 3) * 8, dV + (uint64_t)((kk * 16 * 128) >> 4),
-                           IDESC_PV, kk > 0 ? 1u : acc0);
+            for (int part = 0; part < 2; ++part) {
+              if (!wait_all(B_PFULL + 2 * i + part, p_phase[2 * i + part])) { ok = false; break; }
+              if (part == 0) FA_TR(lane == 0 && u_first, 16 + i, j - 1, 1);
+              p_phase[2 * i + part] ^= 1;
+              tc_fence_after();
+#pragma unroll
+              for (int e = 0; e < 4; ++e) {
+                const int kk = ((e >> 1) << 2) + 2 * part + (e & 1);  // 2q, 2q+1, 4+2q, 5+2q
+                mma_ts_elect(tO[i], tS[i] + (kk >> 2) * 64 + (kk & 3) * 8,
+                             dV + (uint64_t)((kk * 16 * 128) >> 4), IDESC_PV, (part == 0 && e == 0) ? acc0 : 1u);
+              }
+            }
+            if (!ok) break;
             if (j - 1 == n[i] - 1) mma_commit_elect(bar(B_OFULL + i));
+            // V_(j-1) is free once the last tile's P V has read it.
+            if (i == 1 || n[1] == 0 || j - 1 >= n[1]) mma_commit_elect(bar(B_VEMPTY + st_prev));
           }
           if (j < n[i]) {
+            if (!k_ready) {
+              if (!wait_all(B_KFULL + st, kv_phase)) { ok = false; break; }
+              k_ready = true;
+              tc_fence_after();
+            }
             // S_i(j) = Q_i K_j^T
 #pragma unroll
             for (int k = 0; k < D / 16; ++k) {
@@ -414,7 +432,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         if (!ok) break;
         if (j < N) mma_commit_elect(bar(B_KEMPTY + st));
-        if (j > 0) mma_commit_elect(bar(B_VEMPTY + st_prev));
+        FA_TR(lane == 0 && u_first, 16, j, 3);
         st_prev = st;
         ph_prev = kv_phase;
         if (j < N) {
@@ -539,65 +557,47 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const uint64_t scale2 = f2_pack(sl2, sl2);
         const uint64_t negm2 = f2_pack(-mref_use, -mref_use);
         uint64_t acc2[2] = {0ull, 0ull};
-        // 16 scores -> 8 packed P columns, written over this half's first 32
-        // S columns (already read).  On tiles without masked scores one pair
-        // in TC_POLY_EVERY takes 2^x on the FMA pipe.
-        auto exp_chunks = [&](auto use_poly) {
-          // 8 pairs -> 8 packed P columns; POLY selects the FMA-pipe exp2
-          // for the whole sub-chunk (interleaved mode: one pair in
-          // TC_POLY_EVERY instead).
-          auto sub = [&](const float* sc, int cbase, auto poly_all) {
-            uint32_t pk[8];
+        // 8 score pairs -> 8 packed P columns, written over this half's first
+        // 32 S columns (already read).  On tiles without masked scores one
+        // pair in TC_POLY_EVERY takes 2^x on the FMA pipe.
+        auto sub = [&](const float* sc, int cbase, auto use_poly) {
+          uint32_t pk[8];
 #pragma unroll
-            for (int t = 0; t < 8; ++t) {
-              const uint64_t x2 = f2_fma(f2_pack(sc[2 * t], sc[2 * t + 1]), scale2, negm2);
-              float p0, p1;
-              constexpr bool kPolyAll = decltype(poly_all)::value;
-              const bool poly = decltype(use_poly)::value &&
-                                (FA_POLY_MODE == 1 ? kPolyAll : ((t % TC_POLY_EVERY) == TC_POLY_EVERY - 1));
-              if (poly) {
-                exp2_poly_x2(x2, p0, p1);
-              } else {
-                float x0, x1;
-                f2_unpack(x2, x0, x1);
-                p0 = ex2(x0);
-                p1 = ex2(x1);
-              }
-              acc2[t & 1] = f2_add(acc2[t & 1], f2_pack(p0, p1));
-              pk[t] = Pack<T>::two(p0, p1);
+          for (int t = 0; t < 8; ++t) {
+            const uint64_t x2 = f2_fma(f2_pack(sc[2 * t], sc[2 * t + 1]), scale2, negm2);
+            float p0, p1;
+            if (decltype(use_poly)::value && (t % TC_POLY_EVERY) == TC_POLY_EVERY - 1) {
+              exp2_poly_x2(x2, p0, p1);
+            } else {
+              float x0, x1;
+              f2_unpack(x2, x0, x1);
+              p0 = ex2(x0);
+              p1 = ex2(x1);
             }
-            tmem_st8(tS + cbase / 2, pk);
-          };
-          auto mask32 = [&](float(&sc)[32], int cbase) {
-            if (!decltype(use_poly)::value && need_mask) {
-#pragma unroll
-              for (int c = 0; c < 32; ++c)
-                if (col0 + cbase + c >= lim_c) sc[c] = -INFINITY;
-            }
-          };
-          using PY = std::true_type;
-          using PN = std::false_type;
-          tmem_ld_wait32(sa);
-          mask32(sa, 0);
-          if (FA_POLY_MODE == 1 && half == 1) sub(sa, 0, PY{}); else sub(sa, 0, PN{});
-          tmem_ld32_issue(tS + 32, sb);  // columns 32-63 load while 16-31 are processed
-          sub(sa + 16, 16, PN{});
-          tmem_ld_wait32(sb);
-          mask32(sb, 32);
-          sub(sb, 32, PN{});
-          if (FA_POLY_MODE == 1 && half == 0) sub(sb + 16, 48, PY{}); else sub(sb + 16, 48, PN{});
+            acc2[t & 1] = f2_add(acc2[t & 1], f2_pack(p0, p1));
+            pk[t] = Pack<T>::two(p0, p1);
+          }
+          tmem_st8(tS + cbase / 2, pk);
         };
-        if (need_mask)
-          exp_chunks(std::false_type{});
-        else
-          exp_chunks(std::true_type{});
-        FA_TR(this_first && lane == 0, warp, j, 5);
-        float sum;
-        {
-          float a0, a1;
-          f2_unpack(f2_add(acc2[0], acc2[1]), a0, a1);
-          sum = a0 + a1;
+        auto mask32 = [&](float(&sc)[32], int cbase) {
+          if (need_mask) {
+#pragma unroll
+            for (int c = 0; c < 32; ++c)
+              if (col0 + cbase + c >= lim_c) sc[c] = -INFINITY;
+          }
+        };
+        // part 0: this half's keys 0-31 (columns 32-63 load meanwhile)
+        tmem_ld_wait32(sa);
+        mask32(sa, 0);
+        tmem_ld32_issue(tS + 32, sb);
+        if (need_mask) {
+          sub(sa, 0, std::false_type{});
+          sub(sa + 16, 16, std::false_type{});
+        } else {
+          sub(sa, 0, std::true_type{});
+          sub(sa + 16, 16, std::true_type{});
         }
+        // Settle this step's reference before any of its P is handed over.
         bool redo = false;
         if (!waited) {
           float other = -INFINITY;
@@ -609,27 +609,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             m_new = mx2;
           }
         }
-        // The other half moved the reference after this half had computed P
-        // against m_ref: scale this half's P and row sum by 2^(m_ref - m_new)
-        // (rare; one extra rounding of that step's P).
-        if (__any_sync(0xffffffffu, redo)) {
-          const float f = redo ? ex2(m_ref - m_new) : 1.f;
-          float pv[32];
-          tmem_ld32(tS, pv);
-          uint32_t pw[32];
-#pragma unroll
-          for (int t = 0; t < 32; ++t) {
-            const float2 q2 = Pack<T>::unpack(__float_as_uint(pv[t]));
-            pw[t] = Pack<T>::two(q2.x * f, q2.y * f);
-          }
-          tmem_st32(tS, pw);
-          sum *= f;
-        }
         FA_TR(this_first && lane == 0, warp, j, 7);
         const float corr = moved ? ex2(m_ref - m_new) : 1.f;  // 0 when m_ref = -inf
         // Rescale this half of O in place when this warp moved any row's
-        // reference max (O is quiescent: its last P V finished before S_i(j)
-        // was signalled).
+        // reference max, before this step's P V touches O (O is quiescent:
+        // its last P V finished before S_i(j) was signalled).
         if (j > 0 && __any_sync(0xffffffffu, moved)) {
 #pragma unroll 1
           for (int c = 0; c < D / 2; c += 32) {
@@ -641,9 +625,53 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             tmem_st32(tO + c, ow);
           }
         }
+        // Hand part 0 to the MMA warp now, unless this warp's P must still be
+        // rescaled (the other half moved the reference: rare).
+        const bool warp_redo = __any_sync(0xffffffffu, redo);
+        if (!warp_redo) {
+          tmem_wait_st();
+          tc_fence_before();
+          if (p.fault_mode != 1) mbar_arrive_warp(bar(B_PFULL + 2 * tile));
+        }
+        // part 1: keys 32-63
+        tmem_ld_wait32(sb);
+        mask32(sb, 32);
+        if (need_mask) {
+          sub(sb, 32, std::false_type{});
+          sub(sb + 16, 48, std::false_type{});
+        } else {
+          sub(sb, 32, std::true_type{});
+          sub(sb + 16, 48, std::true_type{});
+        }
+        FA_TR(this_first && lane == 0, warp, j, 5);
+        float sum;
+        {
+          float a0, a1;
+          f2_unpack(f2_add(acc2[0], acc2[1]), a0, a1);
+          sum = a0 + a1;
+        }
+        // The other half moved the reference after this half had computed P
+        // against m_ref: scale this half's P and row sum by 2^(m_ref - m_new)
+        // (rare; one extra rounding of that step's P), then hand over part 0.
+        if (warp_redo) {
+          const float f = redo ? ex2(m_ref - m_new) : 1.f;
+          float pv[32];
+          tmem_ld32(tS, pv);
+          uint32_t pw[32];
+#pragma unroll
+          for (int t = 0; t < 32; ++t) {
+            const float2 q2 = Pack<T>::unpack(__float_as_uint(pv[t]));
+            pw[t] = Pack<T>::two(q2.x * f, q2.y * f);
+          }
+          tmem_st32(tS, pw);
+          sum *= f;
+          tmem_wait_st();
+          tc_fence_before();
+          if (p.fault_mode != 1) mbar_arrive_warp(bar(B_PFULL + 2 * tile));
+        }
         tmem_wait_st();
         tc_fence_before();
-        if (p.fault_mode != 1) mbar_arrive_warp(bar(B_PFULL + tile));
+        if (p.fault_mode != 1) mbar_arrive_warp(bar(B_PFULL + 2 * tile + 1));
         m_ref = m_new;
         l = l * corr + sum;
         FA_TR(this_first && lane == 0, warp, j, 6);

@@ -265,17 +265,41 @@ def run_ours(args, wl):
     if rank == 0:
         sampler.start()
         time.sleep(0.3)
-    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    # The K timed steps are recorded once into a CUDA graph (with an event
+    # pair around every launch) and replayed: the device then runs the steps
+    # back to back and host launch overhead stays out of the timing, which
+    # matters for calls of a few microseconds.  --no-graph launches eagerly.
+    use_graph = not args.no_graph
+    ev = [(torch.cuda.Event(enable_timing=True, external=use_graph),
+           torch.cuda.Event(enable_timing=True, external=use_graph)) for _ in range(args.steps)]
     start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    graph = None
+    if use_graph:
+        graph = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream(dev)
+        cap.wait_stream(stream)
+        with torch.cuda.stream(cap):
+            graph.capture_begin()
+            for i in range(args.steps):
+                ev[i][0].record(cap)
+                step(i)
+                ev[i][1].record(cap)
+            graph.capture_end()
+        stream.wait_stream(cap)
+        graph.replay()  # untimed: uploads the graph
+        torch.cuda.synchronize()
     if ws > 1:
         dist.barrier()
     torch.cuda.synchronize()
     t0 = time.time()
     start.record(stream)
-    for i in range(args.steps):
-        ev[i][0].record(stream)
-        step(i)
-        ev[i][1].record(stream)
+    if use_graph:
+        graph.replay()
+    else:
+        for i in range(args.steps):
+            ev[i][0].record(stream)
+            step(i)
+            ev[i][1].record(stream)
     end.record(stream)
     torch.cuda.synchronize()
     t1 = time.time()
@@ -346,7 +370,8 @@ def run_ours(args, wl):
             "vs_baseline": None, "dtype": "bf16" if wl.dtype == "bf16" else wl.dtype,
             "data": "synthetic: seeded i.i.d. N(0,1) Q/K/V of the workload's shape",
             "config": _config(wl, ws), "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": args.steps, "clocks": clocks,
+            "gpu_launches": args.steps, "clocks": clocks, "timing": "cuda-graph replay of the K steps" if use_graph
+            else "eager launches",
             "pct_of_measured_bf16_peak": 100.0 * (value / ws) / float(peaks["bf16_tflops"]),
         }
         print(json.dumps(line), flush=True)
@@ -364,6 +389,7 @@ def main():
     ap.add_argument("--workload", default="llama13b-8k")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-graph", action="store_true", help="launch the timed steps eagerly instead of as one CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
     ap.add_argument("--ref-step-s", type=float, default=2.0)

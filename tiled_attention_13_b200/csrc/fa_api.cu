@@ -263,6 +263,16 @@ int fa_debug_set_fault(int mode) { return g_fault_mode.exchange(mode); }
 
 int fa_abi_version(void) { return (1 << 16) | 0; }
 
+#ifdef FA_TRACE_UNITS
+int fa_debug_trace_units_read(unsigned long long* host, int n) {
+  const int total = 3 * fa::TRU_N * fa::TRU_EV;
+  if (n > total) n = total;
+  if (cudaMemcpyFromSymbol(host, fa::g_trace_units, n * sizeof(unsigned long long)) != cudaSuccess)
+    return FA_ERR_LAUNCH;
+  return n;
+}
+#endif
+
 #ifdef FA_TRACE
 int fa_debug_trace_read(unsigned long long* host, int n) {
   const int total = fa::TRACE_STREAMS * fa::TRACE_J * fa::TRACE_EV;

@@ -72,6 +72,21 @@ __device__ unsigned long long g_trace[TRACE_STREAMS * TRACE_J * TRACE_EV];
   do {                           \
   } while (0)
 #endif
+// Unit-indexed variant (compile with -DFA_TRACE_UNITS): one row per work unit
+// of CTA 0, events per role.  Streams: 0 producer, 1 MMA, 2 softmax warp 0.
+#ifdef FA_TRACE_UNITS
+constexpr int TRU_N = 64, TRU_EV = 8;
+__device__ unsigned long long g_trace_units[3 * TRU_N * TRU_EV];
+#define FA_TRU(cond, stream, k, ev)                                                               \
+  do {                                                                                            \
+    if ((cond) && blockIdx.x == 0 && (k) < TRU_N)                                                 \
+      g_trace_units[((stream) * TRU_N + (k)) * TRU_EV + (ev)] = (unsigned long long)clock64();   \
+  } while (0)
+#else
+#define FA_TRU(cond, stream, k, ev) \
+  do {                              \
+  } while (0)
+#endif
 
 constexpr int TC_SOFTMAX_WARPS = 16;
 constexpr int WARP_MMA = 16;
@@ -152,9 +167,9 @@ __device__ __forceinline__ int kv_tiles_for(int qt, int Nkv, int causal) {
 __device__ __forceinline__ Unit decode_unit(int t, const TcParams& p) {
   Unit w;
   const int BH = p.B * p.H;
-  const long long per_chunk = (long long)p.chunk_heads * p.n_pairs;
-  const int chunk = (int)(t / per_chunk);
-  const int idx = (int)(t - chunk * per_chunk);
+  const int per_chunk = p.chunk_heads * p.n_pairs;  // <= n_units < 2^31
+  const int chunk = t / per_chunk;
+  const int idx = t - chunk * per_chunk;
   const int h0 = chunk * p.chunk_heads;
   const int g = (BH - h0 < p.chunk_heads) ? (BH - h0) : p.chunk_heads;
   const int pair = p.n_pairs - 1 - idx / g;
@@ -274,6 +289,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       bool ok = true;
       int uslot = 0;
       uint32_t uphase = 0;
+      int n_claimed = 0;
+      (void)n_claimed;
       while (ok) {
         // claim the next ticket and hand it to the other roles
         const unsigned int t = atomicAdd(&p.sched->next, 1u);
@@ -283,6 +300,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         mbar_arrive(bar(B_UFULL + uslot));
         if (++uslot == C::UNIT_SLOTS) { uslot = 0; uphase ^= 1; }
         if (tk < 0) break;
+        FA_TRU(true, 0, n_claimed, 0);
         const Unit w = decode_unit(tk, p);
         for (int i = 0; i < 2 && ok; ++i) {
           if (i == 1 && !w.active1) break;
@@ -299,6 +317,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           q_pend[i] = true; q_issued[i] = q_phase[i];
           q_phase[i] ^= 1;
         }
+        FA_TRU(true, 0, n_claimed, 1);
         const int N = w.n0 > w.n1 ? w.n0 : w.n1;
         for (int j = 0; j < N && ok; ++j) {
           const int kv0 = j * TC_BN;
@@ -322,8 +341,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               tma_load_4d(vdst + c * C::CHUNK_BYTES, &tm_v, bar(B_VFULL + st), c * 64, kv0, w.h, w.b, pol_kv);
           }
           v_pend[st] = true; v_issued[st] = kv_phase;
+          FA_TRU(j == N - 1, 0, n_claimed, 2);
           if (++st == C::KST) { st = 0; kv_phase ^= 1; }
         }
+        ++n_claimed;
       }
       // Every copy this thread started lands before the CTA may exit (their
       // barriers complete on their own; the waits are bounded regardless).
@@ -359,6 +380,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     int uslot = 0;
     uint32_t uphase = 0;
     bool first_unit_m = true;
+    int n_units_m = 0;
+    (void)n_units_m;
     while (ok) {
       if (!wait_all(B_UFULL + uslot, uphase)) break;
       const int tk = unit_ring[uslot];
@@ -368,6 +391,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       const bool u_first = first_unit_m;
       first_unit_m = false;
       (void)u_first;
+      FA_TRU(lane == 0, 1, n_units_m, 0);
       const Unit w = decode_unit(tk, p);
       const int n[2] = {w.n0, w.n1};
       const int N = w.n0 > w.n1 ? w.n0 : w.n1;
@@ -401,15 +425,19 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               if (part == 0) FA_TR(lane == 0 && u_first, 16 + i, j - 1, 1);
               p_phase[2 * i + part] ^= 1;
               tc_fence_after();
-#pragma unroll
-              for (int e = 0; e < 4; ++e) {
-                const int kk = ((e >> 1) << 2) + 2 * part + (e & 1);  // 2q, 2q+1, 4+2q, 5+2q
-                mma_ts_elect(tO[i], tS[i] + (kk >> 2) * 64 + (kk & 3) * 8,
-                             dV + (uint64_t)((kk * 16 * 128) >> 4), IDESC_PV, (part == 0 && e == 0) ? acc0 : 1u);
-              }
+              // k-steps 2q, 2q+1 (keys of half 0) and 4+2q, 5+2q (half 1)
+              const int k0 = 2 * part, k1 = 2 * part + 1, k2 = 4 + 2 * part, k3 = 5 + 2 * part;
+              mma_ts4_elect(tO[i], tS[i] + (k0 >> 2) * 64 + (k0 & 3) * 8, dV + (uint64_t)((k0 * 2048) >> 4),
+                            tS[i] + (k1 >> 2) * 64 + (k1 & 3) * 8, dV + (uint64_t)((k1 * 2048) >> 4),
+                            tS[i] + (k2 >> 2) * 64 + (k2 & 3) * 8, dV + (uint64_t)((k2 * 2048) >> 4),
+                            tS[i] + (k3 >> 2) * 64 + (k3 & 3) * 8, dV + (uint64_t)((k3 * 2048) >> 4), IDESC_PV,
+                            part == 0 ? acc0 : 1u);
             }
             if (!ok) break;
-            if (j - 1 == n[i] - 1) mma_commit_elect(bar(B_OFULL + i));
+            if (j - 1 == n[i] - 1) {
+              mma_commit_elect(bar(B_OFULL + i));
+              FA_TRU(lane == 0, 1, n_units_m, 2 + i);
+            }
             // V_(j-1) is free once the last tile's P V has read it.
             if (i == 1 || n[1] == 0 || j - 1 >= n[1]) mma_commit_elect(bar(B_VEMPTY + st_prev));
           }
@@ -420,13 +448,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               tc_fence_after();
             }
             // S_i(j) = Q_i K_j^T
+            // d/16 k-steps, four per issue group (one 64-column chunk each)
 #pragma unroll
-            for (int k = 0; k < D / 16; ++k) {
-              const uint64_t off = (uint64_t)((((k >> 2) * C::CHUNK_BYTES) + (k & 3) * 32) >> 4);
-              mma_ss_elect(tS[i], dQ[i] + off, dK + off, IDESC_S, k > 0 ? 1u : 0u);
+            for (int c = 0; c < C::CHUNKS; ++c) {
+              const uint64_t o0 = (uint64_t)((c * C::CHUNK_BYTES) >> 4);
+              mma_ss4_elect(tS[i], dQ[i] + o0, dK + o0, dQ[i] + o0 + 2, dK + o0 + 2, dQ[i] + o0 + 4, dK + o0 + 4,
+                            dQ[i] + o0 + 6, dK + o0 + 6, IDESC_S, c > 0 ? 1u : 0u);
             }
             mma_commit_elect(bar(B_SFULL + i));
             FA_TR(lane == 0 && u_first, 16 + i, j, 2);
+            if (j == 0) FA_TRU(lane == 0, 1, n_units_m, 4 + i);
             if (j == n[i] - 1) mma_commit_elect(bar(B_QEMPTY + i));
           }
         }
@@ -439,6 +470,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           if (++st == C::KST) { st = 0; kv_phase ^= 1; }
         }
       }
+      ++n_units_m;
     }
     // Let every MMA this warp issued finish before the CTA frees TMEM.
     mma_commit_elect(bar(B_DRAIN));
@@ -477,6 +509,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     int uslot = 0;
     uint32_t uphase = 0;
     bool first_unit = true;
+    int n_units_s = 0;
+    (void)n_units_s;
     while (ok) {
       ok = __all_sync(0xffffffffu, mbar_wait(bar(B_UFULL + uslot), uphase, wctx));
       if (!ok) break;
@@ -484,6 +518,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       mbar_arrive_warp(bar(B_UEMPTY + uslot));
       if (++uslot == C::UNIT_SLOTS) { uslot = 0; uphase ^= 1; }
       if (tk < 0) break;
+      FA_TRU(warp == 0 && lane == 0, 2, n_units_s, 0);
       const Unit w = decode_unit(tk, p);
       const int n = tile ? w.n1 : w.n0;
       const bool this_first = first_unit;
@@ -498,6 +533,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SFULL + tile), s_phase, wctx));
         if (!ok) break;
         FA_TR(this_first && lane == 0, warp, j, 0);
+        FA_TRU(warp == 0 && lane == 0 && j == 0, 2, n_units_s, 1);
         s_phase ^= 1;
         tc_fence_after();
         const int col0 = j * TC_BN + 64 * half;
@@ -675,6 +711,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         m_ref = m_new;
         l = l * corr + sum;
         FA_TR(this_first && lane == 0, warp, j, 6);
+        FA_TRU(warp == 0 && lane == 0 && j == n - 1, 2, n_units_s, 2);
       }
       if (!ok) break;
       // ---------------------------------------------------------- epilogue
@@ -686,6 +723,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OFULL + tile), o_phase, wctx));
       if (!ok) break;
       o_phase ^= 1;
+      FA_TRU(warp == 0 && lane == 0, 2, n_units_s, 3);
       tc_fence_after();
       const float inv_l = 1.f / l;
       const bool valid = row < p.Nq;
@@ -715,6 +753,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       if (valid && half == 0 && p.lse != nullptr) {
         p.lse[((long long)w.b * p.H + w.h) * p.Nq + row] = (m_ref + __log2f(l)) * 0.69314718055994530942f;
       }
+      FA_TRU(warp == 0 && lane == 0, 2, n_units_s, 4);
+      ++n_units_s;
     }
     // Any tcgen05.st of this thread has completed before the CTA frees TMEM.
     tmem_wait_st();

@@ -84,7 +84,11 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   while (true) {
-    if (mbar_try_wait_sleep(bar, parity, 50000u)) return true;
+#ifdef FA_WAIT_SLEEP
+    if (mbar_try_wait_sleep(bar, parity, FA_WAIT_SLEEP)) return true;
+#else
+    if (mbar_try_wait(bar, parity)) return true;
+#endif
     if (*ctx.abort_flag) return false;
     if (globaltimer_ns() - t0 > ctx.timeout_ns) {
       *ctx.abort_flag = 1;
@@ -204,6 +208,37 @@ __device__ __forceinline__ void mma_ts_elect(uint32_t d_tmem, uint32_t a_tmem, u
       "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// Four MMAs under one elect.sync (fewer instructions on the issuing warp).
+// The first accumulates into D when acc0 != 0, the other three always do.
+__device__ __forceinline__ void mma_ss4_elect(uint32_t d_tmem, uint64_t a0, uint64_t b0, uint64_t a1, uint64_t b1,
+                                              uint64_t a2, uint64_t b2, uint64_t a3, uint64_t b3, uint32_t idesc,
+                                              uint32_t acc0) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %10, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %9, p;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %3, %4, %9, 1;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %5, %6, %9, 1;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %7, %8, %9, 1;\n\t}" ::"r"(d_tmem),
+      "l"(a0), "l"(b0), "l"(a1), "l"(b1), "l"(a2), "l"(b2), "l"(a3), "l"(b3), "r"(idesc), "r"(acc0)
+      : "memory");
+}
+__device__ __forceinline__ void mma_ts4_elect(uint32_t d_tmem, uint32_t a0, uint64_t b0, uint32_t a1, uint64_t b1,
+                                              uint32_t a2, uint64_t b2, uint32_t a3, uint64_t b3, uint32_t idesc,
+                                              uint32_t acc0) {
+  asm volatile(
+      "{\n\t.reg .pred p, e;\n\t"
+      "elect.sync _|e, 0xffffffff;\n\t"
+      "setp.ne.b32 p, %10, 0;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %9, p;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%3], %4, %9, 1;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%5], %6, %9, 1;\n\t"
+      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%7], %8, %9, 1;\n\t}" ::"r"(d_tmem),
+      "r"(a0), "l"(b0), "r"(a1), "l"(b1), "r"(a2), "l"(b2), "r"(a3), "l"(b3), "r"(idesc), "r"(acc0)
+      : "memory");
+}
+
 __device__ __forceinline__ void mma_commit_elect(uint32_t bar) {
   asm volatile(
       "{\n\t.reg .pred e;\n\t"

@@ -112,9 +112,9 @@ struct TcCfg {
   static constexpr int OFF_V = OFF_K + KST * TILE_BYTES;    // KST V tiles
   static constexpr int OFF_RED = OFF_V + KST * TILE_BYTES;  // [tile][parity][half][row] fp32 exchange
   static constexpr int RED_BYTES = 2 * 2 * 2 * TC_BM * 4;
-  static constexpr int OFF_UNIT = OFF_RED + RED_BYTES;      // unit-ticket ring (UNIT_SLOTS ints)
+  static constexpr int OFF_UNIT = OFF_RED + RED_BYTES;      // ring of decoded work units (8 ints each)
   static constexpr int UNIT_SLOTS = 4;
-  static constexpr int OFF_BAR = OFF_UNIT + 16 * UNIT_SLOTS;  // barriers
+  static constexpr int OFF_BAR = OFF_UNIT + 32 * UNIT_SLOTS;  // barriers
   static constexpr int NBAR = 2 + 2 + 4 * KST + 2 + 4 + 2 + 1 + 2 + 2 * UNIT_SLOTS;
   static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 /*tmem slot + abort*/ + 1024 /*align slack*/;
   static constexpr int TMEM_S0 = 0, TMEM_S1 = 128, TMEM_O0 = 256, TMEM_O1 = 256 + D;
@@ -228,6 +228,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
+  // Unit ring slot: ticket (-1 = no more work) and the decoded unit.
+  auto ring_put = [&](int slot, int tk, const Unit& w) {
+    volatile int* e = unit_ring + 8 * slot;
+    e[0] = tk; e[1] = w.b; e[2] = w.h; e[3] = w.qt0; e[4] = w.active1; e[5] = w.n0; e[6] = w.n1;
+  };
+  auto ring_get = [&](int slot, Unit& w) -> int {
+    volatile const int* e = unit_ring + 8 * slot;
+    w.b = e[1]; w.h = e[2]; w.qt0 = e[3]; w.active1 = e[4]; w.n0 = e[5]; w.n1 = e[6];
+    return e[0];
+  };
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -293,15 +303,16 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       (void)n_claimed;
       while (ok) {
         // claim the next ticket and hand it to the other roles
+        // (decoded here once: its integer divisions stay off the other roles)
         const unsigned int t = atomicAdd(&p.sched->next, 1u);
         const int tk = (t < (unsigned int)p.n_units) ? (int)t : -1;
+        const Unit w = decode_unit(tk < 0 ? 0 : tk, p);
         if (!mbar_wait(bar(B_UEMPTY + uslot), uphase ^ 1, wctx)) break;
-        unit_ring[uslot] = tk;
+        ring_put(uslot, tk, w);
         mbar_arrive(bar(B_UFULL + uslot));
         if (++uslot == C::UNIT_SLOTS) { uslot = 0; uphase ^= 1; }
         if (tk < 0) break;
         FA_TRU(true, 0, n_claimed, 0);
-        const Unit w = decode_unit(tk, p);
         for (int i = 0; i < 2 && ok; ++i) {
           if (i == 1 && !w.active1) break;
           if (!mbar_wait(bar(B_QEMPTY + i), q_phase[i] ^ 1, wctx)) { ok = false; break; }
@@ -384,7 +395,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     (void)n_units_m;
     while (ok) {
       if (!wait_all(B_UFULL + uslot, uphase)) break;
-      const int tk = unit_ring[uslot];
+      Unit w;
+      const int tk = ring_get(uslot, w);
       mbar_arrive_warp(bar(B_UEMPTY + uslot));
       if (++uslot == C::UNIT_SLOTS) { uslot = 0; uphase ^= 1; }
       if (tk < 0) break;
@@ -392,7 +404,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       first_unit_m = false;
       (void)u_first;
       FA_TRU(lane == 0, 1, n_units_m, 0);
-      const Unit w = decode_unit(tk, p);
       const int n[2] = {w.n0, w.n1};
       const int N = w.n0 > w.n1 ? w.n0 : w.n1;
       for (int i = 0; i < 2 && ok; ++i) {
@@ -421,17 +432,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             const uint32_t acc0 = (j - 1 > 0) ? 1u : 0u;
 #pragma unroll
             for (int part = 0; part < 2; ++part) {
+              // k-steps 2q, 2q+1 (keys of half 0) and 4+2q, 5+2q (half 1);
+              // operands formed before the wait
+              const int k0 = 2 * part, k1 = 2 * part + 1, k2 = 4 + 2 * part, k3 = 5 + 2 * part;
+              const uint32_t a0 = tS[i] + (k0 >> 2) * 64 + (k0 & 3) * 8, a1 = tS[i] + (k1 >> 2) * 64 + (k1 & 3) * 8,
+                             a2 = tS[i] + (k2 >> 2) * 64 + (k2 & 3) * 8, a3 = tS[i] + (k3 >> 2) * 64 + (k3 & 3) * 8;
+              const uint64_t b0 = dV + (uint64_t)((k0 * 2048) >> 4), b1 = dV + (uint64_t)((k1 * 2048) >> 4),
+                             b2 = dV + (uint64_t)((k2 * 2048) >> 4), b3 = dV + (uint64_t)((k3 * 2048) >> 4);
               if (!wait_all(B_PFULL + 2 * i + part, p_phase[2 * i + part])) { ok = false; break; }
               if (part == 0) FA_TR(lane == 0 && u_first, 16 + i, j - 1, 1);
               p_phase[2 * i + part] ^= 1;
               tc_fence_after();
-              // k-steps 2q, 2q+1 (keys of half 0) and 4+2q, 5+2q (half 1)
-              const int k0 = 2 * part, k1 = 2 * part + 1, k2 = 4 + 2 * part, k3 = 5 + 2 * part;
-              mma_ts4_elect(tO[i], tS[i] + (k0 >> 2) * 64 + (k0 & 3) * 8, dV + (uint64_t)((k0 * 2048) >> 4),
-                            tS[i] + (k1 >> 2) * 64 + (k1 & 3) * 8, dV + (uint64_t)((k1 * 2048) >> 4),
-                            tS[i] + (k2 >> 2) * 64 + (k2 & 3) * 8, dV + (uint64_t)((k2 * 2048) >> 4),
-                            tS[i] + (k3 >> 2) * 64 + (k3 & 3) * 8, dV + (uint64_t)((k3 * 2048) >> 4), IDESC_PV,
-                            part == 0 ? acc0 : 1u);
+              mma_ts4_elect(tO[i], a0, b0, a1, b1, a2, b2, a3, b3, IDESC_PV, part == 0 ? acc0 : 1u);
             }
             if (!ok) break;
             if (j - 1 == n[i] - 1) {
@@ -514,12 +526,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
     while (ok) {
       ok = __all_sync(0xffffffffu, mbar_wait(bar(B_UFULL + uslot), uphase, wctx));
       if (!ok) break;
-      const int tk = unit_ring[uslot];
+      Unit w;
+      const int tk = ring_get(uslot, w);
       mbar_arrive_warp(bar(B_UEMPTY + uslot));
       if (++uslot == C::UNIT_SLOTS) { uslot = 0; uphase ^= 1; }
       if (tk < 0) break;
       FA_TRU(warp == 0 && lane == 0, 2, n_units_s, 0);
-      const Unit w = decode_unit(tk, p);
       const int n = tile ? w.n1 : w.n0;
       const bool this_first = first_unit;
       first_unit = false;
@@ -546,18 +558,34 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           float s[64];
           tmem_ld64(tS, s);
           FA_TR(this_first && lane == 0, warp, j, 1);
-          if (need_mask) {
-#pragma unroll
-            for (int c = 0; c < 64; ++c)
-              if (col0 + c >= lim_c) s[c] = -INFINITY;
-          }
           float mx[4];
+          if (!need_mask) {
 #pragma unroll
-          for (int t = 0; t < 4; ++t) mx[t] = fmaxf(s[t], s[t + 4]);
+            for (int t = 0; t < 4; ++t) mx[t] = fmaxf(s[t], s[t + 4]);
 #pragma unroll
-          for (int c = 8; c < 64; c += 8)
+            for (int c = 8; c < 64; c += 8)
 #pragma unroll
-            for (int t = 0; t < 4; ++t) mx[t] = fmax3(mx[t], s[c + t], s[c + 4 + t]);
+              for (int t = 0; t < 4; ++t) mx[t] = fmax3(mx[t], s[c + t], s[c + 4 + t]);
+          } else {
+            // 16-key groups: skipped when masked for every row of the warp,
+            // compared key by key only when partly visible.
+#pragma unroll
+            for (int t = 0; t < 4; ++t) mx[t] = -INFINITY;
+#pragma unroll
+            for (int g = 0; g < 4; ++g) {
+              const int k0 = col0 + 16 * g;
+              if (__all_sync(0xffffffffu, k0 >= lim_c)) continue;
+              if (!__all_sync(0xffffffffu, k0 + 16 <= lim_c)) {
+#pragma unroll
+                for (int c = 0; c < 16; ++c)
+                  if (k0 + c >= lim_c) s[16 * g + c] = -INFINITY;
+              }
+#pragma unroll
+              for (int t = 0; t < 4; ++t) mx[t] = fmax3(mx[t], s[16 * g + t], s[16 * g + 4 + t]);
+#pragma unroll
+              for (int t = 0; t < 4; ++t) mx[t] = fmax3(mx[t], s[16 * g + 8 + t], s[16 * g + 12 + t]);
+            }
+          }
           mt = fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3]));
         }
         // pass 2 re-reads the scores (tensor-memory reads are cheap, registers
@@ -596,11 +624,27 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         // 8 score pairs -> 8 packed P columns, written over this half's first
         // 32 S columns (already read).  On tiles without masked scores one
         // pair in TC_POLY_EVERY takes 2^x on the FMA pipe.
+        // On tiles with masked scores (never the polynomial form) a group
+        // masked for every row of the warp writes zeros without exps, and a
+        // partly visible group masks key by key.
         auto sub = [&](const float* sc, int cbase, auto use_poly) {
           uint32_t pk[8];
+          const int k0 = col0 + cbase;
+          if (!decltype(use_poly)::value && __all_sync(0xffffffffu, k0 >= lim_c)) {
+#pragma unroll
+            for (int t = 0; t < 8; ++t) pk[t] = 0u;
+            tmem_st8(tS + cbase / 2, pk);
+            return;
+          }
+          const bool part = !decltype(use_poly)::value && !__all_sync(0xffffffffu, k0 + 16 <= lim_c);
 #pragma unroll
           for (int t = 0; t < 8; ++t) {
-            const uint64_t x2 = f2_fma(f2_pack(sc[2 * t], sc[2 * t + 1]), scale2, negm2);
+            float v0 = sc[2 * t], v1 = sc[2 * t + 1];
+            if (part) {
+              if (k0 + 2 * t >= lim_c) v0 = -INFINITY;
+              if (k0 + 2 * t + 1 >= lim_c) v1 = -INFINITY;
+            }
+            const uint64_t x2 = f2_fma(f2_pack(v0, v1), scale2, negm2);
             float p0, p1;
             if (decltype(use_poly)::value && (t % TC_POLY_EVERY) == TC_POLY_EVERY - 1) {
               exp2_poly_x2(x2, p0, p1);
@@ -615,16 +659,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           }
           tmem_st8(tS + cbase / 2, pk);
         };
-        auto mask32 = [&](float(&sc)[32], int cbase) {
-          if (need_mask) {
-#pragma unroll
-            for (int c = 0; c < 32; ++c)
-              if (col0 + cbase + c >= lim_c) sc[c] = -INFINITY;
-          }
-        };
         // part 0: this half's keys 0-31 (columns 32-63 load meanwhile)
         tmem_ld_wait32(sa);
-        mask32(sa, 0);
         tmem_ld32_issue(tS + 32, sb);
         if (need_mask) {
           sub(sa, 0, std::false_type{});
@@ -646,11 +682,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           }
         }
         FA_TR(this_first && lane == 0, warp, j, 7);
-        const float corr = moved ? ex2(m_ref - m_new) : 1.f;  // 0 when m_ref = -inf
         // Rescale this half of O in place when this warp moved any row's
         // reference max, before this step's P V touches O (O is quiescent:
-        // its last P V finished before S_i(j) was signalled).
+        // its last P V finished before S_i(j) was signalled).  The factor
+        // (and the SFU op) is only formed when a reference moved.
         if (j > 0 && __any_sync(0xffffffffu, moved)) {
+          const float corr = moved ? ex2(m_ref - m_new) : 1.f;
 #pragma unroll 1
           for (int c = 0; c < D / 2; c += 32) {
             float ov[32];
@@ -671,7 +708,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         // part 1: keys 32-63
         tmem_ld_wait32(sb);
-        mask32(sb, 32);
         if (need_mask) {
           sub(sb, 32, std::false_type{});
           sub(sb + 16, 48, std::false_type{});
@@ -708,8 +744,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         tmem_wait_st();
         tc_fence_before();
         if (p.fault_mode != 1) mbar_arrive_warp(bar(B_PFULL + 2 * tile + 1));
+        if (moved) l *= ex2(m_ref - m_new);  // 0 when m_ref = -inf
         m_ref = m_new;
-        l = l * corr + sum;
+        l += sum;
         FA_TR(this_first && lane == 0, warp, j, 6);
         FA_TRU(warp == 0 && lane == 0 && j == n - 1, 2, n_units_s, 2);
       }

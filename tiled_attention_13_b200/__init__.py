@@ -10,7 +10,9 @@ CPU path: when the library is missing, every call raises.
 CUDA tensors, allocates O and LSE with torch (PyTorch is used for device
 memory and streams only) and launches on the current stream.
 ``forward_host(...)`` is the end-to-end form: pinned host tensors in, host
-tensors out, with the copies on the same stream.
+tensors out, with the copies on the same stream.  ``HostPipeline`` runs a
+sequence of such calls with the host<->device copies of neighbouring calls
+overlapping the computation (separate copy streams, two device buffer sets).
 """
 
 from __future__ import annotations
@@ -23,7 +25,7 @@ __all__ = [
     "FA_LAYOUT_BHND", "FA_LAYOUT_BSND", "FA_DTYPE_BF16", "FA_DTYPE_FP16", "FA_DTYPE_FP32",
     "FaError", "lib", "lib_path", "fa_fwd", "fa_fwd_noalloc", "fa_status_string", "fa_get_device_status",
     "fa_set_wait_timeout_us", "fa_debug_set_fault", "fa_abi_version", "forward", "forward_host",
-    "EXPORTED",
+    "HostForward", "HostPipeline", "EXPORTED",
 ]
 
 FA_LAYOUT_BHND, FA_LAYOUT_BSND = 0, 1
@@ -198,6 +200,74 @@ class HostForward:
         self.o_host.copy_(self.od, non_blocking=True)
         self.lse_host.copy_(self.lsed, non_blocking=True)
         return self.o_host, self.lse_host
+
+
+class HostPipeline:
+    """End-to-end calls over pinned host tensors, pipelined across calls.
+
+    ``submit(q, k, v, o, lse)`` queues one call: the host->device copy of
+    q, k, v (pinned host tensors) on an upload stream, fa_fwd on a compute
+    stream, and the device->host copy of O and LSE into the pinned host
+    tensors ``o`` and ``lse`` on a download stream.  Two device buffer sets
+    alternate, and events order each set's reuse, so call i+1's upload and
+    call i-1's download run while call i computes.  ``synchronize()`` waits
+    for every queued call; a host output is valid once it has returned.
+    """
+
+    def __init__(self, q_host, k_host, causal=False, scale=None, layout="BHND", device="cuda", slots=2):
+        import torch
+
+        self.causal, self.scale, self.layout = causal, scale, layout
+        self.dev = torch.device(device)
+        B, H, Nq, _, _ = _dims(q_host, k_host, layout)
+        self.bufs = []
+        for _ in range(slots):
+            qd = torch.empty_like(q_host, device=self.dev)
+            kd = torch.empty_like(k_host, device=self.dev)
+            vd = torch.empty_like(k_host, device=self.dev)
+            od = torch.empty_like(qd)
+            lsed = torch.empty((B, H, Nq), dtype=torch.float32, device=self.dev)
+            self.bufs.append((qd, kd, vd, od, lsed))
+        self.up = torch.cuda.Stream(self.dev)
+        self.comp = torch.cuda.Stream(self.dev)
+        self.down = torch.cuda.Stream(self.dev)
+        ev = lambda: [torch.cuda.Event() for _ in range(slots)]  # noqa: E731
+        self.uploaded, self.computed, self.downloaded = ev(), ev(), ev()
+        self.used = [False] * slots
+        self.i = 0
+        self.h2d_bytes = (q_host.numel() + 2 * k_host.numel()) * q_host.element_size()
+        self.d2h_bytes = q_host.numel() * q_host.element_size() + B * H * Nq * 4
+
+    def submit(self, q_host, k_host, v_host, o_host, lse_host):
+        import torch
+
+        s = self.i % len(self.bufs)
+        qd, kd, vd, od, lsed = self.bufs[s]
+        with torch.cuda.stream(self.up):
+            if self.used[s]:
+                self.up.wait_event(self.computed[s])  # the slot's inputs were read
+            qd.copy_(q_host, non_blocking=True)
+            kd.copy_(k_host, non_blocking=True)
+            vd.copy_(v_host, non_blocking=True)
+            self.uploaded[s].record(self.up)
+        with torch.cuda.stream(self.comp):
+            self.comp.wait_event(self.uploaded[s])
+            if self.used[s]:
+                self.comp.wait_event(self.downloaded[s])  # the slot's outputs were read back
+            forward(qd, kd, vd, causal=self.causal, scale=self.scale, layout=self.layout, out=od, lse=lsed,
+                    stream=self.comp.cuda_stream)
+            self.computed[s].record(self.comp)
+        with torch.cuda.stream(self.down):
+            self.down.wait_event(self.computed[s])
+            o_host.copy_(od, non_blocking=True)
+            lse_host.copy_(lsed, non_blocking=True)
+            self.downloaded[s].record(self.down)
+        self.used[s] = True
+        self.i += 1
+
+    def synchronize(self):
+        for st in (self.up, self.comp, self.down):
+            st.synchronize()
 
 
 def forward_host(q_host, k_host, v_host, causal=False, scale=None, layout="BHND", device="cuda"):

@@ -764,27 +764,52 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       tc_fence_after();
       const float inv_l = 1.f / l;
       const bool valid = row < p.Nq;
-      T* orow = nullptr;
-      if (valid) {
-        const long long ridx = p.bsnd ? ((long long)w.b * p.Nq + row) * p.H + w.h
-                                      : ((long long)w.b * p.H + w.h) * p.Nq + row;
-        orow = reinterpret_cast<T*>(p.o) + ridx * D + (D / 2) * half;
-      }
-#pragma unroll 1
+      // This half row of O as bf16/fp16 pairs: 16-byte chunk k = pk[4k..4k+3].
+      constexpr int NC = D / 16;  // chunks per half row: 8 (d=128) or 4 (d=64)
+      uint32_t pk[D / 4];
+#pragma unroll
       for (int c = 0; c < D / 2; c += 32) {
         float ov[32];
         tmem_ld32(tO + c, ov);
-        if (valid) {
-          uint4* dst = reinterpret_cast<uint4*>(orow + c);
 #pragma unroll
-          for (int q4 = 0; q4 < 4; ++q4) {
-            uint4 pkt;
-            pkt.x = Pack<T>::two(ov[q4 * 8 + 0] * inv_l, ov[q4 * 8 + 1] * inv_l);
-            pkt.y = Pack<T>::two(ov[q4 * 8 + 2] * inv_l, ov[q4 * 8 + 3] * inv_l);
-            pkt.z = Pack<T>::two(ov[q4 * 8 + 4] * inv_l, ov[q4 * 8 + 5] * inv_l);
-            pkt.w = Pack<T>::two(ov[q4 * 8 + 6] * inv_l, ov[q4 * 8 + 7] * inv_l);
-            dst[q4] = pkt;
+        for (int t = 0; t < 16; ++t) pk[c / 2 + t] = Pack<T>::two(ov[2 * t] * inv_l, ov[2 * t + 1] * inv_l);
+      }
+      // Transpose the chunks within groups of NC lanes (XOR butterfly over
+      // shuffles): lane i of a group then holds chunk i of each of the
+      // group's NC rows, so that one store instruction writes whole
+      // contiguous row segments instead of 32 scattered 16-byte pieces.
+      auto stage = [&](auto DDc) {
+        constexpr int dd = decltype(DDc)::value;
+        const bool up = (lane & dd) != 0;
+#pragma unroll
+        for (int k = 0; k < NC; ++k) {
+          if (k & dd) continue;
+#pragma unroll
+          for (int m = 0; m < 4; ++m) {
+            const uint32_t send = up ? pk[4 * k + m] : pk[4 * (k ^ dd) + m];
+            const uint32_t recv = __shfl_xor_sync(0xffffffffu, send, dd);
+            if (up)
+              pk[4 * k + m] = recv;
+            else
+              pk[4 * (k ^ dd) + m] = recv;
           }
+        }
+      };
+      if constexpr (NC == 8) stage(std::integral_constant<int, 4>{});
+      stage(std::integral_constant<int, 2>{});
+      stage(std::integral_constant<int, 1>{});
+      {
+        const int ci = lane % NC;                                    // chunk this lane stores
+        const int rbase = qt * TC_BM + (warp & 3) * 32 + (lane / NC) * NC;  // first row of its group
+        const long long rstride = p.bsnd ? (long long)p.H * D : (long long)D;
+        T* obase = reinterpret_cast<T*>(p.o) +
+                   (p.bsnd ? ((long long)w.b * p.Nq * p.H + w.h) * D : ((long long)w.b * p.H + w.h) * p.Nq * D) +
+                   (D / 2) * half + 8 * ci;
+#pragma unroll
+        for (int k = 0; k < NC; ++k) {
+          const int rk = rbase + k;
+          if (rk < p.Nq)
+            *reinterpret_cast<uint4*>(obase + rk * rstride) = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
         }
       }
       if (valid && half == 0 && p.lse != nullptr) {

@@ -143,6 +143,29 @@ def test_host_pipeline_matches_device_calls():
     assert torch.equal(o1, outs[0][0]) and torch.equal(l1, outs[0][1])
 
 
+def test_polynomial_exp_option(tmp_path):
+    """The kernel built with FA_POLY_EVERY=4 (one exp pair in four on the FMA
+    pipe, polynomial 2^x) meets the same bars against the oracle, in a process
+    of its own that loads that build."""
+    import os
+    import subprocess
+    import sys
+
+    from tiled_attention_13_b200.build import build_variant
+
+    lib = build_variant(str(tmp_path / "libfa_poly4.so"), {"FA_POLY_EVERY": 4})
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = ("from tests.parity import compare_full\n"
+            "from tiled_attention_13_b200.inputs import Workload\n"
+            "for c in (False, True):\n"
+            "    compare_full(Workload('poly', B=2, H=3, Nq=600, Nkv=700, d=128, dtype='bf16', layout='BSND',"
+            " causal=c, seed=77))\n"
+            "print('ok')\n")
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, env={**os.environ, "FA_B200_LIB": lib},
+                       capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout[-2000:] + r.stderr[-2000:]
+
+
 # ----------------------------------------------------------------- named workloads
 def test_tiny_full():
     for name in ("tiny", "tiny-causal"):

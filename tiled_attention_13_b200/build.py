@@ -49,6 +49,17 @@ def _stale() -> bool:
     return any(os.path.getmtime(p) > t for p in inputs)
 
 
+def build_variant(out_path: str, defines: dict) -> str:
+    """Compile the library with extra preprocessor definitions (compile-time
+    kernel options, e.g. {"FA_POLY_EVERY": 4}) to ``out_path``; load it in a
+    process of its own by setting $FA_B200_LIB."""
+    cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", out_path]
+    cmd += [f"-D{k}={v}" for k, v in defines.items()]
+    cmd += [os.path.join(CSRC, s) for s in SOURCES]
+    subprocess.run(cmd, check=True)
+    return out_path
+
+
 def build(force: bool = False, verbose: bool = False) -> str:
     """Compile the library if any source is newer than it; return its path."""
     if not force and not _stale():

@@ -35,8 +35,10 @@
 //
 //   The two tiles run half a step apart (the MMA issue order staggers them):
 //   one tile's exps, on two warps per SM sub-partition, overlap the other
-//   tile's MMAs.  On tiles without masked scores one exp pair in
-//   TC_POLY_EVERY is computed on the FMA pipe instead of the SFU.
+//   tile's MMAs.  Built with FA_POLY_EVERY=n > 0, one exp pair in n of the
+//   tiles without masked scores is computed on the FMA pipe instead of the
+//   SFU (off by default: with the scores held in registers it measured
+//   slower than SFU-only exps).
 //
 //   Online softmax in the exp2 domain: x = s * scale * log2(e).  The running
 //   reference max m is only moved when a tile's max exceeds it by more than
@@ -96,9 +98,10 @@ constexpr int TC_BM = 128;                    // query rows per Q tile
 constexpr int TC_BN = 128;                    // keys per KV tile
 constexpr float TC_RESCALE_THRESHOLD = 8.0f;  // log2 units
 #ifndef FA_POLY_EVERY
-#define FA_POLY_EVERY 4
+#define FA_POLY_EVERY 0
 #endif
-constexpr int TC_POLY_EVERY = FA_POLY_EVERY;  // one exp pair in TC_POLY_EVERY on the FMA pipe
+constexpr int TC_POLY_EVERY = FA_POLY_EVERY;  // > 0: one exp pair in TC_POLY_EVERY on the FMA pipe
+constexpr int TC_POLY_MOD = TC_POLY_EVERY > 0 ? TC_POLY_EVERY : 1;
 
 
 template <int D>
@@ -552,10 +555,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const bool need_mask = (j * TC_BN + TC_BN > p.Nkv) || (p.causal && j * TC_BN + TC_BN - 1 > qt * TC_BM);
         // visible columns of this row: [.., lim_c)
         const int lim_c = p.causal ? (row + 1 < p.Nkv ? row + 1 : p.Nkv) : p.Nkv;
+        // This half's 64 scores stay in registers from the row max through the
+        // exps (a second read of them from tensor memory delayed the P stores
+        // behind it).
         float mt;
+        float s[64];
         {
-          // pass 1: this half's row max
-          float s[64];
           tmem_ld64(tS, s);
           FA_TR(this_first && lane == 0, warp, j, 1);
           float mx[4];
@@ -588,11 +593,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           }
           mt = fmax3(mx[0], mx[1], fmaxf(mx[2], mx[3]));
         }
-        // pass 2 re-reads the scores (tensor-memory reads are cheap, registers
-        // are not); the first 32 columns are already in flight during the
-        // row-max exchange and the SFU turn wait.
-        float sa[32], sb[32];
-        tmem_ld32_issue(tS, sa);
+        const float* sa = s;       // keys 0-31 of this half
+        const float* sb = s + 32;  // keys 32-63
         FA_TR(this_first && lane == 0, warp, j, 2);
         // Reference max (log2 domain).  A warp waits for the other half's
         // candidate now only when one of its rows must move the reference;
@@ -622,8 +624,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const uint64_t negm2 = f2_pack(-mref_use, -mref_use);
         uint64_t acc2[2] = {0ull, 0ull};
         // 8 score pairs -> 8 packed P columns, written over this half's first
-        // 32 S columns (already read).  On tiles without masked scores one
-        // pair in TC_POLY_EVERY takes 2^x on the FMA pipe.
+        // 32 S columns (already read).  With TC_POLY_EVERY > 0, on tiles
+        // without masked scores one pair in TC_POLY_EVERY takes 2^x on the
+        // FMA pipe.
         // On tiles with masked scores (never the polynomial form) a group
         // masked for every row of the warp writes zeros without exps, and a
         // partly visible group masks key by key.
@@ -646,7 +649,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             }
             const uint64_t x2 = f2_fma(f2_pack(v0, v1), scale2, negm2);
             float p0, p1;
-            if (decltype(use_poly)::value && (t % TC_POLY_EVERY) == TC_POLY_EVERY - 1) {
+            if (decltype(use_poly)::value && TC_POLY_EVERY > 0 && (t % TC_POLY_MOD) == TC_POLY_MOD - 1) {
               exp2_poly_x2(x2, p0, p1);
             } else {
               float x0, x1;
@@ -659,9 +662,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           }
           tmem_st8(tS + cbase / 2, pk);
         };
-        // part 0: this half's keys 0-31 (columns 32-63 load meanwhile)
-        tmem_ld_wait32(sa);
-        tmem_ld32_issue(tS + 32, sb);
+        // part 0: this half's keys 0-31
         if (need_mask) {
           sub(sa, 0, std::false_type{});
           sub(sa + 16, 16, std::false_type{});
@@ -707,7 +708,6 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           if (p.fault_mode != 1) mbar_arrive_warp(bar(B_PFULL + 2 * tile));
         }
         // part 1: keys 32-63
-        tmem_ld_wait32(sb);
         if (need_mask) {
           sub(sb, 32, std::false_type{});
           sub(sb + 16, 48, std::false_type{});

@@ -10,16 +10,20 @@
 // B200 mapping (the pages' Cube/Vector/UB design is prior art only):
 //
 //   work unit   one (batch, head, pair of 128-row Q tiles); a persistent grid
-//               of <= #SM CTAs walks the units in a static strided order,
-//               heaviest causal pairs first (longest-processing-time order).
+//               of <= #SM CTAs takes units from a per-launch ticket counter
+//               (atomicAdd), in chunks of heads whose K/V fit in L2 and,
+//               within a chunk, heaviest causal pairs first.
 //   warps 0-15  four softmax warpgroups: (tile 0, keys 0-63), (tile 0, keys
 //               64-127), (tile 1, keys 0-63), (tile 1, keys 64-127).  A thread
 //               owns one query row (= one TMEM lane) and half of its 128 scores
 //               per KV tile; the two halves of a row agree on the reference max
 //               through shared memory (lazily, see below).  Each warpgroup also
-//               writes its half of O.
+//               writes its half of O (chunks transposed across lanes by
+//               shuffles, so that stores cover whole row segments).
 //   warp 16     TMEM allocator and the MMA issuer (whole warp, elect.sync)
-//   warp 17     TMA producer (Q tiles, K/V ring of KST stages)
+//   warp 17     ticket claims and unit decode (handed to the other roles through
+//               a shared-memory ring), TMA producer (Q tiles, K/V ring of KST
+//               stages)
 //
 //   TMEM (512 columns x 128 lanes, fp32):  S0 [0,128)  S1 [128,256)
 //   O0 [256, 256+D)  O1 [256+D, 256+2D).  P_i (bf16/fp16 pairs) for keys

@@ -1,0 +1,46 @@
+"""Host-side logic of bench.py (no GPU): how many input sets rotate, and when
+the committed DRAM-traffic record may be reported."""
+
+import json
+import os
+
+import bench
+from tiled_attention_13_b200.inputs import WORKLOADS
+
+
+def test_input_sets_exceed_twice_l2():
+    for name, wl in WORKLOADS.items():
+        n = bench.n_input_sets(wl)
+        assert n >= 2, name
+        assert n * wl.bytes_min >= 2 * bench.L2_BYTES, name
+        # no more sets than needed
+        assert n == 2 or (n - 1) * wl.bytes_min < 2 * bench.L2_BYTES, name
+
+
+def test_config_names_the_rotation():
+    cfg = bench._config(WORKLOADS["cross"], 1)
+    assert "16 input sets" in cfg["l2"] and cfg["workload"] == "cross"
+
+
+def test_traffic_record_matches_kernel_source():
+    """The committed record is used only while the kernel source hash matches,
+    and only for its own workload."""
+    path = os.path.join(bench.ROOT, "profiles", "fa_fwd_tc_llama13b_8k.json")
+    rec = json.load(open(path))
+    t = bench.captured_traffic("llama13b-8k")
+    assert t == float(rec["dram_bytes_per_launch"])
+    assert 0.5 * rec["algorithmic_bytes_per_launch"] < t < 2 * rec["algorithmic_bytes_per_launch"]
+    assert bench.captured_traffic("b4-8k") is None  # no record for that workload
+
+
+def test_traffic_record_rejected_when_source_changes(tmp_path, monkeypatch):
+    root = tmp_path
+    (root / "profiles").mkdir()
+    csrc = root / "tiled_attention_13_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "fa_fwd_tc.cuh").write_text("kernel v2\n")
+    (csrc / "ptx.cuh").write_text("helpers\n")
+    rec = {"workload": "llama13b-8k", "kernel_source_sha256": "0" * 64, "dram_bytes_per_launch": 1.0}
+    (root / "profiles" / "fa_fwd_tc_llama13b_8k.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    assert bench.captured_traffic("llama13b-8k") is None

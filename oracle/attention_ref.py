@@ -151,8 +151,15 @@ def attention_rows(q_rows, k, v, rows, scale=None, causal: bool = False):
 def attention_batched(q, k, v, scale=None, causal: bool = False, layout: str = "BHND"):
     """Apply ``attention`` to every (b, h).  Layouts (page 2 input_layout):
 
-    * "BHND": q [B, H, Nq, d], k/v [B, H, Nkv, d]
-    * "BSND": q [B, Nq, H, d], k/v [B, Nkv, H, d]
+    * "BHND": q [B, H, Nq, d], k/v [B, Hkv, Nkv, d]
+    * "BSND": q [B, Nq, H, d], k/v [B, Nkv, Hkv, d]
+
+    Hkv < H is grouped-query attention (page 1, section GatherPAKVCache 的显存
+    管理逻辑: under GQA/MQA there are fewer K/V heads than query heads, and the
+    needed head is selected; page 3, section 7.3 names GQA and MQA).  The pages
+    do not fix which query heads share a K/V head; the reading taken is
+    contiguous groups: query head h uses K/V head h // (H // Hkv).  Hkv must
+    divide H; Hkv == H is ordinary multi-head attention.
 
     Returns O in the input layout and LSE [B, H, Nq] (head-major for both).
     """
@@ -166,11 +173,15 @@ def attention_batched(q, k, v, scale=None, causal: bool = False, layout: str = "
     elif layout != "BHND":
         raise ValueError(f"unknown layout {layout!r}")
     B, H, nq, _ = q.shape
+    hkv = k.shape[1]
+    if hkv < 1 or H % hkv != 0 or v.shape[1] != hkv:
+        raise ValueError(f"K/V heads ({hkv}) must divide the query heads ({H})")
+    group = H // hkv
     o = np.empty((B, H, nq, v.shape[3]))
     lse = np.empty((B, H, nq))
     for b in range(B):
         for h in range(H):
-            o[b, h], lse[b, h] = attention(q[b, h], k[b, h], v[b, h], scale, causal)
+            o[b, h], lse[b, h] = attention(q[b, h], k[b, h // group], v[b, h // group], scale, causal)
     if layout == "BSND":
         o = o.transpose(0, 2, 1, 3)
     return o, lse

@@ -279,3 +279,54 @@ def test_empty_and_invalid():
     assert o.shape == (0, 4) and lse.shape == (0,)
     with pytest.raises(ValueError):
         attention(rnd(2, 4), np.zeros((0, 4)), np.zeros((0, 4)))
+
+
+# ---------------------------------------------------------------- grouped-query attention (K/V heads < query heads)
+def test_gqa_grouping_is_contiguous_closed_form():
+    """H = 6 query heads over Hkv = 3 K/V heads with a constant value row per
+    K/V head: query heads 2g and 2g+1 must return that head's constant (a
+    strided mapping h % Hkv, or a transposed group index, gives other values)."""
+    B, H, hkv, nq, nkv, d = 1, 6, 3, 9, 11, 4
+    q, k = rnd(B, H, nq, d), rnd(B, hkv, nkv, d)
+    consts = np.array([1.5, -2.0, 7.25])
+    v = np.broadcast_to(consts[None, :, None, None], (B, hkv, nkv, d)).copy()
+    for causal in (False, True):
+        o, _ = attention_batched(q, k, v, causal=causal)
+        for h in range(H):
+            assert np.max(np.abs(o[0, h] - consts[h // 2])) <= 1e-13, h
+
+
+def test_mqa_zero_query_gives_mean_of_shared_values():
+    """One K/V head shared by every query head (MQA) with Q = 0: each row is
+    the uniform mean of the visible V rows and LSE = ln(#visible)."""
+    B, H, n, d = 2, 5, 13, 6
+    q, k, v = np.zeros((B, H, n, d)), rnd(B, 1, n, d), rnd(B, 1, n, d)
+    for causal in (False, True):
+        o, lse = attention_batched(q, k, v, causal=causal)
+        for b in range(B):
+            for i in range(n):
+                cnt = i + 1 if causal else n
+                assert np.max(np.abs(o[b, :, i] - v[b, 0, :cnt].mean(axis=0))) <= 1e-13
+                assert np.max(np.abs(lse[b, :, i] - math.log(cnt))) <= 1e-13
+
+
+@pytest.mark.parametrize("hkv", [1, 2, 4])
+@pytest.mark.parametrize("causal", [False, True])
+def test_gqa_torch_sdpa_float64_cross_check(hkv, causal):
+    """Library cross-check: torch's scaled_dot_product_attention with
+    enable_gqa (which repeats each K/V head over a contiguous block of query
+    heads), float64 on the CPU; both layouts."""
+    B, H, n, d = 2, 8, 37, 16
+    q, k, v = rnd(B, H, n, d), rnd(B, hkv, n, d), rnd(B, hkv, n, d)
+    o, _ = attention_batched(q, k, v, causal=causal)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q), torch.from_numpy(k), torch.from_numpy(v), is_causal=causal, enable_gqa=True).numpy()
+    assert np.max(np.abs(o - ref)) <= 1e-12
+    o2, _ = attention_batched(q.transpose(0, 2, 1, 3), k.transpose(0, 2, 1, 3), v.transpose(0, 2, 1, 3),
+                              causal=causal, layout="BSND")
+    assert np.array_equal(o, o2.transpose(0, 2, 1, 3))
+
+
+def test_gqa_rejects_non_dividing_kv_heads():
+    with pytest.raises(ValueError):
+        attention_batched(rnd(1, 6, 4, 4), rnd(1, 4, 4, 4), rnd(1, 4, 4, 4))

@@ -14,8 +14,10 @@ Recipe (stated in DESIGN.md as well):
   at those positions before the rounding.
 * The named workloads are the shapes the surveyed pages benchmark (LLaMA-13B
   self-attention, B=4/H=32/D=128 batched attention, a diffusion cross-attention
-  block, 128K long context).  No dataset, weights or benchmark items are used:
-  every tensor is random and only the shapes follow the pages.
+  block, 128K long context), plus a grouped-query variant of the LLaMA-13B
+  shape (8 K/V heads for its 40 query heads).  No dataset, weights or
+  benchmark items are used: every tensor is random and only the shapes follow
+  the pages.
 """
 
 from __future__ import annotations
@@ -43,6 +45,11 @@ class Workload:
     seed: int = BASE_SEED
     k_outlier: float = 0.0
     outlier_frac: float = 0.0
+    Hkv: int = 0  # K/V heads (grouped-query attention); 0 means H
+
+    @property
+    def kv_heads(self) -> int:
+        return self.Hkv if self.Hkv > 0 else self.H
 
     @property
     def flops(self) -> float:
@@ -54,14 +61,15 @@ class Workload:
     def bytes_min(self) -> int:
         """Compulsory HBM bytes: read Q, K, V once, write O and the fp32 LSE."""
         es = 4 if self.dtype == "fp32" else 2
-        return (es * self.B * self.H * self.d * (2 * self.Nq + 2 * self.Nkv)
+        return (es * self.B * self.d * (2 * self.H * self.Nq + 2 * self.kv_heads * self.Nkv)
                 + 4 * self.B * self.H * self.Nq)
 
     def q_shape(self):
         return (self.B, self.H, self.Nq, self.d) if self.layout == "BHND" else (self.B, self.Nq, self.H, self.d)
 
     def kv_shape(self):
-        return (self.B, self.H, self.Nkv, self.d) if self.layout == "BHND" else (self.B, self.Nkv, self.H, self.d)
+        hk = self.kv_heads
+        return (self.B, hk, self.Nkv, self.d) if self.layout == "BHND" else (self.B, self.Nkv, hk, self.d)
 
     def with_(self, **kw) -> "Workload":
         return replace(self, **kw)
@@ -87,6 +95,8 @@ WORKLOADS = {
     "cross": _wl("cross", 3, B=2, H=8, Nq=4096, Nkv=77, d=64),
     "long": _wl("long", 4, B=1, H=32, Nq=131072, Nkv=131072, d=128, layout="BSND", causal=True,
                 k_outlier=3.0, outlier_frac=0.01),
+    "llama13b-8k-gqa8": _wl("llama13b-8k-gqa8", 5, B=1, H=40, Hkv=8, Nq=8192, Nkv=8192, d=128, layout="BSND",
+                            causal=True),
 }
 
 

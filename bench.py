@@ -152,7 +152,7 @@ def oracle_sample(wl, rows_budget_s: float = 12.0, seed: int = 0):
     from oracle import attention
     from tiled_attention_13_b200.inputs import make_qkv
 
-    one = wl.with_(B=1, H=1)
+    one = wl.with_(B=1, H=1, Hkv=0)
     q, k, v = make_qkv(one, device="cpu")
     if wl.layout == "BSND":
         q, k, v = q[0, :, 0], k[0, :, 0], v[0, :, 0]

@@ -88,6 +88,26 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
            float scale, int causal, int layout, int dtype, void* stream);
 
 /*
+ * fa_fwd_gqa -- fa_fwd for grouped-query (and multi-query) attention: k and v
+ * hold Hkv heads, fewer than q's H (page 1, "CANN ops-transformer
+ * FlashAttentionScore", section GatherPAKVCache 的显存管理逻辑: under GQA/MQA
+ * the K/V head count is below the query head count and the needed K/V head
+ * is selected; page 3, section 7.3 names GQA and MQA).  The pages do not fix
+ * which query heads share a K/V head; here they are contiguous groups: query
+ * head h reads K/V head h / (H / Hkv).
+ *
+ *   k, v   [B,Hkv,Nkv,d] (BHND) or [B,Nkv,Hkv,d] (BSND), device memory
+ *   Hkv    K/V heads, 1 <= Hkv, H % Hkv == 0 (Hkv == H is fa_fwd, Hkv == 1 is
+ *          multi-query attention); otherwise FA_ERR_INVALID_ARG
+ *
+ * q, o and lse keep H heads.  Other arguments, ownership, the first-call
+ * allocation and errors are as for fa_fwd.
+ */
+int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
+               int64_t B, int64_t H, int64_t Hkv, int64_t Nq, int64_t Nkv, int64_t d,
+               float scale, int causal, int layout, int dtype, void* stream);
+
+/*
  * fa_fwd_noalloc -- the same computation, arguments and results as fa_fwd,
  * for callers that must never allocate device memory: code that runs inside
  * a memory pool or arena it does not own, real-time or embedded services that
@@ -152,7 +172,7 @@ uint32_t fa_set_wait_timeout_us(uint32_t us);
  */
 int fa_debug_set_fault(int mode);
 
-/* ABI version of this header, (major << 16) | minor. */
+/* ABI version of this header, (major << 16) | minor (1.1: fa_fwd_gqa). */
 int fa_abi_version(void);
 
 #ifdef __cplusplus

@@ -83,11 +83,13 @@ def compare_sampled(wl: Workload, heads, rows_per_head: int = 48, seed: int = 0,
         o, lse = run_gpu(wl, q, k, v)
     rng = np.random.default_rng(seed)
     worst_o = worst_l = 0.0
+    group = wl.H // wl.kv_heads  # query heads per K/V head (contiguous groups, as the oracle reads GQA)
     for (b, h) in heads:
+        hk = h // group
         if wl.layout == "BHND":
-            qh, kh, vh, oh = q[b, h], k[b, h], v[b, h], o[b, h]
+            qh, kh, vh, oh = q[b, h], k[b, hk], v[b, hk], o[b, h]
         else:
-            qh, kh, vh, oh = q[b, :, h], k[b, :, h], v[b, :, h], o[b, :, h]
+            qh, kh, vh, oh = q[b, :, h], k[b, :, hk], v[b, :, hk], o[b, :, h]
         rows = sample_rows(wl.Nq, rng, rows_per_head)
         idx = torch.tensor(rows, device=q.device)
         o_ref, l_ref = attention_rows(qh.index_select(0, idx).cpu(), kh.cpu(), vh.cpu(), rows,

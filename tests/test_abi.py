@@ -35,7 +35,7 @@ def test_status_strings_and_version(fa_lib):
     for code in range(8):
         assert fa.fa_status_string(code).startswith("FA_")
     assert fa.fa_status_string(99) == "FA_ERR_UNKNOWN"
-    assert fa.fa_abi_version() == (1 << 16)
+    assert fa.fa_abi_version() == (1 << 16) | 1
 
 
 def test_host_settings_roundtrip(fa_lib):
@@ -66,6 +66,22 @@ def test_validation_before_any_cuda_call(fa_lib, kw, code):
     rc = fa.fa_fwd(args["q"], args["k"], args["v"], args["o"], args["lse"], args["B"], args["H"], args["Nq"],
                    args["Nkv"], args["d"], args["scale"], args["causal"], args["layout"], args["dtype"],
                    args["stream"])
+    assert rc == code, fa.fa_status_string(rc)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(Hkv=0), 1), (dict(Hkv=-1), 1), (dict(Hkv=3), 1), (dict(Hkv=5), 1), (dict(Hkv=12), 1),
+    (dict(H=0, Hkv=0), 0), (dict(d=96), 2), (dict(q=A16 + 8), 3),
+])
+def test_gqa_validation_before_any_cuda_call(fa_lib, kw, code):
+    """fa_fwd_gqa: Hkv must be >= 1 and divide H (here H = 4); the other checks
+    are fa_fwd's, in the same order."""
+    args = dict(q=A16, k=A16, v=A16, o=A16, lse=A16, B=1, H=4, Hkv=2, Nq=10, Nkv=10, d=64, scale=-1.0, causal=0,
+                layout=0, dtype=0, stream=None)
+    args.update(kw)
+    rc = fa.fa_fwd_gqa(args["q"], args["k"], args["v"], args["o"], args["lse"], args["B"], args["H"],
+                       args["Hkv"], args["Nq"], args["Nkv"], args["d"], args["scale"], args["causal"],
+                       args["layout"], args["dtype"], args["stream"])
     assert rc == code, fa.fa_status_string(rc)
 
 

@@ -22,14 +22,22 @@ def test_config_names_the_rotation():
     assert "16 input sets" in cfg["l2"] and cfg["workload"] == "cross"
 
 
-def test_traffic_record_matches_kernel_source():
-    """The committed record is used only while the kernel source hash matches,
-    and only for its own workload."""
+def test_traffic_record_follows_kernel_source():
+    """The committed record is used only while the kernel source hash matches
+    (else the bench reports null), and only for its own workload."""
+    import hashlib
+
     path = os.path.join(bench.ROOT, "profiles", "fa_fwd_tc_llama13b_8k.json")
     rec = json.load(open(path))
+    csrc = os.path.join(bench.ROOT, "tiled_attention_13_b200", "csrc")
+    sha = hashlib.sha256(b"".join(open(os.path.join(csrc, f), "rb").read()
+                                  for f in ("fa_fwd_tc.cuh", "ptx.cuh"))).hexdigest()
     t = bench.captured_traffic("llama13b-8k")
-    assert t == float(rec["dram_bytes_per_launch"])
-    assert 0.5 * rec["algorithmic_bytes_per_launch"] < t < 2 * rec["algorithmic_bytes_per_launch"]
+    if sha == rec["kernel_source_sha256"]:
+        assert t == float(rec["dram_bytes_per_launch"])
+    else:
+        assert t is None
+    assert 0.5 < rec["dram_bytes_per_launch"] / rec["algorithmic_bytes_per_launch"] < 2
     assert bench.captured_traffic("b4-8k") is None  # no record for that workload
 
 

@@ -166,6 +166,42 @@ def test_polynomial_exp_option(tmp_path):
     assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout[-2000:] + r.stderr[-2000:]
 
 
+# ----------------------------------------------------------------- grouped-query attention
+GQA_SHAPES = [  # (B, H, Hkv, Nq, Nkv)
+    (1, 8, 1, 300, 333),
+    (2, 8, 2, 255, 257),
+    (1, 8, 4, 129, 1000),
+    (1, 6, 3, 77, 77),
+]
+
+
+@pytest.mark.parametrize("layout", ["BHND", "BSND"])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("shape", GQA_SHAPES, ids=lambda s: "x".join(map(str, s)))
+def test_gqa_bf16(shape, d, causal, layout):
+    B, H, hkv, Nq, Nkv = shape
+    wl = Workload("gqa", B=B, H=H, Hkv=hkv, Nq=Nq, Nkv=Nkv, d=d, dtype="bf16", layout=layout, causal=causal,
+                  seed=sum(shape) + d + 7)
+    compare_full(wl)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_gqa_fp16_and_fp32(causal):
+    for dt in ("fp16", "fp32"):
+        wl = Workload("gqa-" + dt, B=2, H=6, Hkv=2, Nq=200, Nkv=230, d=64, dtype=dt, layout="BSND", causal=causal,
+                      seed=91)
+        compare_full(wl)
+
+
+def test_gqa_llama13b_8k_sampled():
+    """The grouped-query bench workload (40 query heads over 8 K/V heads), in
+    the launch configuration the bench uses, on sampled rows of heads at both
+    ends of several groups."""
+    wl = WORKLOADS["llama13b-8k-gqa8"]
+    compare_sampled(wl, heads=[(0, 0), (0, 4), (0, 5), (0, 22), (0, 39)], rows_per_head=40, seed=3)
+
+
 # ----------------------------------------------------------------- named workloads
 def test_tiny_full():
     for name in ("tiny", "tiny-causal"):

@@ -23,7 +23,7 @@ import os
 
 __all__ = [
     "FA_LAYOUT_BHND", "FA_LAYOUT_BSND", "FA_DTYPE_BF16", "FA_DTYPE_FP16", "FA_DTYPE_FP32",
-    "FaError", "lib", "lib_path", "fa_fwd", "fa_fwd_noalloc", "fa_status_string", "fa_get_device_status",
+    "FaError", "lib", "lib_path", "fa_fwd", "fa_fwd_gqa", "fa_fwd_noalloc", "fa_status_string", "fa_get_device_status",
     "fa_set_wait_timeout_us", "fa_debug_set_fault", "fa_abi_version", "forward", "forward_host",
     "HostForward", "HostPipeline", "EXPORTED",
 ]
@@ -32,8 +32,8 @@ FA_LAYOUT_BHND, FA_LAYOUT_BSND = 0, 1
 FA_DTYPE_BF16, FA_DTYPE_FP16, FA_DTYPE_FP32 = 0, 1, 2
 FA_OK = 0
 
-EXPORTED = ("fa_fwd", "fa_fwd_noalloc", "fa_status_string", "fa_get_device_status", "fa_set_wait_timeout_us",
-            "fa_debug_set_fault", "fa_abi_version")
+EXPORTED = ("fa_fwd", "fa_fwd_gqa", "fa_fwd_noalloc", "fa_status_string", "fa_get_device_status",
+            "fa_set_wait_timeout_us", "fa_debug_set_fault", "fa_abi_version")
 
 _LIB = None
 
@@ -64,6 +64,9 @@ def lib() -> ctypes.CDLL:
     L.fa_fwd.restype = ctypes.c_int
     L.fa_fwd_noalloc.argtypes = L.fa_fwd.argtypes
     L.fa_fwd_noalloc.restype = ctypes.c_int
+    L.fa_fwd_gqa.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, ctypes.c_float, ctypes.c_int,
+                             ctypes.c_int, ctypes.c_int, vp]
+    L.fa_fwd_gqa.restype = ctypes.c_int
     L.fa_status_string.argtypes = [ctypes.c_int]
     L.fa_status_string.restype = ctypes.c_char_p
     L.fa_get_device_status.argtypes = [vp]
@@ -86,6 +89,13 @@ def fa_fwd(q, k, v, o, lse, B, H, Nq, Nkv, d, scale, causal, layout, dtype, stre
     """
     return lib().fa_fwd(q, k, v, o, lse, B, H, Nq, Nkv, d, float(scale), int(causal), int(layout),
                         int(dtype), stream)
+
+
+def fa_fwd_gqa(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, d, scale, causal, layout, dtype, stream) -> int:
+    """int fa_fwd_gqa(...): k and v hold Hkv heads (Hkv divides H); query head h
+    reads K/V head h / (H / Hkv)."""
+    return lib().fa_fwd_gqa(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, d, float(scale), int(causal), int(layout),
+                            int(dtype), stream)
 
 
 def fa_fwd_noalloc(q, k, v, o, lse, B, H, Nq, Nkv, d, scale, causal, layout, dtype, stream) -> int:
@@ -134,11 +144,16 @@ def _dims(q, k, layout):
     return B, H, Nq, Nkv, d
 
 
+def _kv_heads(k, layout):
+    return k.shape[1] if layout == "BHND" else k.shape[2]
+
+
 def forward(q, k, v, causal: bool = False, scale=None, layout: str = "BHND", out=None, lse=None,
             stream=None):
     """O, LSE = softmax(scale Q K^T [+causal]) V on the GPU (returns (o, lse)).
 
-    q: [B,H,Nq,d] (BHND) or [B,Nq,H,d] (BSND); k, v the same with Nkv; all
+    q: [B,H,Nq,d] (BHND) or [B,Nq,H,d] (BSND); k, v the same with Nkv and
+    Hkv heads (Hkv dividing H: grouped-query attention when Hkv < H); all
     contiguous CUDA tensors of one dtype (bf16, fp16 or fp32); d in {64, 128}.
     scale None -> 1/sqrt(d).  LSE is fp32 [B, H, Nq].
     """
@@ -159,11 +174,17 @@ def forward(q, k, v, causal: bool = False, scale=None, layout: str = "BHND", out
     if stream is None:
         stream = torch.cuda.current_stream(q.device).cuda_stream
     sc = -1.0 if scale is None else float(scale)
-    rc = fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lse.data_ptr() if lse.numel() else None,
-                B, H, Nq, Nkv, d, sc, int(bool(causal)), FA_LAYOUT_BHND if layout == "BHND" else FA_LAYOUT_BSND,
-                _dtype_code(q), stream)
+    Hkv = _kv_heads(k, layout)
+    lay = FA_LAYOUT_BHND if layout == "BHND" else FA_LAYOUT_BSND
+    lp = lse.data_ptr() if lse.numel() else None
+    if Hkv == H:
+        rc = fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lp, B, H, Nq, Nkv, d, sc,
+                    int(bool(causal)), lay, _dtype_code(q), stream)
+    else:
+        rc = fa_fwd_gqa(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lp, B, H, Hkv, Nq, Nkv, d, sc,
+                        int(bool(causal)), lay, _dtype_code(q), stream)
     if rc != FA_OK:
-        raise FaError(rc, "fa_fwd")
+        raise FaError(rc, "fa_fwd" if Hkv == H else "fa_fwd_gqa")
     return out, lse
 
 

@@ -128,12 +128,13 @@ bool make_tmap(CUtensorMap* tm, const void* base, bool bf16, bool bsnd, int64_t 
 }
 
 // (batch, head) pairs per scheduling chunk: enough that the chunk's K and V
-// (2 * Nkv * D * 2 bytes per head) stay within a comfortable share of the
-// 126 MB L2 while every CTA works on the chunk.
-int chunk_heads_for(int64_t BH, int64_t Nkv, int64_t D) {
+// (2 * Nkv * D * 2 bytes per K/V head, shared by `group` consecutive query
+// heads) stay within a comfortable share of the 126 MB L2 while every CTA
+// works on the chunk.  A whole number of groups when it holds one at all.
+int chunk_heads_for(int64_t BH, int64_t Nkv, int64_t D, int64_t group = 1) {
   const double kv_head = 4.0 * (double)Nkv * (double)D;
   const double budget = 40.0 * 1024 * 1024;
-  int64_t g = (int64_t)(budget / kv_head);
+  int64_t g = (int64_t)(budget / kv_head) * group;
   if (g < 1) g = 1;
   if (g > BH) g = BH;
   return (int)g;
@@ -141,12 +142,12 @@ int chunk_heads_for(int64_t BH, int64_t Nkv, int64_t D) {
 
 template <int D, typename T>
 int launch_tc(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
-              int64_t Nq, int64_t Nkv, float scale, int causal, bool bsnd, cudaStream_t stream,
+              int64_t Hkv, int64_t Nq, int64_t Nkv, float scale, int causal, bool bsnd, cudaStream_t stream,
               DeviceInfo& di) {
   constexpr bool BF16 = std::is_same<T, __nv_bfloat16>::value;
   CUtensorMap tq, tk, tv;
-  if (!make_tmap(&tq, q, BF16, bsnd, B, H, Nq, D) || !make_tmap(&tk, k, BF16, bsnd, B, H, Nkv, D) ||
-      !make_tmap(&tv, v, BF16, bsnd, B, H, Nkv, D))
+  if (!make_tmap(&tq, q, BF16, bsnd, B, H, Nq, D) || !make_tmap(&tk, k, BF16, bsnd, B, Hkv, Nkv, D) ||
+      !make_tmap(&tv, v, BF16, bsnd, B, Hkv, Nkv, D))
     return FA_ERR_LAUNCH;
   fa::TcParams p;
   p.o = o;
@@ -160,7 +161,8 @@ int launch_tc(const void* q, const void* k, const void* v, void* o, float* lse, 
   const int64_t units = B * H * (int64_t)p.n_pairs;
   if (units > INT32_MAX) return FA_ERR_UNSUPPORTED;
   p.n_units = (int)units;
-  p.chunk_heads = chunk_heads_for(B * H, Nkv, D);
+  p.chunk_heads = chunk_heads_for(B * H, Nkv, D, H / Hkv);
+  p.kv_group = (int)(H / Hkv);
   p.sched = di.sched + (di.launches.fetch_add(1) % kSchedSlots);
   p.timeout_ns = (uint64_t)g_timeout_us.load() * 1000ull;
   p.fault_mode = g_fault_mode.load();
@@ -172,7 +174,7 @@ int launch_tc(const void* q, const void* k, const void* v, void* o, float* lse, 
 
 template <int D>
 int launch_simt(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
-                int64_t Nq, int64_t Nkv, float scale, int causal, bool bsnd, cudaStream_t stream) {
+                int64_t Hkv, int64_t Nq, int64_t Nkv, float scale, int causal, bool bsnd, cudaStream_t stream) {
   fa::SimtParams p;
   p.q = static_cast<const float*>(q);
   p.k = static_cast<const float*>(k);
@@ -180,6 +182,7 @@ int launch_simt(const void* q, const void* k, const void* v, void* o, float* lse
   p.o = static_cast<float*>(o);
   p.lse = lse;
   p.B = (int)B; p.H = (int)H; p.Nq = (int)Nq; p.Nkv = (int)Nkv;
+  p.Hkv = (int)Hkv;
   p.bsnd = bsnd ? 1 : 0;
   p.causal = causal;
   p.scale_log2 = scale * 1.4426950408889634f;
@@ -196,9 +199,17 @@ inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintp
 
 extern "C" {
 
-int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H, int64_t Nq,
-           int64_t Nkv, int64_t d, float scale, int causal, int layout, int dtype, void* stream) {
-  if (B < 0 || H < 0 || Nq < 0 || Nkv < 0 || d <= 0) return FA_ERR_INVALID_ARG;
+}  // extern "C"
+
+namespace {
+
+// fa_fwd and fa_fwd_gqa: validation (in the order the header states), then
+// the launch.  Hkv == H is ordinary multi-head attention.
+int fwd_common(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
+               int64_t Hkv, int64_t Nq, int64_t Nkv, int64_t d, float scale, int causal, int layout, int dtype,
+               void* stream) {
+  if (B < 0 || H < 0 || Hkv < 0 || Nq < 0 || Nkv < 0 || d <= 0) return FA_ERR_INVALID_ARG;
+  if (H > 0 && (Hkv < 1 || H % Hkv != 0)) return FA_ERR_INVALID_ARG;
   if (layout != FA_LAYOUT_BHND && layout != FA_LAYOUT_BSND) return FA_ERR_INVALID_ARG;
   if (dtype != FA_DTYPE_BF16 && dtype != FA_DTYPE_FP16 && dtype != FA_DTYPE_FP32) return FA_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
@@ -222,15 +233,31 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool bsnd = layout == FA_LAYOUT_BSND;
   if (dtype == FA_DTYPE_FP32) {
-    return d == 64 ? launch_simt<64>(q, k, v, o, lse, B, H, Nq, Nkv, scale, causal, bsnd, s)
-                   : launch_simt<128>(q, k, v, o, lse, B, H, Nq, Nkv, scale, causal, bsnd, s);
+    return d == 64 ? launch_simt<64>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s)
+                   : launch_simt<128>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s);
   }
   if (dtype == FA_DTYPE_BF16) {
-    return d == 64 ? launch_tc<64, __nv_bfloat16>(q, k, v, o, lse, B, H, Nq, Nkv, scale, causal, bsnd, s, *di)
-                   : launch_tc<128, __nv_bfloat16>(q, k, v, o, lse, B, H, Nq, Nkv, scale, causal, bsnd, s, *di);
+    return d == 64
+               ? launch_tc<64, __nv_bfloat16>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s, *di)
+               : launch_tc<128, __nv_bfloat16>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s, *di);
   }
-  return d == 64 ? launch_tc<64, __half>(q, k, v, o, lse, B, H, Nq, Nkv, scale, causal, bsnd, s, *di)
-                 : launch_tc<128, __half>(q, k, v, o, lse, B, H, Nq, Nkv, scale, causal, bsnd, s, *di);
+  return d == 64 ? launch_tc<64, __half>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s, *di)
+                 : launch_tc<128, __half>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s, *di);
+}
+
+}  // namespace
+
+extern "C" {
+
+int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H, int64_t Nq,
+           int64_t Nkv, int64_t d, float scale, int causal, int layout, int dtype, void* stream) {
+  return fwd_common(q, k, v, o, lse, B, H, H, Nq, Nkv, d, scale, causal, layout, dtype, stream);
+}
+
+int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
+               int64_t Hkv, int64_t Nq, int64_t Nkv, int64_t d, float scale, int causal, int layout, int dtype,
+               void* stream) {
+  return fwd_common(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, d, scale, causal, layout, dtype, stream);
 }
 
 const char* fa_status_string(int status) {
@@ -261,7 +288,7 @@ uint32_t fa_set_wait_timeout_us(uint32_t us) {
 
 int fa_debug_set_fault(int mode) { return g_fault_mode.exchange(mode); }
 
-int fa_abi_version(void) { return (1 << 16) | 0; }
+int fa_abi_version(void) { return (1 << 16) | 1; }
 
 #ifdef FA_TRACE_UNITS
 int fa_debug_trace_units_read(unsigned long long* host, int n) {
@@ -378,6 +405,7 @@ int launch_tc_noalloc(const void* q, const void* k, const void* v, void* o, floa
   p.n_pairs = (int)((qtiles + 1) / 2);
   p.n_units = (int)(B * H * (int64_t)p.n_pairs);
   p.chunk_heads = chunk_heads_for(B * H, Nkv, D);
+  p.kv_group = 1;        // one K/V head per query head
   p.sched = nd.scratch;  // slot 0 of the static array
   p.timeout_ns = (uint64_t)g_timeout_us.load() * 1000ull;
   p.fault_mode = g_fault_mode.load();
@@ -425,8 +453,8 @@ extern "C" int fa_fwd_noalloc(const void* q, const void* k, const void* v, void*
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool bsnd = layout == FA_LAYOUT_BSND;
   if (dtype == FA_DTYPE_FP32) {  // this kernel uses no scratch at all
-    return d == 64 ? launch_simt<64>(q, k, v, o, lse, B, H, Nq, Nkv, scale, causal, bsnd, s)
-                   : launch_simt<128>(q, k, v, o, lse, B, H, Nq, Nkv, scale, causal, bsnd, s);
+    return d == 64 ? launch_simt<64>(q, k, v, o, lse, B, H, H, Nq, Nkv, scale, causal, bsnd, s)
+                   : launch_simt<128>(q, k, v, o, lse, B, H, H, Nq, Nkv, scale, causal, bsnd, s);
   }
   if (dtype == FA_DTYPE_BF16) {
     return d == 64 ? launch_tc_noalloc<64, __nv_bfloat16>(q, k, v, o, lse, B, H, Nq, Nkv, scale, causal, bsnd, s, *nd)

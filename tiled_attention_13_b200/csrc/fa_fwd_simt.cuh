@@ -26,6 +26,7 @@ struct SimtParams {
   float* o;
   float* lse;
   int B, H, Nq, Nkv;
+  int Hkv;           // K/V heads (divides H); query head h reads K/V head h / (H / Hkv)
   int bsnd, causal;
   float scale_log2;  // scale * log2(e)
   int n_qblocks;     // ceil(Nq / SIMT_ROWS)
@@ -33,6 +34,10 @@ struct SimtParams {
 
 __device__ __forceinline__ long long simt_row(const SimtParams& p, int b, int h, int n, int N) {
   return p.bsnd ? ((long long)b * N + n) * p.H + h : ((long long)b * p.H + h) * N + n;
+}
+// Row (b, K/V head hk, key n) of k or v.
+__device__ __forceinline__ long long simt_kv_row(const SimtParams& p, int b, int hk, int n) {
+  return p.bsnd ? ((long long)b * p.Nkv + n) * p.Hkv + hk : ((long long)b * p.Hkv + hk) * p.Nkv + n;
 }
 
 template <int D>
@@ -51,6 +56,7 @@ __global__ void __launch_bounds__(SIMT_THREADS) fa_fwd_simt_kernel(SimtParams p)
   const int qb = blockIdx.x % p.n_qblocks;
   const int bh = blockIdx.x / p.n_qblocks;
   const int b = bh / p.H, h = bh % p.H;
+  const int hk = h / (p.H / p.Hkv);
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int row0 = qb * SIMT_ROWS;
 
@@ -81,7 +87,7 @@ __global__ void __launch_bounds__(SIMT_THREADS) fa_fwd_simt_kernel(SimtParams p)
       const int r = idx / D, c = idx % D;
       const int n = kb + r;
       const bool in = n < p.Nkv;
-      const long long off = in ? simt_row(p, b, h, n, p.Nkv) * D + c : 0;
+      const long long off = in ? simt_kv_row(p, b, hk, n) * D + c : 0;
       Ks[r][c] = in ? p.k[off] : 0.f;
       Vs[r][c] = in ? p.v[off] : 0.f;
     }

@@ -146,6 +146,7 @@ struct TcParams {
   int n_pairs;       // ceil(ceil(Nq / 128) / 2)
   int n_units;       // B * H * n_pairs
   int chunk_heads;   // (batch, head) pairs per scheduling chunk (L2 working set)
+  int kv_group;      // query heads per K/V head: query head h reads K/V head h / kv_group
   SchedSlot* sched;  // this launch's work-ticket counter
   uint64_t timeout_ns;
   int fault_mode;
@@ -337,6 +338,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         }
         FA_TRU(true, 0, n_claimed, 1);
         const int N = w.n0 > w.n1 ? w.n0 : w.n1;
+        const int hk = w.h / p.kv_group;  // this unit's K/V head
         for (int j = 0; j < N && ok; ++j) {
           const int kv0 = j * TC_BN;
           if (!mbar_wait(bar(B_KEMPTY + st), kv_phase ^ 1, wctx)) { ok = false; break; }
@@ -344,9 +346,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           const uint32_t kdst = sbase + C::OFF_K + st * C::TILE_BYTES;
           for (int c = 0; c < C::CHUNKS; ++c) {
             if (p.bsnd)
-              tma_load_4d(kdst + c * C::CHUNK_BYTES, &tm_k, bar(B_KFULL + st), c * 64, w.h, kv0, w.b, pol_kv);
+              tma_load_4d(kdst + c * C::CHUNK_BYTES, &tm_k, bar(B_KFULL + st), c * 64, hk, kv0, w.b, pol_kv);
             else
-              tma_load_4d(kdst + c * C::CHUNK_BYTES, &tm_k, bar(B_KFULL + st), c * 64, kv0, w.h, w.b, pol_kv);
+              tma_load_4d(kdst + c * C::CHUNK_BYTES, &tm_k, bar(B_KFULL + st), c * 64, kv0, hk, w.b, pol_kv);
           }
           k_pend[st] = true; k_issued[st] = kv_phase;
           if (!mbar_wait(bar(B_VEMPTY + st), kv_phase ^ 1, wctx)) { ok = false; break; }
@@ -354,9 +356,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           const uint32_t vdst = sbase + C::OFF_V + st * C::TILE_BYTES;
           for (int c = 0; c < C::CHUNKS; ++c) {
             if (p.bsnd)
-              tma_load_4d(vdst + c * C::CHUNK_BYTES, &tm_v, bar(B_VFULL + st), c * 64, w.h, kv0, w.b, pol_kv);
+              tma_load_4d(vdst + c * C::CHUNK_BYTES, &tm_v, bar(B_VFULL + st), c * 64, hk, kv0, w.b, pol_kv);
             else
-              tma_load_4d(vdst + c * C::CHUNK_BYTES, &tm_v, bar(B_VFULL + st), c * 64, kv0, w.h, w.b, pol_kv);
+              tma_load_4d(vdst + c * C::CHUNK_BYTES, &tm_v, bar(B_VFULL + st), c * 64, kv0, hk, w.b, pol_kv);
           }
           v_pend[st] = true; v_issued[st] = kv_phase;
           FA_TRU(j == N - 1, 0, n_claimed, 2);

@@ -21,4 +21,6 @@ from .attention_ref import (  # noqa: F401
     online_softmax_step,
     resolve_scale,
     allowed_keys,
+    attention_paged,
+    gather_paged_kv,
 )

@@ -246,3 +246,49 @@ def attention_tiled_online(q, k, v, block_r: int, block_c: int, scale=None, caus
         O[r0:r1] = o / l[:, None]
         LSE[r0:r1] = m + np.log(l)
     return O, LSE
+
+
+def gather_paged_kv(cache, block_table, seq_len: int):
+    """Contiguous keys (or values) of one sequence from a paged cache.
+
+    Page 1, section GatherPAKVCache 的显存管理逻辑: the cache is stored in
+    fixed-size physical blocks; a block table translates the sequence's
+    logical block i (its keys [i*bs, (i+1)*bs)) to the physical block holding
+    them, so the blocks of one sequence need not be adjacent.  Reading of the
+    layout (the page's listing is inconsistent about which axis holds the
+    heads): ``cache`` is [num_blocks, block_size, Hkv, d]; the result is
+    [seq_len, Hkv, d], made of logical blocks 0 .. ceil(seq_len/bs) - 1 in
+    order, cut to seq_len rows.  Table entries past those blocks are not read.
+    """
+    cache = _as_f64(cache)
+    bs = cache.shape[1]
+    n_blocks = -(-seq_len // bs)
+    table = np.asarray(block_table).reshape(-1)
+    if n_blocks > table.shape[0]:
+        raise ValueError("block table shorter than the sequence")
+    rows = []
+    for i in range(n_blocks):
+        phys = int(table[i])
+        if not 0 <= phys < cache.shape[0]:
+            raise ValueError(f"block table entry {i} = {phys} out of range")
+        rows.append(cache[phys])
+    out = np.concatenate(rows, axis=0) if rows else np.zeros((0,) + cache.shape[2:])
+    return out[:seq_len]
+
+
+def attention_paged(q, k_cache, v_cache, block_tables, seq_len: int, scale=None, causal: bool = False,
+                    layout: str = "BSND"):
+    """Attention with K/V read through a paged cache: for every batch entry b,
+    K and V are ``gather_paged_kv`` of ``block_tables[b]`` (``seq_len`` keys,
+    Hkv heads), then ``attention_batched`` as for contiguous K/V (grouped-query
+    when Hkv < H).  q is [B, H, Nq, d] (BHND) or [B, Nq, H, d] (BSND); O comes
+    back in q's layout, LSE as [B, H, Nq]."""
+    tables = np.asarray(block_tables)
+    k = np.stack([gather_paged_kv(k_cache, tables[b], seq_len) for b in range(tables.shape[0])])
+    v = np.stack([gather_paged_kv(v_cache, tables[b], seq_len) for b in range(tables.shape[0])])
+    if layout == "BHND":
+        k = k.transpose(0, 2, 1, 3)
+        v = v.transpose(0, 2, 1, 3)
+    elif layout != "BSND":
+        raise ValueError(f"unknown layout {layout!r}")
+    return attention_batched(q, k, v, scale=scale, causal=causal, layout=layout)

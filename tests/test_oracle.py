@@ -25,6 +25,8 @@ from oracle import (
     attention_tiled_online,
     online_softmax_step,
     resolve_scale,
+    attention_paged,
+    gather_paged_kv,
 )
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -330,3 +332,71 @@ def test_gqa_torch_sdpa_float64_cross_check(hkv, causal):
 def test_gqa_rejects_non_dividing_kv_heads():
     with pytest.raises(ValueError):
         attention_batched(rnd(1, 6, 4, 4), rnd(1, 4, 4, 4), rnd(1, 4, 4, 4))
+
+
+# ---------------------------------------------------------------- paged K/V cache (gather through a block table)
+def _scatter_into_cache(kv, bs, perm, n_phys):
+    """Place the logical blocks of a contiguous [N, Hkv, d] sequence into the
+    physical blocks perm[i] of a fresh cache, by an explicit loop; every other
+    element of the cache (unused blocks, the tail of the last block) is NaN."""
+    n, hkv, d = kv.shape
+    cache = np.full((n_phys, bs, hkv, d), np.nan)
+    for i in range(-(-n // bs)):
+        rows = kv[i * bs:(i + 1) * bs]
+        cache[perm[i], :rows.shape[0]] = rows
+    return cache
+
+
+def test_gather_identity_table_is_a_reshape():
+    bs, nb, hkv, d = 16, 5, 2, 8
+    k = rnd(nb * bs, hkv, d)
+    cache = k.reshape(nb, bs, hkv, d)
+    assert np.array_equal(gather_paged_kv(cache, np.arange(nb), nb * bs), k)
+    assert np.array_equal(gather_paged_kv(cache, np.arange(nb), 37), k[:37])
+
+
+@pytest.mark.parametrize("seq_len", [1, 16, 45, 80])
+def test_gather_scattered_blocks_reads_only_its_rows(seq_len):
+    rng = np.random.default_rng(seq_len)
+    bs, hkv, d, n_phys = 16, 3, 4, 11
+    k = rnd(seq_len, hkv, d)
+    perm = rng.permutation(n_phys)
+    cache = _scatter_into_cache(k, bs, perm, n_phys)
+    table = np.concatenate([perm[:-(-seq_len // bs)], np.full(3, 10_000)])  # entries past the sequence are junk
+    g = gather_paged_kv(cache, table, seq_len)
+    assert np.all(np.isfinite(g)) and np.array_equal(g, k)
+
+
+def test_gather_rejects_bad_tables():
+    cache = rnd(4, 16, 1, 4)
+    with pytest.raises(ValueError):
+        gather_paged_kv(cache, np.array([0, 9]), 20)   # entry out of range
+    with pytest.raises(ValueError):
+        gather_paged_kv(cache, np.array([0]), 20)      # table too short
+
+
+@pytest.mark.parametrize("layout", ["BHND", "BSND"])
+@pytest.mark.parametrize("causal", [False, True])
+def test_attention_paged_equals_contiguous(layout, causal):
+    """Attention through a paged cache (a different block order per batch
+    entry, NaN everywhere the table does not point) equals attention on the
+    contiguous K/V, exactly."""
+    rng = np.random.default_rng(7)
+    B, H, hkv, n, d, bs = 2, 4, 2, 70, 8, 16
+    k, v = rnd(B, n, hkv, d), rnd(B, n, hkv, d)
+    nb = -(-n // bs)
+    n_phys = B * nb + 3
+    order = rng.permutation(n_phys)
+    tables = np.stack([order[b * nb:(b + 1) * nb] for b in range(B)])
+    kc = np.full((n_phys, bs, hkv, d), np.nan)
+    vc = np.full((n_phys, bs, hkv, d), np.nan)
+    for b in range(B):
+        kc_b = _scatter_into_cache(k[b], bs, tables[b], n_phys)
+        vc_b = _scatter_into_cache(v[b], bs, tables[b], n_phys)
+        used = np.isfinite(kc_b)
+        kc[used], vc[used] = kc_b[used], vc_b[used]
+    q = rnd(B, H, n, d) if layout == "BHND" else rnd(B, n, H, d)
+    kk, vv = (k, v) if layout == "BSND" else (k.transpose(0, 2, 1, 3), v.transpose(0, 2, 1, 3))
+    o_ref, l_ref = attention_batched(q, kk, vv, causal=causal, layout=layout)
+    o, lse = attention_paged(q, kc, vc, tables, n, causal=causal, layout=layout)
+    assert np.all(np.isfinite(o)) and np.array_equal(o, o_ref) and np.array_equal(lse, l_ref)

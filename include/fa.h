@@ -108,6 +108,35 @@ int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
                float scale, int causal, int layout, int dtype, void* stream);
 
 /*
+ * fa_fwd_paged -- fa_fwd_gqa with K and V read through a paged cache (page
+ * 1, section GatherPAKVCache 的显存管理逻辑: the cache is kept in fixed-size
+ * physical blocks, and a block table translates each sequence's logical
+ * blocks to the physical blocks that hold them).
+ *
+ *   k_cache, v_cache  [num_blocks, block_size, Hkv, d] device memory: block,
+ *                     then key within the block, head, feature
+ *   block_table       int32 [B, max_blocks] device memory: keys
+ *                     [i*block_size, (i+1)*block_size) of batch entry b are
+ *                     physical block block_table[b*max_blocks + i]; entries for
+ *                     i >= ceil(Nkv / block_size) are not read
+ *   Nkv               keys per sequence (the same for every batch entry)
+ *   block_size        a power of two >= 16
+ *   num_blocks        physical blocks in each cache (>= 1)
+ *   max_blocks        entries per table row, >= ceil(Nkv / block_size)
+ *   dtype             bf16 or fp16 (fp32 returns FA_ERR_UNSUPPORTED)
+ *
+ * q, o, lse (H heads, `layout`), Hkv, scale and causal are as for fa_fwd_gqa.
+ * Cache rows past Nkv in a sequence's last block are never used and may hold
+ * anything; a table entry outside [0, num_blocks) reads as zeros.  Ownership,
+ * the first-call allocation and errors are as for fa_fwd; block_table must be
+ * 4-byte aligned.
+ */
+int fa_fwd_paged(const void* q, const void* k_cache, const void* v_cache, const int* block_table, void* o,
+                 float* lse, int64_t B, int64_t H, int64_t Hkv, int64_t Nq, int64_t Nkv, int64_t d,
+                 int64_t block_size, int64_t num_blocks, int64_t max_blocks, float scale, int causal, int layout,
+                 int dtype, void* stream);
+
+/*
  * fa_fwd_noalloc -- the same computation, arguments and results as fa_fwd,
  * for callers that must never allocate device memory: code that runs inside
  * a memory pool or arena it does not own, real-time or embedded services that
@@ -172,7 +201,7 @@ uint32_t fa_set_wait_timeout_us(uint32_t us);
  */
 int fa_debug_set_fault(int mode);
 
-/* ABI version of this header, (major << 16) | minor (1.1: fa_fwd_gqa). */
+/* ABI version of this header, (major << 16) | minor (1.1: fa_fwd_gqa, 1.2: fa_fwd_paged). */
 int fa_abi_version(void);
 
 #ifdef __cplusplus

@@ -42,6 +42,13 @@ int main(void) {
   expect(fa_fwd_noalloc(a16, a16, a16, a16, l16, 1, 2, 10, 0, 64, -1.0f, 0, FA_LAYOUT_BHND, FA_DTYPE_BF16, NULL),
          FA_ERR_INVALID_ARG, "empty key set");
 
+  expect(fa_fwd_paged(a16, a16, a16, (const int*)a16, a16, l16, 1, 4, 2, 10, 100, 64, 24, 8, 4, -1.0f, 0,
+                      FA_LAYOUT_BSND, FA_DTYPE_BF16, NULL),
+         FA_ERR_INVALID_ARG, "paged block size not a power of two");
+  expect(fa_fwd_paged(a16, a16, a16, (const int*)a16, a16, l16, 1, 4, 2, 10, 100, 64, 32, 8, 4, -1.0f, 0,
+                      FA_LAYOUT_BSND, FA_DTYPE_FP32, NULL),
+         FA_ERR_UNSUPPORTED, "paged fp32");
+
   uint32_t prev = fa_set_wait_timeout_us(5000);
   expect((int)fa_set_wait_timeout_us(prev), 5000, "timeout setting round trip");
 

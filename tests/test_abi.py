@@ -35,7 +35,7 @@ def test_status_strings_and_version(fa_lib):
     for code in range(8):
         assert fa.fa_status_string(code).startswith("FA_")
     assert fa.fa_status_string(99) == "FA_ERR_UNKNOWN"
-    assert fa.fa_abi_version() == (1 << 16) | 1
+    assert fa.fa_abi_version() == (1 << 16) | 2
 
 
 def test_host_settings_roundtrip(fa_lib):
@@ -82,6 +82,27 @@ def test_gqa_validation_before_any_cuda_call(fa_lib, kw, code):
     rc = fa.fa_fwd_gqa(args["q"], args["k"], args["v"], args["o"], args["lse"], args["B"], args["H"],
                        args["Hkv"], args["Nq"], args["Nkv"], args["d"], args["scale"], args["causal"],
                        args["layout"], args["dtype"], args["stream"])
+    assert rc == code, fa.fa_status_string(rc)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(block_size=24), 1), (dict(block_size=8), 1), (dict(block_size=0), 1),
+    (dict(max_blocks=2), 1), (dict(num_blocks=0), 1), (dict(Hkv=3), 1), (dict(bt=None), 1),
+    (dict(dtype=2), 2), (dict(d=96), 2),
+    (dict(bt=A16 + 2), 3), (dict(kc=A16 + 8), 3),
+    (dict(Nq=0), 0), (dict(B=0), 0),
+])
+def test_paged_validation_before_any_cuda_call(fa_lib, kw, code):
+    """fa_fwd_paged: block size a power of two >= 16, a table row long enough
+    for Nkv (here 100 keys in blocks of 32 need 4 entries), at least one
+    physical block, bf16/fp16 only, a 4-byte aligned table."""
+    args = dict(q=A16, kc=A16, vc=A16, bt=A16, o=A16, lse=A16, B=1, H=4, Hkv=2, Nq=10, Nkv=100, d=64,
+                block_size=32, num_blocks=8, max_blocks=4, scale=-1.0, causal=0, layout=1, dtype=0, stream=None)
+    args.update(kw)
+    rc = fa.fa_fwd_paged(args["q"], args["kc"], args["vc"], args["bt"], args["o"], args["lse"], args["B"],
+                         args["H"], args["Hkv"], args["Nq"], args["Nkv"], args["d"], args["block_size"],
+                         args["num_blocks"], args["max_blocks"], args["scale"], args["causal"], args["layout"],
+                         args["dtype"], args["stream"])
     assert rc == code, fa.fa_status_string(rc)
 
 

@@ -202,6 +202,65 @@ def test_gqa_llama13b_8k_sampled():
     compare_sampled(wl, heads=[(0, 0), (0, 4), (0, 5), (0, 22), (0, 39)], rows_per_head=40, seed=3)
 
 
+# ----------------------------------------------------------------- paged K/V cache
+def _paged_parity(wl):
+    """forward_paged on a cache built from the seeded K/V (shuffled physical
+    blocks, NaN in every element the table does not point at) against the
+    oracle's gather-then-attend on the same cache and table."""
+    from oracle import attention_paged
+    from tiled_attention_13_b200.inputs import make_paged_kv
+
+    from .parity import LSE_TOL, o_bar
+
+    q, k, v = make_qkv(wl)
+    kc, vc, table = make_paged_kv(wl, k, v)
+    o, lse = fa.forward_paged(q.cuda(), kc.cuda(), vc.cuda(), table.cuda(), wl.Nkv, causal=wl.causal,
+                              layout=wl.layout)
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_status(None) == 0
+    o_ref, l_ref = attention_paged(q, kc, vc, table.numpy(), wl.Nkv, causal=wl.causal, layout=wl.layout)
+    o_gpu, l_gpu = o.double().cpu().numpy(), lse.double().cpu().numpy()
+    assert np.all(np.isfinite(o_gpu)) and np.all(np.isfinite(l_gpu))
+    assert np.all(np.abs(o_gpu - o_ref) <= o_bar(o_ref, wl.dtype)), float(np.abs(o_gpu - o_ref).max())
+    assert np.abs(l_gpu - l_ref).max() <= LSE_TOL
+
+
+@pytest.mark.parametrize("block_size", [16, 64, 128, 256])
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("d", [64, 128])
+def test_paged_bf16(block_size, d, causal):
+    wl = Workload("paged", B=2, H=8, Hkv=2, Nq=300, Nkv=300, d=d, dtype="bf16", layout="BSND", causal=causal,
+                  block_size=block_size, seed=block_size + d)
+    _paged_parity(wl)
+
+
+@pytest.mark.parametrize("layout", ["BHND", "BSND"])
+def test_paged_ragged_mha_and_fp16(layout):
+    """Nkv neither a multiple of the block size nor of 128 (the tail rows of
+    the last block are NaN in the cache), one K/V head per query head, and
+    fp16; query layout BHND and BSND."""
+    for dt, hkv in (("bf16", 3), ("fp16", 1)):
+        wl = Workload("paged-r", B=2, H=3, Hkv=hkv, Nq=129, Nkv=1000, d=128, dtype=dt, layout=layout,
+                      causal=False, block_size=32, seed=17)
+        _paged_parity(wl)
+
+
+def test_paged_llama13b_8k_sampled():
+    """The paged bench workload (16-key blocks, 40 query heads over 8 K/V
+    heads) on sampled rows: the contiguous K/V it was built from is the
+    reference input for the oracle, row by row."""
+    from tiled_attention_13_b200.inputs import make_paged_kv
+
+    wl = WORKLOADS["llama13b-8k-gqa8-paged16"]
+    q, k, v = make_qkv(wl, device="cuda")
+    kc, vc, table = make_paged_kv(wl, k, v)
+    o, lse = fa.forward_paged(q, kc, vc, table, wl.Nkv, causal=wl.causal, layout=wl.layout)
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_status(None) == 0
+    compare_sampled(wl, heads=[(0, 0), (0, 7), (0, 21), (0, 39)], rows_per_head=32, seed=5, o=o, lse=lse,
+                    qkv=(q, k, v))
+
+
 # ----------------------------------------------------------------- named workloads
 def test_tiny_full():
     for name in ("tiny", "tiny-causal"):

@@ -23,8 +23,9 @@ import os
 
 __all__ = [
     "FA_LAYOUT_BHND", "FA_LAYOUT_BSND", "FA_DTYPE_BF16", "FA_DTYPE_FP16", "FA_DTYPE_FP32",
-    "FaError", "lib", "lib_path", "fa_fwd", "fa_fwd_gqa", "fa_fwd_noalloc", "fa_status_string", "fa_get_device_status",
-    "fa_set_wait_timeout_us", "fa_debug_set_fault", "fa_abi_version", "forward", "forward_host",
+    "FaError", "lib", "lib_path", "fa_fwd", "fa_fwd_gqa", "fa_fwd_paged", "fa_fwd_noalloc", "fa_status_string",
+    "fa_get_device_status", "fa_set_wait_timeout_us", "fa_debug_set_fault", "fa_abi_version", "forward",
+    "forward_paged", "forward_host",
     "HostForward", "HostPipeline", "EXPORTED",
 ]
 
@@ -32,7 +33,7 @@ FA_LAYOUT_BHND, FA_LAYOUT_BSND = 0, 1
 FA_DTYPE_BF16, FA_DTYPE_FP16, FA_DTYPE_FP32 = 0, 1, 2
 FA_OK = 0
 
-EXPORTED = ("fa_fwd", "fa_fwd_gqa", "fa_fwd_noalloc", "fa_status_string", "fa_get_device_status",
+EXPORTED = ("fa_fwd", "fa_fwd_gqa", "fa_fwd_paged", "fa_fwd_noalloc", "fa_status_string", "fa_get_device_status",
             "fa_set_wait_timeout_us", "fa_debug_set_fault", "fa_abi_version")
 
 _LIB = None
@@ -67,6 +68,9 @@ def lib() -> ctypes.CDLL:
     L.fa_fwd_gqa.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, ctypes.c_float, ctypes.c_int,
                              ctypes.c_int, ctypes.c_int, vp]
     L.fa_fwd_gqa.restype = ctypes.c_int
+    L.fa_fwd_paged.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64, i64, i64, ctypes.c_float,
+                               ctypes.c_int, ctypes.c_int, ctypes.c_int, vp]
+    L.fa_fwd_paged.restype = ctypes.c_int
     L.fa_status_string.argtypes = [ctypes.c_int]
     L.fa_status_string.restype = ctypes.c_char_p
     L.fa_get_device_status.argtypes = [vp]
@@ -96,6 +100,14 @@ def fa_fwd_gqa(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, d, scale, causal, layout, dt
     reads K/V head h / (H / Hkv)."""
     return lib().fa_fwd_gqa(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, d, float(scale), int(causal), int(layout),
                             int(dtype), stream)
+
+
+def fa_fwd_paged(q, k_cache, v_cache, block_table, o, lse, B, H, Hkv, Nq, Nkv, d, block_size, num_blocks,
+                 max_blocks, scale, causal, layout, dtype, stream) -> int:
+    """int fa_fwd_paged(...): K/V through a paged cache [num_blocks, block_size,
+    Hkv, d] and an int32 block table [B, max_blocks]."""
+    return lib().fa_fwd_paged(q, k_cache, v_cache, block_table, o, lse, B, H, Hkv, Nq, Nkv, d, block_size,
+                              num_blocks, max_blocks, float(scale), int(causal), int(layout), int(dtype), stream)
 
 
 def fa_fwd_noalloc(q, k, v, o, lse, B, H, Nq, Nkv, d, scale, causal, layout, dtype, stream) -> int:
@@ -185,6 +197,46 @@ def forward(q, k, v, causal: bool = False, scale=None, layout: str = "BHND", out
                         int(bool(causal)), lay, _dtype_code(q), stream)
     if rc != FA_OK:
         raise FaError(rc, "fa_fwd" if Hkv == H else "fa_fwd_gqa")
+    return out, lse
+
+
+def forward_paged(q, k_cache, v_cache, block_table, seq_len: int, causal: bool = False, scale=None,
+                  layout: str = "BSND", out=None, lse=None, stream=None):
+    """O, LSE with K and V gathered through a paged cache (returns (o, lse)).
+
+    q: [B,H,Nq,d] (BHND) or [B,Nq,H,d] (BSND), bf16 or fp16; k_cache, v_cache:
+    [num_blocks, block_size, Hkv, d] of q's dtype; block_table: int32
+    [B, max_blocks] CUDA tensor; seq_len: keys per sequence.  All contiguous.
+    """
+    import torch
+
+    for t in (q, k_cache, v_cache, block_table):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, caches and block_table must be contiguous CUDA tensors")
+    if not (q.dtype == k_cache.dtype == v_cache.dtype) or k_cache.shape != v_cache.shape:
+        raise ValueError("q and the caches must share one dtype; the two caches one shape")
+    if block_table.dtype != torch.int32 or block_table.dim() != 2:
+        raise ValueError("block_table must be an int32 [B, max_blocks] tensor")
+    if layout == "BHND":
+        B, H, Nq, d = q.shape
+    elif layout == "BSND":
+        B, Nq, H, d = q.shape
+    else:
+        raise ValueError(f"layout must be 'BHND' or 'BSND', got {layout!r}")
+    num_blocks, block_size, Hkv, _ = k_cache.shape
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    sc = -1.0 if scale is None else float(scale)
+    rc = fa_fwd_paged(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_table.data_ptr(), out.data_ptr(),
+                      lse.data_ptr() if lse.numel() else None, B, H, Hkv, Nq, int(seq_len), d, block_size,
+                      num_blocks, block_table.shape[1], sc, int(bool(causal)),
+                      FA_LAYOUT_BHND if layout == "BHND" else FA_LAYOUT_BSND, _dtype_code(q), stream)
+    if rc != FA_OK:
+        raise FaError(rc, "fa_fwd_paged")
     return out, lse
 
 

@@ -74,6 +74,10 @@ int device_setup(int dev, DeviceInfo** out) {
       ok &= set_smem_attr(fa::fa_fwd_tc_kernel<128, __nv_bfloat16>, fa::TcCfg<128>::SMEM_BYTES);
       ok &= set_smem_attr(fa::fa_fwd_tc_kernel<64, __half>, fa::TcCfg<64>::SMEM_BYTES);
       ok &= set_smem_attr(fa::fa_fwd_tc_kernel<128, __half>, fa::TcCfg<128>::SMEM_BYTES);
+      ok &= set_smem_attr(fa::fa_fwd_tc_kernel<64, __nv_bfloat16, true>, fa::TcCfg<64>::SMEM_BYTES);
+      ok &= set_smem_attr(fa::fa_fwd_tc_kernel<128, __nv_bfloat16, true>, fa::TcCfg<128>::SMEM_BYTES);
+      ok &= set_smem_attr(fa::fa_fwd_tc_kernel<64, __half, true>, fa::TcCfg<64>::SMEM_BYTES);
+      ok &= set_smem_attr(fa::fa_fwd_tc_kernel<128, __half, true>, fa::TcCfg<128>::SMEM_BYTES);
       ok &= set_smem_attr(fa::fa_fwd_simt_kernel<64>, fa::simt_smem_bytes<64>());
       ok &= set_smem_attr(fa::fa_fwd_simt_kernel<128>, fa::simt_smem_bytes<128>());
       if (!ok) return FA_ERR_LAUNCH;
@@ -127,6 +131,29 @@ bool make_tmap(CUtensorMap* tm, const void* base, bool bf16, bool bsnd, int64_t 
   return r == CUDA_SUCCESS;
 }
 
+// 4-D tensor map over a paged cache [num_blocks, block_size, Hkv, D] of 16-bit
+// values: dims (D, Hkv, block_size, num_blocks), box = 64 columns x
+// min(block_size, 128) rows of one (block, head), 128-byte swizzle, reads
+// outside the cache (e.g. block index num_blocks) fill with zeros.
+bool make_tmap_paged(CUtensorMap* tm, const void* base, bool bf16, int64_t Hkv, int64_t bs, int64_t num_blocks,
+                     int64_t D) {
+  const cuuint64_t es = 2;
+  cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)bs, (cuuint64_t)num_blocks};
+  cuuint64_t strides[3] = {D * es, Hkv * D * es, bs * Hkv * D * es};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)(bs < 128 ? bs : 128), 1}, estr[4] = {1, 1, 1, 1};
+  CUresult r = g_encode(tm, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
+                        const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+// A paged K/V cache as fa_fwd_paged receives it.
+struct PagedKV {
+  const int* block_table;  // [B, max_blocks] physical block of each logical block
+  int64_t block_size, num_blocks, max_blocks;
+};
+
 // (batch, head) pairs per scheduling chunk: enough that the chunk's K and V
 // (2 * Nkv * D * 2 bytes per K/V head, shared by `group` consecutive query
 // heads) stay within a comfortable share of the 126 MB L2 while every CTA
@@ -143,12 +170,18 @@ int chunk_heads_for(int64_t BH, int64_t Nkv, int64_t D, int64_t group = 1) {
 template <int D, typename T>
 int launch_tc(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
               int64_t Hkv, int64_t Nq, int64_t Nkv, float scale, int causal, bool bsnd, cudaStream_t stream,
-              DeviceInfo& di) {
+              DeviceInfo& di, const PagedKV* pg = nullptr) {
   constexpr bool BF16 = std::is_same<T, __nv_bfloat16>::value;
   CUtensorMap tq, tk, tv;
-  if (!make_tmap(&tq, q, BF16, bsnd, B, H, Nq, D) || !make_tmap(&tk, k, BF16, bsnd, B, Hkv, Nkv, D) ||
-      !make_tmap(&tv, v, BF16, bsnd, B, Hkv, Nkv, D))
-    return FA_ERR_LAUNCH;
+  if (!make_tmap(&tq, q, BF16, bsnd, B, H, Nq, D)) return FA_ERR_LAUNCH;
+  if (pg == nullptr) {
+    if (!make_tmap(&tk, k, BF16, bsnd, B, Hkv, Nkv, D) || !make_tmap(&tv, v, BF16, bsnd, B, Hkv, Nkv, D))
+      return FA_ERR_LAUNCH;
+  } else {
+    if (!make_tmap_paged(&tk, k, BF16, Hkv, pg->block_size, pg->num_blocks, D) ||
+        !make_tmap_paged(&tv, v, BF16, Hkv, pg->block_size, pg->num_blocks, D))
+      return FA_ERR_LAUNCH;
+  }
   fa::TcParams p;
   p.o = o;
   p.lse = lse;
@@ -163,12 +196,20 @@ int launch_tc(const void* q, const void* k, const void* v, void* o, float* lse, 
   p.n_units = (int)units;
   p.chunk_heads = chunk_heads_for(B * H, Nkv, D, H / Hkv);
   p.kv_group = (int)(H / Hkv);
+  p.block_table = pg != nullptr ? pg->block_table : nullptr;
+  p.block_size = pg != nullptr ? (int)pg->block_size : 0;
+  p.max_blocks = pg != nullptr ? (int)pg->max_blocks : 0;
+  p.num_blocks = pg != nullptr ? (int)pg->num_blocks : 0;
   p.sched = di.sched + (di.launches.fetch_add(1) % kSchedSlots);
   p.timeout_ns = (uint64_t)g_timeout_us.load() * 1000ull;
   p.fault_mode = g_fault_mode.load();
   const int grid = (int)(units < di.num_sms ? units : di.num_sms);
-  fa::fa_fwd_tc_kernel<D, T><<<grid, fa::TC_THREADS, fa::TcCfg<D>::SMEM_BYTES, stream>>>(tq, tk, tv, p,
-                                                                                         di.status);
+  if (pg == nullptr)
+    fa::fa_fwd_tc_kernel<D, T, false><<<grid, fa::TC_THREADS, fa::TcCfg<D>::SMEM_BYTES, stream>>>(tq, tk, tv, p,
+                                                                                                  di.status);
+  else
+    fa::fa_fwd_tc_kernel<D, T, true><<<grid, fa::TC_THREADS, fa::TcCfg<D>::SMEM_BYTES, stream>>>(tq, tk, tv, p,
+                                                                                                 di.status);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
@@ -260,6 +301,52 @@ int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
   return fwd_common(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, d, scale, causal, layout, dtype, stream);
 }
 
+int fa_fwd_paged(const void* q, const void* k_cache, const void* v_cache, const int* block_table, void* o,
+                 float* lse, int64_t B, int64_t H, int64_t Hkv, int64_t Nq, int64_t Nkv, int64_t d,
+                 int64_t block_size, int64_t num_blocks, int64_t max_blocks, float scale, int causal, int layout,
+                 int dtype, void* stream) {
+  if (B < 0 || H < 0 || Hkv < 0 || Nq < 0 || Nkv < 0 || d <= 0 || block_size <= 0 || num_blocks < 0 ||
+      max_blocks < 0)
+    return FA_ERR_INVALID_ARG;
+  if (H > 0 && (Hkv < 1 || H % Hkv != 0)) return FA_ERR_INVALID_ARG;
+  if (layout != FA_LAYOUT_BHND && layout != FA_LAYOUT_BSND) return FA_ERR_INVALID_ARG;
+  if (dtype != FA_DTYPE_BF16 && dtype != FA_DTYPE_FP16 && dtype != FA_DTYPE_FP32) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if ((block_size & (block_size - 1)) != 0 || block_size < 16) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (dtype == FA_DTYPE_FP32) return FA_ERR_UNSUPPORTED;  // the paged path is the tensor-core kernel's
+  if (B == 0 || H == 0 || Nq == 0) return FA_OK;          // nothing to compute
+  if (Nkv == 0) return FA_ERR_INVALID_ARG;                // softmax over an empty key set
+  if (num_blocks == 0 || max_blocks < (Nkv + block_size - 1) / block_size) return FA_ERR_INVALID_ARG;
+  if (q == nullptr || k_cache == nullptr || v_cache == nullptr || block_table == nullptr || o == nullptr)
+    return FA_ERR_INVALID_ARG;
+  if (B > INT32_MAX || H > INT32_MAX || B * H > INT32_MAX || Nq > INT32_MAX - 256 || Nkv > INT32_MAX - 256 ||
+      block_size > (1 << 20) || num_blocks > INT32_MAX - 1 || max_blocks > INT32_MAX || B * max_blocks > INT32_MAX)
+    return FA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k_cache, 16) || !aligned(v_cache, 16) || !aligned(o, 16) ||
+      !aligned(block_table, 4) || (lse != nullptr && !aligned(lse, 4)))
+    return FA_ERR_MISALIGNED;
+  if (!(scale > 0.f) || std::isinf(scale)) scale = 1.0f / std::sqrt((float)d);
+
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_NO_DEVICE;
+  DeviceInfo* di = nullptr;
+  const int st = device_setup(dev, &di);
+  if (st != FA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool bsnd = layout == FA_LAYOUT_BSND;
+  const PagedKV pg{block_table, block_size, num_blocks, max_blocks};
+  if (dtype == FA_DTYPE_BF16)
+    return d == 64 ? launch_tc<64, __nv_bfloat16>(q, k_cache, v_cache, o, lse, B, H, Hkv, Nq, Nkv, scale, causal,
+                                                  bsnd, s, *di, &pg)
+                   : launch_tc<128, __nv_bfloat16>(q, k_cache, v_cache, o, lse, B, H, Hkv, Nq, Nkv, scale, causal,
+                                                   bsnd, s, *di, &pg);
+  return d == 64 ? launch_tc<64, __half>(q, k_cache, v_cache, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s,
+                                         *di, &pg)
+                 : launch_tc<128, __half>(q, k_cache, v_cache, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s,
+                                          *di, &pg);
+}
+
 const char* fa_status_string(int status) {
   switch (status) {
     case FA_OK: return "FA_OK";
@@ -288,7 +375,7 @@ uint32_t fa_set_wait_timeout_us(uint32_t us) {
 
 int fa_debug_set_fault(int mode) { return g_fault_mode.exchange(mode); }
 
-int fa_abi_version(void) { return (1 << 16) | 1; }
+int fa_abi_version(void) { return (1 << 16) | 2; }
 
 #ifdef FA_TRACE_UNITS
 int fa_debug_trace_units_read(unsigned long long* host, int n) {
@@ -406,6 +493,8 @@ int launch_tc_noalloc(const void* q, const void* k, const void* v, void* o, floa
   p.n_units = (int)(B * H * (int64_t)p.n_pairs);
   p.chunk_heads = chunk_heads_for(B * H, Nkv, D);
   p.kv_group = 1;        // one K/V head per query head
+  p.block_table = nullptr;  // contiguous K/V
+  p.block_size = p.max_blocks = p.num_blocks = 0;
   p.sched = nd.scratch;  // slot 0 of the static array
   p.timeout_ns = (uint64_t)g_timeout_us.load() * 1000ull;
   p.fault_mode = g_fault_mode.load();

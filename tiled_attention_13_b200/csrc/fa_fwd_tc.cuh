@@ -147,6 +147,12 @@ struct TcParams {
   int n_units;       // B * H * n_pairs
   int chunk_heads;   // (batch, head) pairs per scheduling chunk (L2 working set)
   int kv_group;      // query heads per K/V head: query head h reads K/V head h / kv_group
+  // Paged K/V (the kernel's PAGED instantiation): the K and V tensor maps cover caches of
+  // [num_blocks, block_size, Hkv, d]; key n of batch entry b lives in
+  // physical block block_table[b * max_blocks + n / block_size], row
+  // n % block_size.  block_size is a power of two >= 16.
+  const int* block_table;
+  int block_size, max_blocks, num_blocks;
   SchedSlot* sched;  // this launch's work-ticket counter
   uint64_t timeout_ns;
   int fault_mode;
@@ -214,7 +220,7 @@ struct Pack<__half> {
   }
 };
 
-template <int D, typename T>
+template <int D, typename T, bool PAGED = false>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     fa_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, TcParams p, unsigned int* status_word) {
@@ -309,6 +315,23 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       uint32_t uphase = 0;
       int n_claimed = 0;
       (void)n_claimed;
+      // One 128-key K or V tile from a paged cache: sub-boxes of min(block
+      // size, 128) rows, each from the physical block its keys live in.
+      // Blocks past the sequence read at block index num_blocks, outside the
+      // tensor map, which the copy fills with zeros.
+      const int pbox = PAGED ? (p.block_size < TC_BN ? p.block_size : TC_BN) : TC_BN;
+      const int pvalid = PAGED ? (p.Nkv + p.block_size - 1) / p.block_size : 0;
+      auto paged_load = [&](uint32_t dst, const CUtensorMap* tm, uint32_t b_full, int kv0, int b, int hk,
+                            uint64_t pol) {
+        for (int r0 = 0; r0 < TC_BN; r0 += pbox) {
+          const int key = kv0 + r0;
+          const int lb = key / p.block_size;
+          const int phys = lb < pvalid ? p.block_table[(long long)b * p.max_blocks + lb] : p.num_blocks;
+          const int off = key - lb * p.block_size;
+          for (int c = 0; c < C::CHUNKS; ++c)
+            tma_load_4d(dst + c * C::CHUNK_BYTES + r0 * 128, tm, b_full, c * 64, hk, off, phys, pol);
+        }
+      };
       while (ok) {
         // claim the next ticket and hand it to the other roles
         // (decoded here once: its integer divisions stay off the other roles)
@@ -344,21 +367,29 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           if (!mbar_wait(bar(B_KEMPTY + st), kv_phase ^ 1, wctx)) { ok = false; break; }
           mbar_arrive_expect_tx(bar(B_KFULL + st), C::TILE_BYTES);
           const uint32_t kdst = sbase + C::OFF_K + st * C::TILE_BYTES;
-          for (int c = 0; c < C::CHUNKS; ++c) {
-            if (p.bsnd)
-              tma_load_4d(kdst + c * C::CHUNK_BYTES, &tm_k, bar(B_KFULL + st), c * 64, hk, kv0, w.b, pol_kv);
-            else
-              tma_load_4d(kdst + c * C::CHUNK_BYTES, &tm_k, bar(B_KFULL + st), c * 64, kv0, hk, w.b, pol_kv);
+          if constexpr (PAGED) {
+            paged_load(kdst, &tm_k, bar(B_KFULL + st), kv0, w.b, hk, pol_kv);
+          } else {
+            for (int c = 0; c < C::CHUNKS; ++c) {
+              if (p.bsnd)
+                tma_load_4d(kdst + c * C::CHUNK_BYTES, &tm_k, bar(B_KFULL + st), c * 64, hk, kv0, w.b, pol_kv);
+              else
+                tma_load_4d(kdst + c * C::CHUNK_BYTES, &tm_k, bar(B_KFULL + st), c * 64, kv0, hk, w.b, pol_kv);
+            }
           }
           k_pend[st] = true; k_issued[st] = kv_phase;
           if (!mbar_wait(bar(B_VEMPTY + st), kv_phase ^ 1, wctx)) { ok = false; break; }
           mbar_arrive_expect_tx(bar(B_VFULL + st), C::TILE_BYTES);
           const uint32_t vdst = sbase + C::OFF_V + st * C::TILE_BYTES;
-          for (int c = 0; c < C::CHUNKS; ++c) {
-            if (p.bsnd)
-              tma_load_4d(vdst + c * C::CHUNK_BYTES, &tm_v, bar(B_VFULL + st), c * 64, hk, kv0, w.b, pol_kv);
-            else
-              tma_load_4d(vdst + c * C::CHUNK_BYTES, &tm_v, bar(B_VFULL + st), c * 64, kv0, hk, w.b, pol_kv);
+          if constexpr (PAGED) {
+            paged_load(vdst, &tm_v, bar(B_VFULL + st), kv0, w.b, hk, pol_kv);
+          } else {
+            for (int c = 0; c < C::CHUNKS; ++c) {
+              if (p.bsnd)
+                tma_load_4d(vdst + c * C::CHUNK_BYTES, &tm_v, bar(B_VFULL + st), c * 64, hk, kv0, w.b, pol_kv);
+              else
+                tma_load_4d(vdst + c * C::CHUNK_BYTES, &tm_v, bar(B_VFULL + st), c * 64, kv0, hk, w.b, pol_kv);
+            }
           }
           v_pend[st] = true; v_issued[st] = kv_phase;
           FA_TRU(j == N - 1, 0, n_claimed, 2);
@@ -430,6 +461,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (j > 0 && !wait_all(B_VFULL + st_prev, ph_prev)) { ok = false; break; }
         FA_TR(lane == 0 && u_first, 17, j, 0);
         tc_fence_after();
+        if (PAGED && j > 0 && (j - 1) * TC_BN + TC_BN > p.Nkv) {
+          // Rows past Nkv of this V tile hold whatever the cache has there
+          // (stale or never written).  Their P is 0, but 0 x NaN would still
+          // reach O: clear them before the P V that reads this tile.
+          const int r0 = p.Nkv - (j - 1) * TC_BN;
+          const uint32_t vbase = sbase + C::OFF_V + st_prev * C::TILE_BYTES;
+          for (int c = 0; c < C::CHUNKS; ++c)
+            for (int i = r0 * 8 + lane; i < TC_BN * 8; i += 32)  // 8 x 16 bytes per 128-byte row
+              st_shared_v4(vbase + c * C::CHUNK_BYTES + i * 16, 0u, 0u, 0u, 0u);
+          fence_proxy_async_smem();
+          __syncwarp();
+        }
         const uint64_t dK = dK0 + (uint64_t)((st * C::TILE_BYTES) >> 4);
         const uint64_t dV = dV0 + (uint64_t)((st_prev * C::TILE_BYTES) >> 4);
         for (int i = 0; i < 2 && ok; ++i) {

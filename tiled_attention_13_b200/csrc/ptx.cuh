@@ -103,6 +103,16 @@ __device__ __forceinline__ void mbar_arrive_warp(uint32_t bar) {
   if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
 }
 
+// Ordinary shared-memory store of 16 bytes, and the fence that makes this
+// thread's ordinary shared-memory writes visible to the async proxy (tensor
+// core operand reads) that a later MMA issue starts.
+__device__ __forceinline__ void st_shared_v4(uint32_t addr, uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  asm volatile("st.shared.v4.b32 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(a), "r"(b), "r"(c), "r"(d) : "memory");
+}
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // ---------------------------------------------------------------- TMA
 // 4-D tiled bulk tensor load global -> shared, completion counted on `bar`.
 // c0 (innermost) must be a multiple of 16 bytes / element size: callers pass

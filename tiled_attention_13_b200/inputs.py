@@ -12,6 +12,11 @@ Recipe (stated in DESIGN.md as well):
   ``torch.randperm`` on a CPU generator seeded ``4*seed + 3`` (the same
   positions for every batch and head); ``+3.0`` is added to all d entries of K
   at those positions before the rounding.
+* Paged K/V (``block_size > 0``): the keys and values above are placed into
+  a cache of ``B * ceil(Nkv / block_size) + 3`` physical blocks in an order
+  drawn by ``torch.randperm`` on a CPU generator seeded ``10**9 + seed``;
+  every cache element no block-table entry points at (spare blocks, rows past
+  Nkv in each sequence's last block) is NaN, so that any read of them shows.
 * The named workloads are the shapes the surveyed pages benchmark (LLaMA-13B
   self-attention, B=4/H=32/D=128 batched attention, a diffusion cross-attention
   block, 128K long context), plus a grouped-query variant of the LLaMA-13B
@@ -46,6 +51,7 @@ class Workload:
     k_outlier: float = 0.0
     outlier_frac: float = 0.0
     Hkv: int = 0  # K/V heads (grouped-query attention); 0 means H
+    block_size: int = 0  # > 0: K/V read through a paged cache with blocks of this many keys
 
     @property
     def kv_heads(self) -> int:
@@ -97,6 +103,8 @@ WORKLOADS = {
                 k_outlier=3.0, outlier_frac=0.01),
     "llama13b-8k-gqa8": _wl("llama13b-8k-gqa8", 5, B=1, H=40, Hkv=8, Nq=8192, Nkv=8192, d=128, layout="BSND",
                             causal=True),
+    "llama13b-8k-gqa8-paged16": _wl("llama13b-8k-gqa8-paged16", 5, B=1, H=40, Hkv=8, Nq=8192, Nkv=8192, d=128,
+                                    layout="BSND", causal=True, block_size=16),
 }
 
 
@@ -144,3 +152,33 @@ class _null:
 
 def storage_dtype(name: str) -> torch.dtype:
     return _DTYPES[name]
+
+
+def make_paged_kv(wl: Workload, k, v, spare: int = 3):
+    """Place contiguous k, v (``wl``'s layout) into a paged cache.
+
+    Returns (k_cache, v_cache, block_table): caches [num_blocks, block_size,
+    Hkv, d] in k's dtype and device, NaN wherever the table does not point;
+    block_table int32 [B, ceil(Nkv / block_size)], logical block i of batch
+    entry b -> physical block.  Layout only: no attention arithmetic.
+    """
+    bs = wl.block_size
+    if bs <= 0:
+        raise ValueError("workload has no block size")
+    kk = k if wl.layout == "BSND" else k.transpose(1, 2)  # [B, Nkv, Hkv, d]
+    vv = v if wl.layout == "BSND" else v.transpose(1, 2)
+    B, n, hk, d = kk.shape
+    nb = -(-n // bs)
+    num_blocks = B * nb + spare
+    order = torch.randperm(num_blocks, generator=_gen(10**9 + wl.seed, "cpu"))
+    table = order[:B * nb].reshape(B, nb).to(torch.int32)
+    kc = torch.full((num_blocks, bs, hk, d), float("nan"), dtype=k.dtype, device=k.device)
+    vc = torch.full_like(kc, float("nan"))
+    for b in range(B):
+        for i in range(nb):
+            rows = min(bs, n - i * bs)
+            phys = int(table[b, i])
+            kc[phys, :rows] = kk[b, i * bs:i * bs + rows]
+            vc[phys, :rows] = vv[b, i * bs:i * bs + rows]
+    return kc, vc, table.to(k.device)
+

@@ -315,21 +315,32 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       uint32_t uphase = 0;
       int n_claimed = 0;
       (void)n_claimed;
-      // One 128-key K or V tile from a paged cache: sub-boxes of min(block
-      // size, 128) rows, each from the physical block its keys live in.
-      // Blocks past the sequence read at block index num_blocks, outside the
-      // tensor map, which the copy fills with zeros.
+      // One 128-key K or V tile from a paged cache: TC_BN / pbox sub-boxes of
+      // pbox = min(block size, 128) rows, sub-box u from physical block
+      // phys[u].  Blocks past the sequence read at block index num_blocks,
+      // outside the tensor map, which the copy fills with zeros.
+      constexpr int PSUB = TC_BN / 16;  // sub-boxes per tile at the smallest block size
       const int pbox = PAGED ? (p.block_size < TC_BN ? p.block_size : TC_BN) : TC_BN;
       const int pvalid = PAGED ? (p.Nkv + p.block_size - 1) / p.block_size : 0;
-      auto paged_load = [&](uint32_t dst, const CUtensorMap* tm, uint32_t b_full, int kv0, int b, int hk,
-                            uint64_t pol) {
-        for (int r0 = 0; r0 < TC_BN; r0 += pbox) {
-          const int key = kv0 + r0;
-          const int lb = key / p.block_size;
-          const int phys = lb < pvalid ? p.block_table[(long long)b * p.max_blocks + lb] : p.num_blocks;
-          const int off = key - lb * p.block_size;
+      int phys[PSUB];
+      // the tile's table entries, read together (independent loads) before
+      // any of its copies is issued, and used for both K and V
+      auto paged_lookup = [&](int kv0, int b) {
+#pragma unroll
+        for (int u = 0; u < PSUB; ++u) {
+          const int lb = (kv0 + u * pbox) / p.block_size;
+          phys[u] = (u * pbox < TC_BN && lb < pvalid) ? p.block_table[(long long)b * p.max_blocks + lb]
+                                                      : p.num_blocks;
+        }
+      };
+      auto paged_load = [&](uint32_t dst, const CUtensorMap* tm, uint32_t b_full, int kv0, int hk, uint64_t pol) {
+#pragma unroll
+        for (int u = 0; u < PSUB; ++u) {
+          if (u * pbox >= TC_BN) break;
+          const int key = kv0 + u * pbox;
+          const int off = key % p.block_size;
           for (int c = 0; c < C::CHUNKS; ++c)
-            tma_load_4d(dst + c * C::CHUNK_BYTES + r0 * 128, tm, b_full, c * 64, hk, off, phys, pol);
+            tma_load_4d(dst + c * C::CHUNK_BYTES + u * pbox * 128, tm, b_full, c * 64, hk, off, phys[u], pol);
         }
       };
       while (ok) {
@@ -368,7 +379,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           mbar_arrive_expect_tx(bar(B_KFULL + st), C::TILE_BYTES);
           const uint32_t kdst = sbase + C::OFF_K + st * C::TILE_BYTES;
           if constexpr (PAGED) {
-            paged_load(kdst, &tm_k, bar(B_KFULL + st), kv0, w.b, hk, pol_kv);
+            paged_lookup(kv0, w.b);
+            paged_load(kdst, &tm_k, bar(B_KFULL + st), kv0, hk, pol_kv);
           } else {
             for (int c = 0; c < C::CHUNKS; ++c) {
               if (p.bsnd)
@@ -382,7 +394,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           mbar_arrive_expect_tx(bar(B_VFULL + st), C::TILE_BYTES);
           const uint32_t vdst = sbase + C::OFF_V + st * C::TILE_BYTES;
           if constexpr (PAGED) {
-            paged_load(vdst, &tm_v, bar(B_VFULL + st), kv0, w.b, hk, pol_kv);
+            paged_load(vdst, &tm_v, bar(B_VFULL + st), kv0, hk, pol_kv);
           } else {
             for (int c = 0; c < C::CHUNKS; ++c) {
               if (p.bsnd)

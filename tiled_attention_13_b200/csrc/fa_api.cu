@@ -2,7 +2,9 @@
 // descriptor encoding, launch configuration and the device status word.
 //
 // One translation unit holds every kernel so that they share the status word
-// (a static __device__ variable: no device allocation anywhere).
+// (a static __device__ variable).  The only device allocation is fa_fwd's
+// 8 KB of tile-scheduler counters, made once per device on its first call;
+// fa_fwd_noalloc uses a static array instead.
 #include <cuda.h>
 #include <cuda_runtime.h>
 

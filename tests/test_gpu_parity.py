@@ -261,6 +261,19 @@ def test_paged_llama13b_8k_sampled():
                     qkv=(q, k, v))
 
 
+# ----------------------------------------------------------------- decode-shaped calls
+@pytest.mark.parametrize("nkv", [1, 129, 4097])
+@pytest.mark.parametrize("nq", [1, 7])
+def test_decode_shapes_contiguous_and_paged(nq, nkv):
+    """A few query rows (one partly filled Q tile) against short to long,
+    ragged K/V with grouped heads: contiguous, and through a paged cache of
+    16-key blocks (the decode use of a paged cache)."""
+    wl = Workload("decode", B=2, H=8, Hkv=2, Nq=nq, Nkv=nkv, d=128, dtype="bf16", layout="BSND", causal=False,
+                  seed=nq * 7 + nkv)
+    compare_full(wl)
+    _paged_parity(wl.with_(block_size=16))
+
+
 # ----------------------------------------------------------------- named workloads
 def test_tiny_full():
     for name in ("tiny", "tiny-causal"):

@@ -123,3 +123,20 @@ def test_binding_does_not_import_oracle():
     for f in os.listdir(os.path.join(ROOT, "tiled_attention_13_b200", "csrc")):
         src += open(os.path.join(ROOT, "tiled_attention_13_b200", "csrc", f)).read()
     assert "oracle" not in src
+
+
+def test_binding_rejects_host_tensors_and_bad_tables(fa_lib):
+    """The Python wrappers check their tensors before calling the library:
+    host (CPU) tensors raise ValueError for the contiguous and the paged form
+    (without a GPU that check is the first one reached).""
+    import torch
+
+    q = torch.zeros((1, 2, 8, 64), dtype=torch.bfloat16)
+    with pytest.raises(ValueError):
+        fa.forward(q, q, q)
+    kc = torch.zeros((4, 16, 2, 64), dtype=torch.bfloat16)
+    table = torch.zeros((1, 4), dtype=torch.int32)
+    with pytest.raises(ValueError):
+        fa.forward_paged(q, kc, kc, table, 40)
+    with pytest.raises(ValueError):
+        fa.forward(q, q.float(), q)

@@ -128,7 +128,7 @@ def test_binding_does_not_import_oracle():
 def test_binding_rejects_host_tensors_and_bad_tables(fa_lib):
     """The Python wrappers check their tensors before calling the library:
     host (CPU) tensors raise ValueError for the contiguous and the paged form
-    (without a GPU that check is the first one reached).""
+    (without a GPU that check is the first one reached)."""
     import torch
 
     q = torch.zeros((1, 2, 8, 64), dtype=torch.bfloat16)

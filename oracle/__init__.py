@@ -23,4 +23,10 @@ from .attention_ref import (  # noqa: F401
     allowed_keys,
     attention_paged,
     gather_paged_kv,
+    merge_partials,
+)
+from .backward_ref import (  # noqa: F401
+    attention_backward,
+    attention_backward_batched,
+    attention_backward_tiled,
 )

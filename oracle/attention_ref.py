@@ -292,3 +292,24 @@ def attention_paged(q, k_cache, v_cache, block_tables, seq_len: int, scale=None,
     elif layout != "BSND":
         raise ValueError(f"unknown layout {layout!r}")
     return attention_batched(q, k, v, scale=scale, causal=causal, layout=layout)
+
+
+def merge_partials(o_parts, lse_parts):
+    """Attention over a key set split into parts, from each part's own result:
+    with O_r, LSE_r the attention of the same query rows over key part r,
+    LSE = log sum_r exp(LSE_r) and O = sum_r exp(LSE_r - LSE) O_r.  This is the
+    online-softmax merge (page 1, section 在线 Softmax 的数学原理拆解) applied
+    to whole parts, the step that splitting the keys across workers (page 1's
+    Ring Attention, split-KV decoding) needs.  A part with no visible key for a
+    row has LSE_r = -inf and weight 0.  o_parts [R, ..., d], lse_parts [R, ...].
+    """
+    o = _as_f64(o_parts)
+    lse = _as_f64(lse_parts)
+    m = np.max(lse, axis=0)
+    m_safe = np.where(np.isfinite(m), m, 0.0)
+    w = np.exp(lse - m_safe)
+    tot = np.sum(w, axis=0)
+    out_lse = m_safe + np.log(tot)
+    out_o = np.sum(w[..., None] * o, axis=0) / tot[..., None]
+    return out_o, out_lse
+

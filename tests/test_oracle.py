@@ -27,6 +27,10 @@ from oracle import (
     resolve_scale,
     attention_paged,
     gather_paged_kv,
+    merge_partials,
+    attention_backward,
+    attention_backward_batched,
+    attention_backward_tiled,
 )
 
 GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
@@ -400,3 +404,98 @@ def test_attention_paged_equals_contiguous(layout, causal):
     o_ref, l_ref = attention_batched(q, kk, vv, causal=causal, layout=layout)
     o, lse = attention_paged(q, kc, vc, tables, n, causal=causal, layout=layout)
     assert np.all(np.isfinite(o)) and np.array_equal(o, o_ref) and np.array_equal(lse, l_ref)
+
+
+# ---------------------------------------------------------------- split key sets: merging partial results
+@pytest.mark.parametrize("causal", [False, True])
+def test_merge_of_key_parts_equals_whole(causal):
+    """Attention over the whole key set equals the merge of attention over
+    disjoint key ranges (for causal rows, ranges they cannot see have
+    LSE = -inf and weight 0)."""
+    nq, nkv, d = 23, 41, 8
+    q, k, v = rnd(nq, d), rnd(nkv, d), rnd(nkv, d)
+    o, lse = attention(q, k, v, causal=causal)
+    cuts = [0, 5, 17, 18, 41]
+    parts_o, parts_l = [], []
+    for a, b in zip(cuts[:-1], cuts[1:]):
+        po, pl = np.zeros((nq, d)), np.full(nq, -np.inf)
+        for i in range(nq):
+            hi = min(b, i + 1) if causal else b
+            if hi > a:
+                ro, rl = attention(q[i:i + 1], k[a:hi], v[a:hi])
+                po[i], pl[i] = ro[0], rl[0]
+        parts_o.append(po)
+        parts_l.append(pl)
+    mo, ml = merge_partials(np.stack(parts_o), np.stack(parts_l))
+    assert np.max(np.abs(mo - o)) <= 1e-13 and np.max(np.abs(ml - lse)) <= 1e-13
+
+
+# ---------------------------------------------------------------- gradients (backward)
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_matches_finite_differences(causal):
+    """Central differences of L = sum(O * W) + sum(LSE * u), through the forward
+    oracle, against the gradient oracle, at every entry of Q, K and V."""
+    nq, nkv, d = 5, 7, 4
+    q, k, v = rnd(nq, d), rnd(nkv, d), rnd(nkv, d)
+    w, u = rnd(nq, d), rnd(nq)
+
+    def loss(qq, kk, vv):
+        o, lse = attention(qq, kk, vv, causal=causal)
+        return float(np.sum(o * w) + np.sum(lse * u))
+
+    dq, dk, dv = attention_backward(q, k, v, w, causal=causal, dlse=u)
+    h = 1e-6
+    for x, g in ((q, dq), (k, dk), (v, dv)):
+        for idx in np.ndindex(x.shape):
+            old = x[idx]
+            x[idx] = old + h
+            lp = loss(q, k, v)
+            x[idx] = old - h
+            lm = loss(q, k, v)
+            x[idx] = old
+            assert abs((lp - lm) / (2 * h) - g[idx]) <= 1e-7, idx
+
+
+@pytest.mark.parametrize("hkv", [4, 2, 1])
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_torch_autograd_cross_check(hkv, causal):
+    """Library cross-check: torch float64 scaled_dot_product_attention with
+    autograd (grouped K/V heads included), both layouts."""
+    B, H, n, d = 2, 4, 19, 8
+    q, k, v, do = rnd(B, H, n, d), rnd(B, hkv, n, d), rnd(B, hkv, n, d), rnd(B, H, n, d)
+    tq, tk, tv = (torch.from_numpy(x.copy()).requires_grad_(True) for x in (q, k, v))
+    out = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=causal, enable_gqa=True)
+    out.backward(torch.from_numpy(do))
+    dq, dk, dv = attention_backward_batched(q, k, v, do, causal=causal)
+    for mine, ref in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+        assert np.max(np.abs(mine - ref.numpy())) <= 1e-10
+    t = (0, 2, 1, 3)
+    dq2, dk2, dv2 = attention_backward_batched(q.transpose(t), k.transpose(t), v.transpose(t), do.transpose(t),
+                                               causal=causal, layout="BSND")
+    assert np.array_equal(dq2.transpose(t), dq) and np.array_equal(dk2.transpose(t), dk)
+
+
+@pytest.mark.parametrize("br,bc", [(1, 1), (3, 5), (16, 16), (64, 7)])
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_tiled_recompute_equals_definition(br, bc, causal):
+    """The page's recompute scheme (tiles rebuilt from the forward's LSE only)
+    gives the definition's gradients, for any tile sizes."""
+    nq, nkv, d = 29, 37, 8
+    q, k, v, do = rnd(nq, d), rnd(nkv, d), rnd(nkv, d), rnd(nq, d)
+    _, lse = attention(q, k, v, causal=causal)
+    ref = attention_backward(q, k, v, do, causal=causal)
+    got = attention_backward_tiled(q, k, v, do, lse, br, bc, causal=causal)
+    for a, b in zip(got, ref):
+        assert np.max(np.abs(a - b)) <= 1e-12
+
+
+def test_backward_equal_keys_give_zero_query_gradient():
+    """All keys equal: every row's scores are constant, the softmax does not
+    depend on Q, so dQ = 0 (the rows of dS sum to zero)."""
+    nq, nkv, d = 6, 9, 5
+    q, v, do = rnd(nq, d), rnd(nkv, d), rnd(nq, d)
+    k = np.tile(rnd(1, d), (nkv, 1))
+    dq, _, dv = attention_backward(q, k, v, do)
+    assert np.max(np.abs(dq)) <= 1e-13
+    assert np.max(np.abs(dv - np.tile(do.sum(axis=0) / nkv, (nkv, 1)))) <= 1e-13  # uniform P = 1/Nkv: dV_j = sum_i dO_i / Nkv
+

@@ -1,7 +1,6 @@
 """C-ABI checks that need no GPU: the library loads, exports every entry point
 declared in include/fa.h, and rejects bad arguments before touching CUDA."""
 
-import ctypes
 import os
 import re
 import subprocess

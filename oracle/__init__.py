@@ -24,6 +24,9 @@ from .attention_ref import (  # noqa: F401
     attention_paged,
     gather_paged_kv,
     merge_partials,
+    band_mask,
+    block_sparse_mask,
+    attention_masked,
 )
 from .backward_ref import (  # noqa: F401
     attention_backward,

@@ -313,3 +313,43 @@ def merge_partials(o_parts, lse_parts):
     out_o = np.sum(w[..., None] * o, axis=0) / tot[..., None]
     return out_o, out_lse
 
+
+def band_mask(nq: int, nkv: int, pre_tokens: int, next_tokens: int) -> np.ndarray:
+    """Visible (query, key) pairs of a band: key j is visible to query i iff
+    i - pre_tokens <= j <= i + next_tokens.  Page 2's flash_attention_score
+    takes pre_tokens / next_tokens and calls it with pre_tokens = seq_len,
+    next_tokens = 0 for causal inference; that call's meaning (every earlier
+    key, no later one) is the reading taken for other values."""
+    i = np.arange(nq).reshape(-1, 1)
+    j = np.arange(nkv).reshape(1, -1)
+    return (j >= i - pre_tokens) & (j <= i + next_tokens)
+
+
+def block_sparse_mask(block_mask, block_r: int, block_c: int, nq: int, nkv: int) -> np.ndarray:
+    """Element mask of a block-sparse pattern (page 1, SparseFlashAttention:
+    key blocks marked as not needed are skipped): query tile a (rows
+    [a*block_r, ...)) sees key tile b (keys [b*block_c, ...)) iff
+    block_mask[a, b]."""
+    bm = np.asarray(block_mask, dtype=bool)
+    rows = np.arange(nq) // block_r
+    cols = np.arange(nkv) // block_c
+    return bm[rows][:, cols]
+
+
+def attention_masked(q, k, v, mask, scale=None):
+    """The definition with an explicit boolean mask [Nq, Nkv] of visible
+    (query, key) pairs: softmax over each row's visible keys only.  Every row
+    must see at least one key."""
+    q, k, v = _as_f64(q), _as_f64(k), _as_f64(v)
+    mask = np.asarray(mask, dtype=bool)
+    if mask.shape != (q.shape[0], k.shape[0]):
+        raise ValueError("mask must be [Nq, Nkv]")
+    if q.shape[0] and not np.all(mask.any(axis=1)):
+        raise ValueError("a query row sees no key")
+    sc = resolve_scale(scale, q.shape[1])
+    s = np.where(mask, sc * (q @ k.T), -np.inf)
+    m = np.max(s, axis=1, keepdims=True) if q.shape[0] else np.zeros((0, 1))
+    e = np.exp(s - m)
+    z = np.sum(e, axis=1, keepdims=True)
+    return (e @ v) / z, (m + np.log(z)).reshape(-1)
+

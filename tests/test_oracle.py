@@ -28,6 +28,9 @@ from oracle import (
     attention_paged,
     gather_paged_kv,
     merge_partials,
+    band_mask,
+    block_sparse_mask,
+    attention_masked,
     attention_backward,
     attention_backward_batched,
     attention_backward_tiled,
@@ -498,4 +501,60 @@ def test_backward_equal_keys_give_zero_query_gradient():
     dq, _, dv = attention_backward(q, k, v, do)
     assert np.max(np.abs(dq)) <= 1e-13
     assert np.max(np.abs(dv - np.tile(do.sum(axis=0) / nkv, (nkv, 1)))) <= 1e-13  # uniform P = 1/Nkv: dV_j = sum_i dO_i / Nkv
+
+
+# ---------------------------------------------------------------- band and block-sparse masks
+def test_band_reduces_to_causal_and_full():
+    """pre_tokens >= N, next_tokens = 0 (page 2's causal call) is the causal
+    path; both >= N is unmasked attention."""
+    n, d = 33, 8
+    q, k, v = rnd(n, d), rnd(n, d), rnd(n, d)
+    o_c, l_c = attention(q, k, v, causal=True)
+    o_b, l_b = attention_masked(q, k, v, band_mask(n, n, n, 0))
+    assert np.max(np.abs(o_b - o_c)) <= 1e-13 and np.max(np.abs(l_b - l_c)) <= 1e-13
+    for i in range(n):  # the same visible sets as the causal reading
+        assert np.array_equal(np.flatnonzero(band_mask(n, n, n, 0)[i]), allowed_keys(i, n, True))
+    o_f, l_f = attention(q, k, v)
+    o_b2, l_b2 = attention_masked(q, k, v, band_mask(n, n, n, n))
+    assert np.max(np.abs(o_b2 - o_f)) <= 1e-13 and np.max(np.abs(l_b2 - l_f)) <= 1e-13
+
+
+def test_band_of_width_one_is_the_diagonal():
+    """pre = next = 0: every query sees only its own key: O_i = V_i and
+    LSE_i = scale * q_i . k_i."""
+    n, d = 7, 4
+    q, k, v = rnd(n, d), rnd(n, d), rnd(n, d)
+    o, lse = attention_masked(q, k, v, band_mask(n, n, 0, 0))
+    assert np.max(np.abs(o - v)) <= 1e-14
+    assert np.max(np.abs(lse - np.sum(q * k, axis=1) / math.sqrt(d))) <= 1e-13
+
+
+@pytest.mark.parametrize("pre,nxt", [(3, 2), (0, 5), (10, 0), (1, 1)])
+def test_band_torch_sdpa_cross_check(pre, nxt):
+    """Library cross-check: torch float64 scaled_dot_product_attention with the
+    band as an explicit boolean attn_mask."""
+    n, d = 21, 8
+    q, k, v = rnd(1, 1, n, d), rnd(1, 1, n, d), rnd(1, 1, n, d)
+    mask = band_mask(n, n, pre, nxt)
+    o, _ = attention_masked(q[0, 0], k[0, 0], v[0, 0], mask)
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        torch.from_numpy(q), torch.from_numpy(k), torch.from_numpy(v), attn_mask=torch.from_numpy(mask)).numpy()
+    assert np.max(np.abs(o - ref[0, 0])) <= 1e-12
+
+
+def test_block_sparse_mask_expands_tiles():
+    """Each (query tile, key tile) entry covers exactly its rectangle, ragged
+    last tiles included; an all-true block mask is unmasked attention."""
+    nq, nkv, br, bc = 10, 13, 4, 5
+    bm = np.array([[1, 0, 1], [0, 1, 0], [1, 1, 0]], dtype=bool)
+    m = block_sparse_mask(bm, br, bc, nq, nkv)
+    for i in range(nq):
+        for j in range(nkv):
+            assert m[i, j] == bm[i // br, j // bc]
+    q, k, v = rnd(nq, 4), rnd(nkv, 4), rnd(nkv, 4)
+    o, lse = attention_masked(q, k, v, block_sparse_mask(np.ones((3, 3), bool), br, bc, nq, nkv))
+    o2, l2 = attention(q, k, v)
+    assert np.max(np.abs(o - o2)) <= 1e-13 and np.max(np.abs(lse - l2)) <= 1e-13
+    with pytest.raises(ValueError):
+        attention_masked(q, k, v, block_sparse_mask(np.zeros((3, 3), bool), br, bc, nq, nkv))
 

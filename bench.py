@@ -149,7 +149,7 @@ def oracle_sample(wl, rows_budget_s: float = 12.0, seed: int = 0):
     import torch
     from threadpoolctl import threadpool_info
 
-    from oracle import attention
+    from oracle import attention, attention_masked, band_mask
     from tiled_attention_13_b200.inputs import make_qkv
 
     one = wl.with_(B=1, H=1, Hkv=0)
@@ -169,6 +169,14 @@ def oracle_sample(wl, rows_budget_s: float = 12.0, seed: int = 0):
     rng.shuffle(starts)
     for r0 in starts:
         r1 = min(wl.Nq, r0 + block)
+        if wl.band:
+            mask = band_mask(wl.Nq, wl.Nkv, wl.band[0], wl.band[1])[r0:r1]
+            attention_masked(qn[r0:r1], kn, vn, mask)
+            flops += 4.0 * wl.d * float(mask.sum())
+            rows_done += r1 - r0
+            if time.perf_counter() - t0 > rows_budget_s:
+                break
+            continue
         attention(qn[r0:r1], kn, vn, causal=wl.causal, row_offset=r0)
         if wl.causal:
             flops += 4.0 * wl.d * sum(min(i + 1, wl.Nkv) for i in range(r0, r1))
@@ -231,6 +239,7 @@ def _config(wl, ws):
             "layout": wl.layout, "causal": wl.causal, "input_dtype": wl.dtype,
             **({"Hkv": wl.kv_heads} if wl.kv_heads != wl.H else {}),
             **({"kv_cache": f"paged, {wl.block_size}-key blocks in shuffled order"} if wl.block_size > 0 else {}),
+            **({"band": {"pre_tokens": wl.band[0], "next_tokens": wl.band[1]}} if wl.band else {}),
             "parallelism": f"independent replicas x{ws} (no collective)",
             "l2": (f"{n} input sets of {wl.bytes_min / 1e6:.1f} MB (Q, K, V, O, LSE) rotate between steps, "
                    f"{n * wl.bytes_min / 1e6:.0f} MB in all > 2x the 126 MB L2"),
@@ -271,7 +280,7 @@ def run_ours(args, wl):
     def step(i):
         q, k, v, o, lse, paged = sets[i % n_sets]
         if paged is None:
-            fa.forward(q, k, v, causal=wl.causal, layout=wl.layout, out=o, lse=lse)
+            fa.forward(q, k, v, causal=wl.causal, layout=wl.layout, out=o, lse=lse, band=wl.band or None)
         else:
             kc, vc, table = paged
             fa.forward_paged(q, kc, vc, table, wl.Nkv, causal=wl.causal, layout=wl.layout, out=o, lse=lse)
@@ -342,9 +351,9 @@ def run_ours(args, wl):
 
     # ---- end-to-end through the public API: pinned host in, host out
     e2e = None
-    if not args.no_e2e and wl.block_size > 0:
-        e2e = {"value": None, "unit": UNIT, "skipped": "HostPipeline takes contiguous K/V; the paged path is "
-               "measured on the device only"}
+    if not args.no_e2e and (wl.block_size > 0 or wl.band):
+        e2e = {"value": None, "unit": UNIT, "skipped": "HostPipeline takes contiguous K/V without a band; this "
+               "path is measured on the device only"}
     elif not args.no_e2e:
         # Every step copies its inputs from pinned host memory and reads its
         # O and LSE back; HostPipeline overlaps step i+1's upload and step

@@ -108,6 +108,26 @@ int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
                float scale, int causal, int layout, int dtype, void* stream);
 
 /*
+ * fa_fwd_band -- fa_fwd_gqa with a band mask in place of the causal flag:
+ * key j is visible to query row i iff i - pre_tokens <= j <= i + next_tokens
+ * (and j < Nkv).  Page 2's flash_attention_score takes pre_tokens and
+ * next_tokens and calls them with pre_tokens = seq_len, next_tokens = 0 for
+ * causal attention; other values are read the same way (a sliding window:
+ * pre_tokens = W - 1, next_tokens = 0).  KV tiles outside a query tile's band
+ * are skipped.
+ *
+ *   pre_tokens, next_tokens  >= 0, and pre_tokens >= Nq - Nkv so that every
+ *                            query row sees at least one key; otherwise
+ *                            FA_ERR_INVALID_ARG
+ *   dtype                    bf16 or fp16 (fp32 returns FA_ERR_UNSUPPORTED)
+ *
+ * Other arguments, ownership and errors are as for fa_fwd_gqa.
+ */
+int fa_fwd_band(const void* q, const void* k, const void* v, void* o, float* lse,
+                int64_t B, int64_t H, int64_t Hkv, int64_t Nq, int64_t Nkv, int64_t d,
+                float scale, int64_t pre_tokens, int64_t next_tokens, int layout, int dtype, void* stream);
+
+/*
  * fa_fwd_paged -- fa_fwd_gqa with K and V read through a paged cache (page
  * 1, section GatherPAKVCache 的显存管理逻辑: the cache is kept in fixed-size
  * physical blocks, and a block table translates each sequence's logical
@@ -201,7 +221,7 @@ uint32_t fa_set_wait_timeout_us(uint32_t us);
  */
 int fa_debug_set_fault(int mode);
 
-/* ABI version of this header, (major << 16) | minor (1.1: fa_fwd_gqa, 1.2: fa_fwd_paged). */
+/* ABI version of this header, (major << 16) | minor (1.1: fa_fwd_gqa, 1.2: fa_fwd_paged, 1.3: fa_fwd_band). */
 int fa_abi_version(void);
 
 #ifdef __cplusplus

@@ -34,7 +34,7 @@ def test_status_strings_and_version(fa_lib):
     for code in range(8):
         assert fa.fa_status_string(code).startswith("FA_")
     assert fa.fa_status_string(99) == "FA_ERR_UNKNOWN"
-    assert fa.fa_abi_version() == (1 << 16) | 2
+    assert fa.fa_abi_version() == (1 << 16) | 3
 
 
 def test_host_settings_roundtrip(fa_lib):
@@ -102,6 +102,23 @@ def test_paged_validation_before_any_cuda_call(fa_lib, kw, code):
                          args["H"], args["Hkv"], args["Nq"], args["Nkv"], args["d"], args["block_size"],
                          args["num_blocks"], args["max_blocks"], args["scale"], args["causal"], args["layout"],
                          args["dtype"], args["stream"])
+    assert rc == code, fa.fa_status_string(rc)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(pre=-1), 1), (dict(nxt=-1), 1), (dict(Nq=200, Nkv=100, pre=50), 1), (dict(Hkv=3), 1),
+    (dict(dtype=2), 2), (dict(d=96), 2), (dict(q=A16 + 8), 3),
+    (dict(B=0), 0), (dict(Nq=0), 0),
+])
+def test_band_validation_before_any_cuda_call(fa_lib, kw, code):
+    """fa_fwd_band: non-negative widths, and pre_tokens >= Nq - Nkv so that the
+    last query rows still see a key; bf16/fp16 only."""
+    args = dict(q=A16, k=A16, v=A16, o=A16, lse=A16, B=1, H=4, Hkv=2, Nq=10, Nkv=10, d=64, scale=-1.0, pre=3,
+                nxt=1, layout=0, dtype=0, stream=None)
+    args.update(kw)
+    rc = fa.fa_fwd_band(args["q"], args["k"], args["v"], args["o"], args["lse"], args["B"], args["H"], args["Hkv"],
+                        args["Nq"], args["Nkv"], args["d"], args["scale"], args["pre"], args["nxt"], args["layout"],
+                        args["dtype"], args["stream"])
     assert rc == code, fa.fa_status_string(rc)
 
 

@@ -274,6 +274,44 @@ def test_decode_shapes_contiguous_and_paged(nq, nkv):
     _paged_parity(wl.with_(block_size=16))
 
 
+# ----------------------------------------------------------------- band masks
+BAND_CASES = [  # (B, H, Hkv, Nq, Nkv, pre_tokens, next_tokens, d, layout)
+    (1, 2, 2, 300, 300, 64, 0, 128, "BSND"),     # sliding window of 65 keys
+    (2, 2, 1, 300, 333, 100, 50, 64, "BHND"),    # two-sided band, MQA
+    (1, 2, 2, 257, 257, 0, 0, 128, "BSND"),      # each row sees only its own key
+    (1, 2, 2, 129, 1000, 1000, 1000, 128, "BHND"),  # wider than the sequences: full attention
+    (1, 2, 2, 300, 300, 300, 0, 64, "BSND"),     # page 2's causal call
+    (1, 8, 2, 513, 513, 200, 17, 128, "BSND"),   # grouped heads, band across tile edges
+    (1, 2, 2, 700, 500, 200, 3, 128, "BHND"),    # Nq > Nkv: pre >= Nq - Nkv
+]
+
+
+@pytest.mark.parametrize("case", BAND_CASES, ids=lambda c: "x".join(map(str, c[:7])) + c[8])
+def test_band_bf16(case):
+    """fa_fwd_band against the oracle's explicit-mask attention on the band."""
+    from oracle import attention_masked, band_mask
+
+    from .parity import LSE_TOL, o_bar
+
+    B, H, hkv, nq, nkv, pre, nxt, d, layout = case
+    wl = Workload("band", B=B, H=H, Hkv=hkv, Nq=nq, Nkv=nkv, d=d, dtype="bf16", layout=layout, seed=nq + pre + nxt)
+    q, k, v = make_qkv(wl)
+    o, lse = fa.forward(q.cuda(), k.cuda(), v.cuda(), layout=layout, band=(pre, nxt))
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_status(None) == 0
+    if layout == "BSND":
+        q, k, v, o = (t.transpose(1, 2) for t in (q, k, v, o))
+    mask = band_mask(nq, nkv, pre, nxt)
+    g = H // hkv
+    for b in range(B):
+        for h in range(H):
+            o_ref, l_ref = attention_masked(q[b, h], k[b, h // g], v[b, h // g], mask)
+            o_gpu, l_gpu = o[b, h].double().cpu().numpy(), lse[b, h].double().cpu().numpy()
+            assert np.all(np.isfinite(o_gpu)) and np.all(np.isfinite(l_gpu))
+            assert np.all(np.abs(o_gpu - o_ref) <= o_bar(o_ref, "bf16")), (b, h, float(np.abs(o_gpu - o_ref).max()))
+            assert np.abs(l_gpu - l_ref).max() <= LSE_TOL
+
+
 # ----------------------------------------------------------------- named workloads
 def test_tiny_full():
     for name in ("tiny", "tiny-causal"):

@@ -23,7 +23,8 @@ import os
 
 __all__ = [
     "FA_LAYOUT_BHND", "FA_LAYOUT_BSND", "FA_DTYPE_BF16", "FA_DTYPE_FP16", "FA_DTYPE_FP32",
-    "FaError", "lib", "lib_path", "fa_fwd", "fa_fwd_gqa", "fa_fwd_paged", "fa_fwd_noalloc", "fa_status_string",
+    "FaError", "lib", "lib_path", "fa_fwd", "fa_fwd_gqa", "fa_fwd_band", "fa_fwd_paged", "fa_fwd_noalloc",
+    "fa_status_string",
     "fa_get_device_status", "fa_set_wait_timeout_us", "fa_debug_set_fault", "fa_abi_version", "forward",
     "forward_paged", "forward_host",
     "HostForward", "HostPipeline", "EXPORTED",
@@ -33,8 +34,8 @@ FA_LAYOUT_BHND, FA_LAYOUT_BSND = 0, 1
 FA_DTYPE_BF16, FA_DTYPE_FP16, FA_DTYPE_FP32 = 0, 1, 2
 FA_OK = 0
 
-EXPORTED = ("fa_fwd", "fa_fwd_gqa", "fa_fwd_paged", "fa_fwd_noalloc", "fa_status_string", "fa_get_device_status",
-            "fa_set_wait_timeout_us", "fa_debug_set_fault", "fa_abi_version")
+EXPORTED = ("fa_fwd", "fa_fwd_gqa", "fa_fwd_band", "fa_fwd_paged", "fa_fwd_noalloc", "fa_status_string",
+            "fa_get_device_status", "fa_set_wait_timeout_us", "fa_debug_set_fault", "fa_abi_version")
 
 _LIB = None
 
@@ -68,6 +69,9 @@ def lib() -> ctypes.CDLL:
     L.fa_fwd_gqa.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, ctypes.c_float, ctypes.c_int,
                              ctypes.c_int, ctypes.c_int, vp]
     L.fa_fwd_gqa.restype = ctypes.c_int
+    L.fa_fwd_band.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, ctypes.c_float, i64, i64, ctypes.c_int,
+                              ctypes.c_int, vp]
+    L.fa_fwd_band.restype = ctypes.c_int
     L.fa_fwd_paged.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64, i64, i64, ctypes.c_float,
                                ctypes.c_int, ctypes.c_int, ctypes.c_int, vp]
     L.fa_fwd_paged.restype = ctypes.c_int
@@ -100,6 +104,13 @@ def fa_fwd_gqa(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, d, scale, causal, layout, dt
     reads K/V head h / (H / Hkv)."""
     return lib().fa_fwd_gqa(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, d, float(scale), int(causal), int(layout),
                             int(dtype), stream)
+
+
+def fa_fwd_band(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, d, scale, pre_tokens, next_tokens, layout, dtype, stream) -> int:
+    """int fa_fwd_band(...): key j visible to query i iff i - pre_tokens <= j <=
+    i + next_tokens."""
+    return lib().fa_fwd_band(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, d, float(scale), int(pre_tokens), int(next_tokens),
+                             int(layout), int(dtype), stream)
 
 
 def fa_fwd_paged(q, k_cache, v_cache, block_table, o, lse, B, H, Hkv, Nq, Nkv, d, block_size, num_blocks,
@@ -161,13 +172,15 @@ def _kv_heads(k, layout):
 
 
 def forward(q, k, v, causal: bool = False, scale=None, layout: str = "BHND", out=None, lse=None,
-            stream=None):
+            stream=None, band=None):
     """O, LSE = softmax(scale Q K^T [+causal]) V on the GPU (returns (o, lse)).
 
     q: [B,H,Nq,d] (BHND) or [B,Nq,H,d] (BSND); k, v the same with Nkv and
     Hkv heads (Hkv dividing H: grouped-query attention when Hkv < H); all
     contiguous CUDA tensors of one dtype (bf16, fp16 or fp32); d in {64, 128}.
-    scale None -> 1/sqrt(d).  LSE is fp32 [B, H, Nq].
+    scale None -> 1/sqrt(d).  LSE is fp32 [B, H, Nq].  band = (pre_tokens,
+    next_tokens) replaces ``causal``: key j visible to query i iff
+    i - pre_tokens <= j <= i + next_tokens (fa_fwd_band; bf16/fp16).
     """
     import torch
 
@@ -189,6 +202,15 @@ def forward(q, k, v, causal: bool = False, scale=None, layout: str = "BHND", out
     Hkv = _kv_heads(k, layout)
     lay = FA_LAYOUT_BHND if layout == "BHND" else FA_LAYOUT_BSND
     lp = lse.data_ptr() if lse.numel() else None
+    if band is not None:
+        if causal:
+            raise ValueError("give either causal or band")
+        pre, nxt = band
+        rc = fa_fwd_band(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lp, B, H, Hkv, Nq, Nkv, d, sc,
+                         int(pre), int(nxt), lay, _dtype_code(q), stream)
+        if rc != FA_OK:
+            raise FaError(rc, "fa_fwd_band")
+        return out, lse
     if Hkv == H:
         rc = fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lp, B, H, Nq, Nkv, d, sc,
                     int(bool(causal)), lay, _dtype_code(q), stream)

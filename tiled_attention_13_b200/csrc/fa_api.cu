@@ -80,6 +80,10 @@ int device_setup(int dev, DeviceInfo** out) {
       ok &= set_smem_attr(fa::fa_fwd_tc_kernel<128, __nv_bfloat16, true>, fa::TcCfg<128>::SMEM_BYTES);
       ok &= set_smem_attr(fa::fa_fwd_tc_kernel<64, __half, true>, fa::TcCfg<64>::SMEM_BYTES);
       ok &= set_smem_attr(fa::fa_fwd_tc_kernel<128, __half, true>, fa::TcCfg<128>::SMEM_BYTES);
+      ok &= set_smem_attr(fa::fa_fwd_tc_kernel<64, __nv_bfloat16, false, true>, fa::TcCfg<64>::SMEM_BYTES);
+      ok &= set_smem_attr(fa::fa_fwd_tc_kernel<128, __nv_bfloat16, false, true>, fa::TcCfg<128>::SMEM_BYTES);
+      ok &= set_smem_attr(fa::fa_fwd_tc_kernel<64, __half, false, true>, fa::TcCfg<64>::SMEM_BYTES);
+      ok &= set_smem_attr(fa::fa_fwd_tc_kernel<128, __half, false, true>, fa::TcCfg<128>::SMEM_BYTES);
       ok &= set_smem_attr(fa::fa_fwd_simt_kernel<64>, fa::simt_smem_bytes<64>());
       ok &= set_smem_attr(fa::fa_fwd_simt_kernel<128>, fa::simt_smem_bytes<128>());
       if (!ok) return FA_ERR_LAUNCH;
@@ -150,6 +154,11 @@ bool make_tmap_paged(CUtensorMap* tm, const void* base, bool bf16, int64_t Hkv, 
   return r == CUDA_SUCCESS;
 }
 
+// The band of fa_fwd_band: key j visible to query i iff i - pre <= j <= i + next.
+struct Band {
+  int pre_tokens, next_tokens;
+};
+
 // A paged K/V cache as fa_fwd_paged receives it.
 struct PagedKV {
   const int* block_table;  // [B, max_blocks] physical block of each logical block
@@ -172,7 +181,7 @@ int chunk_heads_for(int64_t BH, int64_t Nkv, int64_t D, int64_t group = 1) {
 template <int D, typename T>
 int launch_tc(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
               int64_t Hkv, int64_t Nq, int64_t Nkv, float scale, int causal, bool bsnd, cudaStream_t stream,
-              DeviceInfo& di, const PagedKV* pg = nullptr) {
+              DeviceInfo& di, const PagedKV* pg = nullptr, const Band* band = nullptr) {
   constexpr bool BF16 = std::is_same<T, __nv_bfloat16>::value;
   CUtensorMap tq, tk, tv;
   if (!make_tmap(&tq, q, BF16, bsnd, B, H, Nq, D)) return FA_ERR_LAUNCH;
@@ -202,11 +211,16 @@ int launch_tc(const void* q, const void* k, const void* v, void* o, float* lse, 
   p.block_size = pg != nullptr ? (int)pg->block_size : 0;
   p.max_blocks = pg != nullptr ? (int)pg->max_blocks : 0;
   p.num_blocks = pg != nullptr ? (int)pg->num_blocks : 0;
+  p.pre_tokens = band != nullptr ? band->pre_tokens : 0;
+  p.next_tokens = band != nullptr ? band->next_tokens : 0;
   p.sched = di.sched + (di.launches.fetch_add(1) % kSchedSlots);
   p.timeout_ns = (uint64_t)g_timeout_us.load() * 1000ull;
   p.fault_mode = g_fault_mode.load();
   const int grid = (int)(units < di.num_sms ? units : di.num_sms);
-  if (pg == nullptr)
+  if (band != nullptr)
+    fa::fa_fwd_tc_kernel<D, T, false, true><<<grid, fa::TC_THREADS, fa::TcCfg<D>::SMEM_BYTES, stream>>>(
+        tq, tk, tv, p, di.status);
+  else if (pg == nullptr)
     fa::fa_fwd_tc_kernel<D, T, false><<<grid, fa::TC_THREADS, fa::TcCfg<D>::SMEM_BYTES, stream>>>(tq, tk, tv, p,
                                                                                                   di.status);
   else
@@ -303,6 +317,47 @@ int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
   return fwd_common(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, d, scale, causal, layout, dtype, stream);
 }
 
+int fa_fwd_band(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
+                int64_t Hkv, int64_t Nq, int64_t Nkv, int64_t d, float scale, int64_t pre_tokens,
+                int64_t next_tokens, int layout, int dtype, void* stream) {
+  if (B < 0 || H < 0 || Hkv < 0 || Nq < 0 || Nkv < 0 || d <= 0 || pre_tokens < 0 || next_tokens < 0)
+    return FA_ERR_INVALID_ARG;
+  if (H > 0 && (Hkv < 1 || H % Hkv != 0)) return FA_ERR_INVALID_ARG;
+  if (layout != FA_LAYOUT_BHND && layout != FA_LAYOUT_BSND) return FA_ERR_INVALID_ARG;
+  if (dtype != FA_DTYPE_BF16 && dtype != FA_DTYPE_FP16 && dtype != FA_DTYPE_FP32) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (dtype == FA_DTYPE_FP32) return FA_ERR_UNSUPPORTED;  // the band path is the tensor-core kernel's
+  if (B == 0 || H == 0 || Nq == 0) return FA_OK;          // nothing to compute
+  if (Nkv == 0) return FA_ERR_INVALID_ARG;                // softmax over an empty key set
+  if (pre_tokens < Nq - Nkv) return FA_ERR_INVALID_ARG;   // the last query rows would see no key
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return FA_ERR_INVALID_ARG;
+  if (B > INT32_MAX || H > INT32_MAX || B * H > INT32_MAX || Nq > INT32_MAX - 256 || Nkv > INT32_MAX - 256)
+    return FA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      (lse != nullptr && !aligned(lse, 4)))
+    return FA_ERR_MISALIGNED;
+  if (!(scale > 0.f) || std::isinf(scale)) scale = 1.0f / std::sqrt((float)d);
+  // widths past the sequences change nothing; keep them in int range
+  const int64_t cap = Nq + Nkv;
+  const Band band{(int)(pre_tokens < cap ? pre_tokens : cap), (int)(next_tokens < cap ? next_tokens : cap)};
+
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_NO_DEVICE;
+  DeviceInfo* di = nullptr;
+  const int st = device_setup(dev, &di);
+  if (st != FA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool bsnd = layout == FA_LAYOUT_BSND;
+  if (dtype == FA_DTYPE_BF16)
+    return d == 64 ? launch_tc<64, __nv_bfloat16>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, 0, bsnd, s, *di,
+                                                  nullptr, &band)
+                   : launch_tc<128, __nv_bfloat16>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, 0, bsnd, s, *di,
+                                                   nullptr, &band);
+  return d == 64 ? launch_tc<64, __half>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, 0, bsnd, s, *di, nullptr, &band)
+                 : launch_tc<128, __half>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, 0, bsnd, s, *di, nullptr,
+                                          &band);
+}
+
 int fa_fwd_paged(const void* q, const void* k_cache, const void* v_cache, const int* block_table, void* o,
                  float* lse, int64_t B, int64_t H, int64_t Hkv, int64_t Nq, int64_t Nkv, int64_t d,
                  int64_t block_size, int64_t num_blocks, int64_t max_blocks, float scale, int causal, int layout,
@@ -377,7 +432,7 @@ uint32_t fa_set_wait_timeout_us(uint32_t us) {
 
 int fa_debug_set_fault(int mode) { return g_fault_mode.exchange(mode); }
 
-int fa_abi_version(void) { return (1 << 16) | 2; }
+int fa_abi_version(void) { return (1 << 16) | 3; }
 
 #ifdef FA_TRACE_UNITS
 int fa_debug_trace_units_read(unsigned long long* host, int n) {
@@ -497,6 +552,7 @@ int launch_tc_noalloc(const void* q, const void* k, const void* v, void* o, floa
   p.kv_group = 1;        // one K/V head per query head
   p.block_table = nullptr;  // contiguous K/V
   p.block_size = p.max_blocks = p.num_blocks = 0;
+  p.pre_tokens = p.next_tokens = 0;
   p.sched = nd.scratch;  // slot 0 of the static array
   p.timeout_ns = (uint64_t)g_timeout_us.load() * 1000ull;
   p.fault_mode = g_fault_mode.load();

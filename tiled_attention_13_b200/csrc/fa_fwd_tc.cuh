@@ -119,9 +119,9 @@ struct TcCfg {
   static constexpr int OFF_V = OFF_K + KST * TILE_BYTES;    // KST V tiles
   static constexpr int OFF_RED = OFF_V + KST * TILE_BYTES;  // [tile][parity][half][row] fp32 exchange
   static constexpr int RED_BYTES = 2 * 2 * 2 * TC_BM * 4;
-  static constexpr int OFF_UNIT = OFF_RED + RED_BYTES;      // ring of decoded work units (8 ints each)
+  static constexpr int OFF_UNIT = OFF_RED + RED_BYTES;      // ring of decoded work units (16 ints each)
   static constexpr int UNIT_SLOTS = 4;
-  static constexpr int OFF_BAR = OFF_UNIT + 32 * UNIT_SLOTS;  // barriers
+  static constexpr int OFF_BAR = OFF_UNIT + 64 * UNIT_SLOTS;  // barriers
   static constexpr int NBAR = 2 + 2 + 4 * KST + 2 + 4 + 2 + 1 + 2 + 2 * UNIT_SLOTS;
   static constexpr int SMEM_BYTES = OFF_BAR + NBAR * 8 + 16 /*tmem slot + abort*/ + 1024 /*align slack*/;
   static constexpr int TMEM_S0 = 0, TMEM_S1 = 128, TMEM_O0 = 256, TMEM_O1 = 256 + D;
@@ -153,6 +153,9 @@ struct TcParams {
   // n % block_size.  block_size is a power of two >= 16.
   const int* block_table;
   int block_size, max_blocks, num_blocks;
+  // Band (the kernel's BAND instantiation): key j is visible to query row i
+  // iff i - pre_tokens <= j <= i + next_tokens (and j < Nkv).
+  int pre_tokens, next_tokens;
   SchedSlot* sched;  // this launch's work-ticket counter
   uint64_t timeout_ns;
   int fault_mode;
@@ -163,6 +166,7 @@ struct Unit {
   int b, h, qt0;      // qt0 = first Q tile index (even), second = qt0 + 1
   int active1;        // second Q tile has at least one valid row
   int n0, n1;         // KV tiles for tile 0 / tile 1 (0 if inactive)
+  int lo0, s1;        // band: first KV tile of tile 0; tile 1 starts s1 tiles later (else 0, 0)
 };
 
 __device__ __forceinline__ int kv_tiles_for(int qt, int Nkv, int causal) {
@@ -197,6 +201,36 @@ __device__ __forceinline__ Unit decode_unit(int t, const TcParams& p) {
   return w;
 }
 
+// KV tile range [lo, hi) of Q tile qt under a band: the keys its rows can see,
+// [qt*128 - pre, qt*128 + 127 + next], cut to [0, Nkv).
+__device__ __forceinline__ int band_lo(int qt, const TcParams& p) {
+  const long long k = (long long)qt * TC_BM - p.pre_tokens;
+  return k <= 0 ? 0 : (int)(k / TC_BN);
+}
+__device__ __forceinline__ int band_hi(int qt, const TcParams& p) {
+  long long k = (long long)qt * TC_BM + TC_BM + p.next_tokens;  // one past the last visible key
+  if (k > p.Nkv) k = p.Nkv;
+  return (int)((k + TC_BN - 1) / TC_BN);
+}
+
+template <bool BAND>
+__device__ __forceinline__ Unit decode_unit_t(int t, const TcParams& p) {
+  Unit w = decode_unit(t, p);
+  w.lo0 = 0;
+  w.s1 = 0;
+  if constexpr (BAND) {
+    const int lo0 = band_lo(w.qt0, p);
+    w.lo0 = lo0;
+    w.n0 = band_hi(w.qt0, p) - lo0;
+    if (w.active1) {
+      const int lo1 = band_lo(w.qt0 + 1, p);
+      w.s1 = lo1 - lo0;
+      w.n1 = band_hi(w.qt0 + 1, p) - lo1;
+    }
+  }
+  return w;
+}
+
 template <typename T>
 struct Pack;
 template <>
@@ -220,7 +254,7 @@ struct Pack<__half> {
   }
 };
 
-template <int D, typename T, bool PAGED = false>
+template <int D, typename T, bool PAGED = false, bool BAND = false>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     fa_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, TcParams p, unsigned int* status_word) {
@@ -244,12 +278,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
   // Unit ring slot: ticket (-1 = no more work) and the decoded unit.
   auto ring_put = [&](int slot, int tk, const Unit& w) {
-    volatile int* e = unit_ring + 8 * slot;
+    volatile int* e = unit_ring + 16 * slot;
     e[0] = tk; e[1] = w.b; e[2] = w.h; e[3] = w.qt0; e[4] = w.active1; e[5] = w.n0; e[6] = w.n1;
+    e[7] = w.lo0; e[8] = w.s1;
   };
   auto ring_get = [&](int slot, Unit& w) -> int {
-    volatile const int* e = unit_ring + 8 * slot;
+    volatile const int* e = unit_ring + 16 * slot;
     w.b = e[1]; w.h = e[2]; w.qt0 = e[3]; w.active1 = e[4]; w.n0 = e[5]; w.n1 = e[6];
+    w.lo0 = BAND ? e[7] : 0;
+    w.s1 = BAND ? e[8] : 0;
     return e[0];
   };
 
@@ -348,7 +385,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         // (decoded here once: its integer divisions stay off the other roles)
         const unsigned int t = atomicAdd(&p.sched->next, 1u);
         const int tk = (t < (unsigned int)p.n_units) ? (int)t : -1;
-        const Unit w = decode_unit(tk < 0 ? 0 : tk, p);
+        const Unit w = decode_unit_t<BAND>(tk < 0 ? 0 : tk, p);
         if (!mbar_wait(bar(B_UEMPTY + uslot), uphase ^ 1, wctx)) break;
         ring_put(uslot, tk, w);
         mbar_arrive(bar(B_UFULL + uslot));
@@ -371,10 +408,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           q_phase[i] ^= 1;
         }
         FA_TRU(true, 0, n_claimed, 1);
-        const int N = w.n0 > w.n1 ? w.n0 : w.n1;
+        const int N = w.n0 > w.s1 + w.n1 ? w.n0 : w.s1 + w.n1;  // KV tiles lo0 .. lo0 + N - 1
         const int hk = w.h / p.kv_group;  // this unit's K/V head
         for (int j = 0; j < N && ok; ++j) {
-          const int kv0 = j * TC_BN;
+          const int kv0 = (w.lo0 + j) * TC_BN;
           if (!mbar_wait(bar(B_KEMPTY + st), kv_phase ^ 1, wctx)) { ok = false; break; }
           mbar_arrive_expect_tx(bar(B_KFULL + st), C::TILE_BYTES);
           const uint32_t kdst = sbase + C::OFF_K + st * C::TILE_BYTES;
@@ -456,8 +493,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       first_unit_m = false;
       (void)u_first;
       FA_TRU(lane == 0, 1, n_units_m, 0);
+      // Tile i takes part in KV steps [s_[i], s_[i] + n[i]) of the unit's walk
+      // over tiles lo0 .. lo0 + N - 1 (s_ = {0, 0} unless a band shifts tile 1).
       const int n[2] = {w.n0, w.n1};
-      const int N = w.n0 > w.n1 ? w.n0 : w.n1;
+      const int s_[2] = {0, BAND ? w.s1 : 0};
+      const int N = w.n0 > s_[1] + w.n1 ? w.n0 : s_[1] + w.n1;
       for (int i = 0; i < 2 && ok; ++i) {
         if (n[i] == 0) continue;
         if (!wait_all(B_QFULL + i, q_phase[i])) ok = false;
@@ -473,11 +513,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (j > 0 && !wait_all(B_VFULL + st_prev, ph_prev)) { ok = false; break; }
         FA_TR(lane == 0 && u_first, 17, j, 0);
         tc_fence_after();
-        if (PAGED && j > 0 && (j - 1) * TC_BN + TC_BN > p.Nkv) {
+        if (PAGED && j > 0 && ((BAND ? w.lo0 : 0) + j - 1) * TC_BN + TC_BN > p.Nkv) {
           // Rows past Nkv of this V tile hold whatever the cache has there
           // (stale or never written).  Their P is 0, but 0 x NaN would still
           // reach O: clear them before the P V that reads this tile.
-          const int r0 = p.Nkv - (j - 1) * TC_BN;
+          const int r0 = p.Nkv - ((BAND ? w.lo0 : 0) + j - 1) * TC_BN;
           const uint32_t vbase = sbase + C::OFF_V + st_prev * C::TILE_BYTES;
           for (int c = 0; c < C::CHUNKS; ++c)
             for (int i = r0 * 8 + lane; i < TC_BN * 8; i += 32)  // 8 x 16 bytes per 128-byte row
@@ -489,11 +529,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         const uint64_t dV = dV0 + (uint64_t)((st_prev * C::TILE_BYTES) >> 4);
         for (int i = 0; i < 2 && ok; ++i) {
           if (n[i] == 0) continue;
-          if (j >= 1 && j - 1 < n[i]) {
+          if (j >= 1 + s_[i] && j - 1 < s_[i] + n[i]) {
             // O_i += P_i(j-1) V_(j-1), in two parts as the softmax hands them
             // over: part q holds keys [32q, 32q+32) of both key halves, i.e.
             // k-steps {2q, 2q+1, 4+2q, 5+2q}.
-            const uint32_t acc0 = (j - 1 > 0) ? 1u : 0u;
+            const uint32_t acc0 = (j - 1 > s_[i]) ? 1u : 0u;
 #pragma unroll
             for (int part = 0; part < 2; ++part) {
               // k-steps 2q, 2q+1 (keys of half 0) and 4+2q, 5+2q (half 1);
@@ -510,14 +550,15 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
               mma_ts4_elect(tO[i], a0, b0, a1, b1, a2, b2, a3, b3, IDESC_PV, part == 0 ? acc0 : 1u);
             }
             if (!ok) break;
-            if (j - 1 == n[i] - 1) {
+            if (j - 1 == s_[i] + n[i] - 1) {
               mma_commit_elect(bar(B_OFULL + i));
               FA_TRU(lane == 0, 1, n_units_m, 2 + i);
             }
             // V_(j-1) is free once the last tile's P V has read it.
-            if (i == 1 || n[1] == 0 || j - 1 >= n[1]) mma_commit_elect(bar(B_VEMPTY + st_prev));
+            const bool t1_uses = n[1] > 0 && j - 1 >= s_[1] && j - 1 < s_[1] + n[1];
+            if (i == 1 || !t1_uses) mma_commit_elect(bar(B_VEMPTY + st_prev));
           }
-          if (j < n[i]) {
+          if (j >= s_[i] && j < s_[i] + n[i]) {
             if (!k_ready) {
               if (!wait_all(B_KFULL + st, kv_phase)) { ok = false; break; }
               k_ready = true;
@@ -533,11 +574,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             }
             mma_commit_elect(bar(B_SFULL + i));
             FA_TR(lane == 0 && u_first, 16 + i, j, 2);
-            if (j == 0) FA_TRU(lane == 0, 1, n_units_m, 4 + i);
-            if (j == n[i] - 1) mma_commit_elect(bar(B_QEMPTY + i));
+            if (j == s_[i]) FA_TRU(lane == 0, 1, n_units_m, 4 + i);
+            if (j == s_[i] + n[i] - 1) mma_commit_elect(bar(B_QEMPTY + i));
           }
         }
         if (!ok) break;
+        if (BAND && j >= 1) {
+          // a V tile no tile read (cannot happen for adjacent 128-row tiles,
+          // whose key ranges overlap or touch): release it all the same
+          const bool t0_uses = n[0] > 0 && j - 1 < n[0];
+          const bool t1_uses = n[1] > 0 && j - 1 >= s_[1] && j - 1 < s_[1] + n[1];
+          if (!t0_uses && !t1_uses) mma_commit_elect(bar(B_VEMPTY + st_prev));
+        }
         if (j < N) mma_commit_elect(bar(B_KEMPTY + st));
         FA_TR(lane == 0 && u_first, 16, j, 3);
         st_prev = st;
@@ -612,10 +660,22 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         FA_TRU(warp == 0 && lane == 0 && j == 0, 2, n_units_s, 1);
         s_phase ^= 1;
         tc_fence_after();
-        const int col0 = j * TC_BN + 64 * half;
-        const bool need_mask = (j * TC_BN + TC_BN > p.Nkv) || (p.causal && j * TC_BN + TC_BN - 1 > qt * TC_BM);
-        // visible columns of this row: [.., lim_c)
-        const int lim_c = p.causal ? (row + 1 < p.Nkv ? row + 1 : p.Nkv) : p.Nkv;
+        // KV tile of this step (a band starts the tile's walk at tile kt0)
+        const int kt = (BAND ? w.lo0 + (tile ? w.s1 : 0) : 0) + j;
+        const int col0 = kt * TC_BN + 64 * half;
+        bool need_mask = (kt * TC_BN + TC_BN > p.Nkv) || (p.causal && kt * TC_BN + TC_BN - 1 > qt * TC_BM);
+        // visible keys of this row: [lo_c, lim_c)
+        int lim_c = p.causal ? (row + 1 < p.Nkv ? row + 1 : p.Nkv) : p.Nkv;
+        int lo_c = 0;
+        if constexpr (BAND) {
+          const long long first = (long long)kt * TC_BN, last = first + TC_BN - 1;
+          need_mask = need_mask || first < (long long)qt * TC_BM + TC_BM - 1 - p.pre_tokens ||
+                      last > (long long)qt * TC_BM + p.next_tokens;
+          const long long hi = (long long)row + p.next_tokens + 1;
+          lim_c = hi < p.Nkv ? (int)hi : p.Nkv;
+          const long long lo = (long long)row - p.pre_tokens;
+          lo_c = lo > 0 ? (int)lo : 0;
+        }
         // This half's 64 scores stay in registers from the row max through the
         // exps (a second read of them from tensor memory delayed the P stores
         // behind it).
@@ -640,11 +700,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
             for (int g = 0; g < 4; ++g) {
               const int k0 = col0 + 16 * g;
-              if (__all_sync(0xffffffffu, k0 >= lim_c)) continue;
-              if (!__all_sync(0xffffffffu, k0 + 16 <= lim_c)) {
+              if (__all_sync(0xffffffffu, k0 >= lim_c || (BAND && k0 + 16 <= lo_c))) continue;
+              if (!__all_sync(0xffffffffu, k0 + 16 <= lim_c && (!BAND || k0 >= lo_c))) {
 #pragma unroll
                 for (int c = 0; c < 16; ++c)
-                  if (k0 + c >= lim_c) s[16 * g + c] = -INFINITY;
+                  if (k0 + c >= lim_c || (BAND && k0 + c < lo_c)) s[16 * g + c] = -INFINITY;
               }
 #pragma unroll
               for (int t = 0; t < 4; ++t) mx[t] = fmax3(mx[t], s[16 * g + t], s[16 * g + 4 + t]);
@@ -694,19 +754,20 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         auto sub = [&](const float* sc, int cbase, auto use_poly) {
           uint32_t pk[8];
           const int k0 = col0 + cbase;
-          if (!decltype(use_poly)::value && __all_sync(0xffffffffu, k0 >= lim_c)) {
+          if (!decltype(use_poly)::value && __all_sync(0xffffffffu, k0 >= lim_c || (BAND && k0 + 16 <= lo_c))) {
 #pragma unroll
             for (int t = 0; t < 8; ++t) pk[t] = 0u;
             tmem_st8(tS + cbase / 2, pk);
             return;
           }
-          const bool part = !decltype(use_poly)::value && !__all_sync(0xffffffffu, k0 + 16 <= lim_c);
+          const bool part =
+              !decltype(use_poly)::value && !__all_sync(0xffffffffu, k0 + 16 <= lim_c && (!BAND || k0 >= lo_c));
 #pragma unroll
           for (int t = 0; t < 8; ++t) {
             float v0 = sc[2 * t], v1 = sc[2 * t + 1];
             if (part) {
-              if (k0 + 2 * t >= lim_c) v0 = -INFINITY;
-              if (k0 + 2 * t + 1 >= lim_c) v1 = -INFINITY;
+              if (k0 + 2 * t >= lim_c || (BAND && k0 + 2 * t < lo_c)) v0 = -INFINITY;
+              if (k0 + 2 * t + 1 >= lim_c || (BAND && k0 + 2 * t + 1 < lo_c)) v1 = -INFINITY;
             }
             const uint64_t x2 = f2_fma(f2_pack(v0, v1), scale2, negm2);
             float p0, p1;

@@ -52,6 +52,7 @@ class Workload:
     outlier_frac: float = 0.0
     Hkv: int = 0  # K/V heads (grouped-query attention); 0 means H
     block_size: int = 0  # > 0: K/V read through a paged cache with blocks of this many keys
+    band: tuple = ()  # (pre_tokens, next_tokens): key j visible to query i iff i - pre <= j <= i + next
 
     @property
     def kv_heads(self) -> int:
@@ -59,7 +60,15 @@ class Workload:
 
     @property
     def flops(self) -> float:
-        """Algorithmic FLOPs: 4*B*H*Nq*Nkv*d, halved when causal."""
+        """Algorithmic FLOPs: 4*B*H*Nq*Nkv*d, halved when causal; with a band,
+        4*B*H*d times the number of visible (query, key) pairs."""
+        if self.band:
+            pre, nxt = self.band
+            i = torch.arange(self.Nq, dtype=torch.float64)
+            lo = torch.clamp(i - pre, min=0)
+            hi = torch.clamp(i + nxt, max=self.Nkv - 1)
+            pairs = float(torch.clamp(hi - lo + 1, min=0).sum())
+            return 4.0 * self.B * self.H * self.d * pairs
         f = 4.0 * self.B * self.H * self.Nq * self.Nkv * self.d
         return f / 2 if self.causal else f
 
@@ -103,6 +112,8 @@ WORKLOADS = {
                 k_outlier=3.0, outlier_frac=0.01),
     "llama13b-8k-gqa8": _wl("llama13b-8k-gqa8", 5, B=1, H=40, Hkv=8, Nq=8192, Nkv=8192, d=128, layout="BSND",
                             causal=True),
+    "llama13b-8k-swa2k": _wl("llama13b-8k-swa2k", 1, B=1, H=40, Nq=8192, Nkv=8192, d=128, layout="BSND",
+                             band=(2047, 0)),
     "llama13b-8k-gqa8-paged16": _wl("llama13b-8k-gqa8-paged16", 5, B=1, H=40, Hkv=8, Nq=8192, Nkv=8192, d=128,
                                     layout="BSND", causal=True, block_size=16),
 }

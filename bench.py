@@ -163,11 +163,13 @@ def oracle_sample(wl, rows_budget_s: float = 12.0, seed: int = 0):
     flops = 0.0
     t0 = time.perf_counter()
     rows_done = 0
-    # row blocks taken evenly over the sequence so causal work is representative
+    # row blocks taken evenly over the sequence so causal work is representative;
+    # when one head's rows take less than the budget (decoding: a row or a few),
+    # the same head's data stands for the workload's next heads, up to B*H
     starts = list(range(0, wl.Nq, block))
     rng = np.random.default_rng(seed)
     rng.shuffle(starts)
-    for r0 in starts:
+    for r0 in [r for _ in range(wl.B * wl.H) for r in starts]:
         r1 = min(wl.Nq, r0 + block)
         if wl.band:
             mask = band_mask(wl.Nq, wl.Nkv, wl.band[0], wl.band[1])[r0:r1]
@@ -187,7 +189,9 @@ def oracle_sample(wl, rows_budget_s: float = 12.0, seed: int = 0):
             break
     el = time.perf_counter() - t0
     threads = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
-    desc = f"{rows_done} query rows (blocks of {block}) of one head of {wl.name}, float64 numpy oracle"
+    heads_done = -(-rows_done // wl.Nq)
+    desc = (f"{rows_done} query rows (blocks of {block}) of one head of {wl.name}"
+            + (f", its data standing for {heads_done} heads" if heads_done > 1 else "") + ", float64 numpy oracle")
     return flops / el / 1e12, desc, threads, el
 
 
@@ -240,6 +244,7 @@ def _config(wl, ws):
             **({"Hkv": wl.kv_heads} if wl.kv_heads != wl.H else {}),
             **({"kv_cache": f"paged, {wl.block_size}-key blocks in shuffled order"} if wl.block_size > 0 else {}),
             **({"band": {"pre_tokens": wl.band[0], "next_tokens": wl.band[1]}} if wl.band else {}),
+            **({"num_splits": wl.num_splits} if wl.num_splits >= 0 else {}),
             "parallelism": f"independent replicas x{ws} (no collective)",
             "l2": (f"{n} input sets of {wl.bytes_min / 1e6:.1f} MB (Q, K, V, O, LSE) rotate between steps, "
                    f"{n * wl.bytes_min / 1e6:.0f} MB in all > 2x the 126 MB L2"),
@@ -277,13 +282,23 @@ def run_ours(args, wl):
         sets.append((q, k, v, o, lse, paged))
     torch.cuda.synchronize()
 
+    splits = wl.num_splits if wl.num_splits >= 0 else None
+    # kernels per step: the split kernel and the merge when the plan has
+    # more than one slice, else the one attention kernel
+    launches_per_step, s_used = 1, None
+    if splits is not None:
+        s_used, _ = fa.splitkv_plan(wl.B, wl.H, wl.Nq, wl.Nkv, wl.d, splits)
+        launches_per_step = 2 if s_used > 1 else 1
+
     def step(i):
         q, k, v, o, lse, paged = sets[i % n_sets]
         if paged is None:
-            fa.forward(q, k, v, causal=wl.causal, layout=wl.layout, out=o, lse=lse, band=wl.band or None)
+            fa.forward(q, k, v, causal=wl.causal, layout=wl.layout, out=o, lse=lse, band=wl.band or None,
+                       num_splits=splits)
         else:
             kc, vc, table = paged
-            fa.forward_paged(q, kc, vc, table, wl.Nkv, causal=wl.causal, layout=wl.layout, out=o, lse=lse)
+            fa.forward_paged(q, kc, vc, table, wl.Nkv, causal=wl.causal, layout=wl.layout, out=o, lse=lse,
+                             num_splits=splits)
 
     for i in range(args.warmup):
         step(i)
@@ -351,9 +366,9 @@ def run_ours(args, wl):
 
     # ---- end-to-end through the public API: pinned host in, host out
     e2e = None
-    if not args.no_e2e and (wl.block_size > 0 or wl.band):
-        e2e = {"value": None, "unit": UNIT, "skipped": "HostPipeline takes contiguous K/V without a band; this "
-               "path is measured on the device only"}
+    if not args.no_e2e and (wl.block_size > 0 or wl.band or splits is not None):
+        e2e = {"value": None, "unit": UNIT, "skipped": "HostPipeline takes contiguous K/V without a band or "
+               "split-KV; this path is measured on the device only"}
     elif not args.no_e2e:
         # Every step copies its inputs from pinned host memory and reads its
         # O and LSE back; HostPipeline overlaps step i+1's upload and step
@@ -387,7 +402,10 @@ def run_ours(args, wl):
         kmean = sum(kern_ms) / len(kern_ms)
         traffic = args.traffic if args.traffic is not None else captured_traffic(wl.name)
         achieved = wl.flops / (kmean * 1e-3) / 1e12
-        bound = "tensor" if wl.Nkv >= 512 else "hbm"
+        # the bound: tensor when the work's arithmetic intensity (algorithmic
+        # FLOPs per compulsory byte) is above the measured ridge point
+        ridge = float(peaks["bf16_tflops"]) * 1e12 / (float(peaks["hbm_gbs"]) * 1e9)
+        bound = "tensor" if wl.flops / wl.bytes_min >= ridge else "hbm"
         if bound == "tensor":
             peak = float(peaks["bf16_tflops"])
             roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
@@ -400,6 +418,9 @@ def run_ours(args, wl):
             roof = {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
                     "traffic": traffic, "peak_source": f"{src} hbm_gbs", "kernel_ms_mean": kmean,
                     "kernel_ms_min": min(kern_ms), "algorithmic_bytes": wl.bytes_min}
+        if launches_per_step > 1:
+            roof["timed"] = ("each step's event pair spans both kernels (split kernel and merge); achieved "
+                             "counts the compulsory bytes only")
         cpu = None
         if not args.no_cpu_baseline and ws == 1:
             tf, desc, threads, el = oracle_sample(wl, rows_budget_s=args.cpu_budget_s)
@@ -412,10 +433,12 @@ def run_ours(args, wl):
             "vs_baseline": None, "dtype": "bf16" if wl.dtype == "bf16" else wl.dtype,
             "data": "synthetic: seeded i.i.d. N(0,1) Q/K/V of the workload's shape",
             "config": _config(wl, ws), "roofline": roof, "cpu_baseline": cpu, "e2e": e2e,
-            "gpu_launches": args.steps, "clocks": clocks, "timing": "cuda-graph replay of the K steps" if use_graph
+            "gpu_launches": args.steps * launches_per_step, "clocks": clocks, "timing": "cuda-graph replay of the K steps" if use_graph
             else "eager launches",
             "pct_of_measured_bf16_peak": 100.0 * (value / ws) / float(peaks["bf16_tflops"]),
         }
+        if s_used is not None:
+            line["config"]["splits_used"] = s_used
         print(json.dumps(line), flush=True)
     if ws > 1:
         dist.barrier()
@@ -430,6 +453,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--workload", default="llama13b-8k")
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--num-splits", type=int, default=None,
+                    help="override the workload's split-KV setting: -1 unsplit, 0 the library's count, n slices")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-graph", action="store_true", help="launch the timed steps eagerly instead of as one CUDA graph")
     ap.add_argument("--no-cpu-baseline", action="store_true")
@@ -443,6 +468,8 @@ def main():
     from tiled_attention_13_b200.inputs import WORKLOADS
 
     wl = WORKLOADS[args.workload]
+    if args.num_splits is not None:
+        wl = wl.with_(num_splits=args.num_splits)
     if args.impl == "reference":
         return run_reference(args, wl)
     return run_ours(args, wl)

@@ -157,6 +157,77 @@ int fa_fwd_paged(const void* q, const void* k_cache, const void* v_cache, const 
                  int dtype, void* stream);
 
 /*
+ * Split-KV (flash-decoding) forms, for calls with few query rows per head
+ * (decoding: one new token per step against a long key cache, page 1,
+ * sections GatherPAKVCache 的显存管理逻辑 and the inference path's decode
+ * stage), where one unit per (batch, head, pair of 128-row query tiles)
+ * would leave most SMs idle while each unit walks every key tile.
+ *
+ * The key tiles (128 keys each) are cut into n_splits slices of equal length
+ * (the last may be shorter, none is empty).  A unit per (batch, head, tile
+ * pair, slice) computes its rows' attention over its slice alone: O_s,
+ * normalised, and LSE_s, written in fp32 to the caller's workspace.  A merge
+ * kernel then combines the slices with the online softmax's rule applied to
+ * whole slices (page 1, section 在线 Softmax 的数学原理拆解):
+ *     LSE = m + ln sum_s exp(LSE_s - m),  m = max_s LSE_s
+ *     O   = sum_s exp(LSE_s - LSE) O_s
+ * The result is attention over all Nkv keys, as from fa_fwd_gqa with
+ * causal = 0 (these forms take no mask: every query row sees every key, as
+ * a decoding step's new tokens see the whole cache).  O and LSE differ from
+ * the unsplit call only by rounding.
+ *
+ * fa_splitkv_plan -- the slice count and workspace size of a split-KV call.
+ *
+ *   num_splits       > 0: that many slices, at most one per key tile;
+ *                    <= 0: chosen by the library for num_sms SMs (a wave
+ *                    model of its persistent grid: enough units to fill the
+ *                    SMs in whole waves, slices no shorter than needed)
+ *   num_sms          SMs to plan for; <= 0: the current device's (which then
+ *                    needs a usable sm_100 device, else FA_ERR_NO_DEVICE)
+ *   *splits          out: the slice count the call will use (1 means the call
+ *                    runs the unsplit kernel and needs no workspace)
+ *   *workspace_bytes out: bytes of device workspace the call needs,
+ *                    splits * B*H*Nq * (d + 1) * 4, or 0 for one slice
+ *
+ * Errors: FA_ERR_INVALID_ARG (negative size, d not in {64, 128}, null out
+ * pointer), FA_ERR_UNSUPPORTED (sizes beyond the index range).
+ */
+int fa_splitkv_plan(int64_t B, int64_t H, int64_t Nq, int64_t Nkv, int64_t d, int num_splits, int num_sms,
+                    int* splits, int64_t* workspace_bytes);
+
+/*
+ * fa_fwd_splitkv -- fa_fwd_gqa (causal = 0) computed as above.
+ *
+ *   num_splits       as for fa_splitkv_plan, planned for the current device
+ *   workspace        device memory of at least the planned workspace_bytes,
+ *                    16-byte aligned, owned by the caller and not read after
+ *                    the call's work on `stream` has finished; it holds the
+ *                    slices' fp32 O [splits, B, H, Nq, d] and then their LSE
+ *                    [splits, B, H, Nq].  May be NULL when the plan has one
+ *                    slice.
+ *   workspace_bytes  its size in bytes
+ *   dtype            bf16 or fp16 (fp32 returns FA_ERR_UNSUPPORTED)
+ *
+ * The other arguments are as for fa_fwd_gqa.  Two kernels are launched on
+ * `stream` (the split kernel, then the merge), or one when the plan has one
+ * slice.  Errors as for fa_fwd_gqa, and FA_ERR_INVALID_ARG for a missing or
+ * too small workspace, FA_ERR_MISALIGNED for a misaligned one.
+ */
+int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
+                   int64_t Hkv, int64_t Nq, int64_t Nkv, int64_t d, float scale, int num_splits, void* workspace,
+                   int64_t workspace_bytes, int layout, int dtype, void* stream);
+
+/*
+ * fa_fwd_paged_splitkv -- fa_fwd_paged (causal = 0) computed as above: K and
+ * V through the paged cache and block table, described as for fa_fwd_paged;
+ * num_splits and the workspace as for fa_fwd_splitkv.
+ */
+int fa_fwd_paged_splitkv(const void* q, const void* k_cache, const void* v_cache, const int* block_table, void* o,
+                         float* lse, int64_t B, int64_t H, int64_t Hkv, int64_t Nq, int64_t Nkv, int64_t d,
+                         int64_t block_size, int64_t num_blocks, int64_t max_blocks, float scale, int num_splits,
+                         void* workspace, int64_t workspace_bytes, int layout, int dtype, void* stream);
+
+/*
  * fa_fwd_noalloc -- the same computation, arguments and results as fa_fwd,
  * for callers that must never allocate device memory: code that runs inside
  * a memory pool or arena it does not own, real-time or embedded services that
@@ -221,7 +292,8 @@ uint32_t fa_set_wait_timeout_us(uint32_t us);
  */
 int fa_debug_set_fault(int mode);
 
-/* ABI version of this header, (major << 16) | minor (1.1: fa_fwd_gqa, 1.2: fa_fwd_paged, 1.3: fa_fwd_band). */
+/* ABI version of this header, (major << 16) | minor (1.1: fa_fwd_gqa, 1.2: fa_fwd_paged, 1.3: fa_fwd_band,
+ * 1.4: fa_splitkv_plan, fa_fwd_splitkv, fa_fwd_paged_splitkv). */
 int fa_abi_version(void);
 
 #ifdef __cplusplus

@@ -49,6 +49,20 @@ int main(void) {
                       FA_LAYOUT_BSND, FA_DTYPE_FP32, NULL),
          FA_ERR_UNSUPPORTED, "paged fp32");
 
+  {
+    int splits = 0;
+    int64_t ws = -1;
+    expect(fa_splitkv_plan(1, 40, 1, 8192, 128, 5, 148, &splits, &ws), FA_OK, "split-KV plan");
+    expect(splits, 5, "split-KV plan: slices");
+    if (ws != (int64_t)5 * 40 * 129 * 4) ++failures;
+  }
+  expect(fa_fwd_splitkv(a16, a16, a16, a16, l16, 1, 4, 2, 1, 1000, 128, -1.0f, 0, a16, 1 << 20, FA_LAYOUT_BSND,
+                        FA_DTYPE_FP32, NULL),
+         FA_ERR_UNSUPPORTED, "split-KV fp32");
+  expect(fa_fwd_paged_splitkv(a16, a16, a16, (const int*)a16, a16, l16, 1, 4, 2, 1, 1000, 128, 128, 9, 7, -1.0f, 0,
+                              a16, 1 << 20, FA_LAYOUT_BSND, FA_DTYPE_BF16, NULL),
+         FA_ERR_INVALID_ARG, "paged split-KV short table");
+
   uint32_t prev = fa_set_wait_timeout_us(5000);
   expect((int)fa_set_wait_timeout_us(prev), 5000, "timeout setting round trip");
 

@@ -34,7 +34,7 @@ def test_status_strings_and_version(fa_lib):
     for code in range(8):
         assert fa.fa_status_string(code).startswith("FA_")
     assert fa.fa_status_string(99) == "FA_ERR_UNKNOWN"
-    assert fa.fa_abi_version() == (1 << 16) | 3
+    assert fa.fa_abi_version() == (1 << 16) | 4
 
 
 def test_host_settings_roundtrip(fa_lib):
@@ -120,6 +120,87 @@ def test_band_validation_before_any_cuda_call(fa_lib, kw, code):
                         args["Nq"], args["Nkv"], args["d"], args["scale"], args["pre"], args["nxt"], args["layout"],
                         args["dtype"], args["stream"])
     assert rc == code, fa.fa_status_string(rc)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(B=-1), 1), (dict(Hkv=3), 1), (dict(layout=2), 1), (dict(dtype=3), 1), (dict(ws_bytes=-1), 1),
+    (dict(Nkv=0), 1), (dict(q=None), 1),
+    (dict(dtype=2), 2), (dict(d=96), 2), (dict(B=1 << 31), 2),
+    (dict(q=A16 + 8), 3), (dict(lse=A16 + 2), 3),
+    (dict(B=0), 0), (dict(Nq=0), 0),
+])
+def test_splitkv_validation_before_any_cuda_call(fa_lib, kw, code):
+    """fa_fwd_splitkv: fa_fwd_gqa's checks (no causal flag), bf16/fp16 only,
+    a non-negative workspace size; the workspace itself is checked against
+    the plan, which needs the device."""
+    args = dict(q=A16, k=A16, v=A16, o=A16, lse=A16, B=1, H=4, Hkv=2, Nq=1, Nkv=1000, d=128, scale=-1.0, S=0,
+                ws=A16, ws_bytes=1 << 20, layout=1, dtype=0, stream=None)
+    args.update(kw)
+    rc = fa.fa_fwd_splitkv(args["q"], args["k"], args["v"], args["o"], args["lse"], args["B"], args["H"],
+                           args["Hkv"], args["Nq"], args["Nkv"], args["d"], args["scale"], args["S"], args["ws"],
+                           args["ws_bytes"], args["layout"], args["dtype"], args["stream"])
+    assert rc == code, fa.fa_status_string(rc)
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(block_size=24), 1), (dict(max_blocks=7), 1), (dict(num_blocks=0), 1), (dict(bt=None), 1),
+    (dict(dtype=2), 2), (dict(bt=A16 + 2), 3), (dict(Nq=0), 0),
+])
+def test_paged_splitkv_validation_before_any_cuda_call(fa_lib, kw, code):
+    """fa_fwd_paged_splitkv: fa_fwd_paged's table and block checks (1000 keys
+    in blocks of 128 need 8 table entries)."""
+    args = dict(q=A16, kc=A16, vc=A16, bt=A16, o=A16, lse=A16, B=1, H=4, Hkv=2, Nq=1, Nkv=1000, d=128,
+                block_size=128, num_blocks=9, max_blocks=8, scale=-1.0, S=0, ws=A16, ws_bytes=1 << 20, layout=1,
+                dtype=0, stream=None)
+    args.update(kw)
+    rc = fa.fa_fwd_paged_splitkv(args["q"], args["kc"], args["vc"], args["bt"], args["o"], args["lse"], args["B"],
+                                 args["H"], args["Hkv"], args["Nq"], args["Nkv"], args["d"], args["block_size"],
+                                 args["num_blocks"], args["max_blocks"], args["scale"], args["S"], args["ws"],
+                                 args["ws_bytes"], args["layout"], args["dtype"], args["stream"])
+    assert rc == code, fa.fa_status_string(rc)
+
+
+def _plan_cost(base, nt, s, sms):
+    """The plan's wave model, written out: slices of ceil(nt / s) tiles."""
+    t = -(-nt // s)
+    sc = -(-nt // t)
+    return -(-base * sc // sms) * (t + 1), sc
+
+
+@pytest.mark.parametrize("B,H,Nq,Nkv", [(1, 40, 1, 8192), (8, 32, 1, 32768), (1, 8, 7, 129), (2, 8, 4096, 77),
+                                        (1, 40, 8192, 8192), (1, 1, 1, 1), (1, 2, 300, 100000)])
+def test_splitkv_plan_follows_its_wave_model(fa_lib, B, H, Nq, Nkv):
+    """fa_splitkv_plan with an explicit SM count (no GPU needed): the chosen
+    slice count has the least modelled cost of every count up to about four
+    units per SM, no slice is empty, and the workspace is splits * B*H*Nq *
+    (d + 1) fp32 values (none for one slice)."""
+    sms, d = 148, 128
+    S, nbytes = fa.splitkv_plan(B, H, Nq, Nkv, d, 0, sms)
+    nt = -(-Nkv // 128)
+    base = B * H * (-(-(-(-Nq // 128)) // 2))
+    smax = min(nt, -(-4 * sms // base), 4096)
+    costs = [_plan_cost(base, nt, s, sms) for s in range(1, smax + 1)]
+    best = min(c for c, _ in costs)
+    assert _plan_cost(base, nt, S, sms)[0] == best
+    t = -(-nt // S)
+    assert (S - 1) * t < nt <= S * t  # every slice holds at least one tile
+    assert nbytes == (S * B * H * Nq * (d + 1) * 4 if S > 1 else 0)
+
+
+def test_splitkv_plan_explicit_counts(fa_lib):
+    """An explicit count is capped at one slice per key tile and rounded so
+    that no slice is empty: 64 tiles in 5 asked slices are 5 slices of 13
+    (the last 12); 3 tiles in 9 asked slices are 3."""
+    assert fa.splitkv_plan(1, 40, 1, 8192, 128, 5, 148) == (5, 5 * 40 * 129 * 4)
+    assert fa.splitkv_plan(1, 40, 1, 300, 128, 9, 148) == (3, 3 * 40 * 129 * 4)
+    assert fa.splitkv_plan(1, 40, 1, 8192, 64, 1, 148) == (1, 0)
+    assert fa.splitkv_plan(1, 40, 1, 8192, 64, 64, 148) == (64, 64 * 40 * 65 * 4)
+    # 7 tiles in 4 asked slices: slices of 2 tiles, so 4 slices (2, 2, 2, 1)
+    assert fa.splitkv_plan(1, 1, 1, 7 * 128, 128, 4, 148)[0] == 4
+    # 9 tiles in 4 asked slices: slices of 3 tiles, so 3 slices
+    assert fa.splitkv_plan(1, 1, 1, 9 * 128, 128, 4, 148)[0] == 3
+    rc, _, _ = fa.fa_splitkv_plan(1, 1, 1, 100, 96, 0, 148)
+    assert rc == 1
 
 
 def test_product_path_has_no_cpu_fallback(monkeypatch, tmp_path):

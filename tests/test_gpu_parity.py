@@ -203,10 +203,11 @@ def test_gqa_llama13b_8k_sampled():
 
 
 # ----------------------------------------------------------------- paged K/V cache
-def _paged_parity(wl):
+def _paged_parity(wl, num_splits=None):
     """forward_paged on a cache built from the seeded K/V (shuffled physical
     blocks, NaN in every element the table does not point at) against the
-    oracle's gather-then-attend on the same cache and table."""
+    oracle's gather-then-attend on the same cache and table; with num_splits,
+    the split-KV form of the same call."""
     from oracle import attention_paged
     from tiled_attention_13_b200.inputs import make_paged_kv
 
@@ -215,7 +216,7 @@ def _paged_parity(wl):
     q, k, v = make_qkv(wl)
     kc, vc, table = make_paged_kv(wl, k, v)
     o, lse = fa.forward_paged(q.cuda(), kc.cuda(), vc.cuda(), table.cuda(), wl.Nkv, causal=wl.causal,
-                              layout=wl.layout)
+                              layout=wl.layout, num_splits=num_splits)
     torch.cuda.synchronize()
     assert fa.fa_get_device_status(None) == 0
     o_ref, l_ref = attention_paged(q, kc, vc, table.numpy(), wl.Nkv, causal=wl.causal, layout=wl.layout)
@@ -339,3 +340,66 @@ def test_long_context_sampled():
     heads = [(0, 0), (0, wl.H - 1)]
     compare_sampled(wl, heads, rows_per_head=24)
     torch.cuda.empty_cache()
+
+
+# ----------------------------------------------------------------- split-KV
+SPLIT_CASES = [  # (B, H, Hkv, Nq, Nkv, d, layout, dtype, num_splits); 0 = the library's count
+    (1, 8, 2, 1, 4097, 128, "BSND", "bf16", 0),     # decode-shaped, ragged last key tile
+    (2, 4, 4, 7, 1000, 64, "BHND", "bf16", 3),      # ragged last slice and tile
+    (1, 4, 1, 300, 2000, 128, "BSND", "bf16", 5),   # three Q tiles: a pair with an inactive second tile; MQA
+    (1, 2, 2, 1, 128, 128, "BSND", "bf16", 4),      # one key tile: one slice, the unsplit kernel
+    (1, 2, 2, 129, 9000, 64, "BHND", "bf16", 71),   # one key tile per slice, two Q tiles
+    (1, 6, 3, 5, 3000, 128, "BHND", "fp16", 0),     # fp16
+    (1, 40, 40, 1, 8192, 128, "BSND", "bf16", 0),   # the LLaMA-13B decode step's shape
+]
+
+
+@pytest.mark.parametrize("case", SPLIT_CASES, ids=lambda c: "x".join(map(str, c[:6])) + c[6] + c[7] + f"s{c[8]}")
+def test_splitkv(case):
+    """fa_fwd_splitkv (slices of the key tiles, fp32 partials, LSE merge)
+    against the oracle's attention over all keys."""
+    from oracle import attention_batched
+
+    from .parity import LSE_TOL, o_bar
+
+    B, H, hkv, nq, nkv, d, layout, dtype, S = case
+    wl = Workload("splitkv", B=B, H=H, Hkv=hkv, Nq=nq, Nkv=nkv, d=d, dtype=dtype, layout=layout, causal=False,
+                  seed=nq + nkv + S)
+    q, k, v = make_qkv(wl)
+    o, lse = fa.forward(q.cuda(), k.cuda(), v.cuda(), layout=layout, num_splits=S)
+    torch.cuda.synchronize()
+    assert fa.fa_get_device_status(None) == 0
+    o_ref, l_ref = attention_batched(q, k, v, causal=False, layout=layout)
+    o_gpu, l_gpu = o.double().cpu().numpy(), lse.double().cpu().numpy()
+    assert np.all(np.isfinite(o_gpu)) and np.all(np.isfinite(l_gpu))
+    err_o = np.abs(o_gpu - o_ref)
+    assert np.all(err_o <= o_bar(o_ref, dtype)), float(err_o.max())
+    assert np.abs(l_gpu - l_ref).max() <= LSE_TOL, float(np.abs(l_gpu - l_ref).max())
+
+
+@pytest.mark.parametrize("num_splits", [0, 3])
+@pytest.mark.parametrize("block_size", [16, 128])
+def test_paged_splitkv(block_size, num_splits):
+    """fa_fwd_paged_splitkv on decode shapes: one and seven query rows per head
+    against 4097 keys in a shuffled paged cache (NaN wherever the table does
+    not point)."""
+    for nq in (1, 7):
+        wl = Workload("decode", B=2, H=8, Hkv=2, Nq=nq, Nkv=4097, d=128, dtype="bf16", layout="BSND", causal=False,
+                      seed=nq + block_size + num_splits, block_size=block_size)
+        _paged_parity(wl, num_splits=num_splits)
+
+
+def test_splitkv_rejects_a_short_workspace():
+    """The workspace is checked against the plan before anything is launched."""
+    B, H, nq, nkv, d = 1, 4, 1, 4096, 128
+    S, nbytes = fa.splitkv_plan(B, H, nq, nkv, d, 4)
+    assert S == 4 and nbytes > 0
+    x = torch.zeros((B, nkv, H, d), dtype=torch.bfloat16, device="cuda")
+    o = torch.empty((B, nq, H, d), dtype=torch.bfloat16, device="cuda")
+    lse = torch.empty((B, H, nq), dtype=torch.float32, device="cuda")
+    ws = torch.empty(nbytes, dtype=torch.uint8, device="cuda")
+    args = (x.data_ptr(), x.data_ptr(), x.data_ptr(), o.data_ptr(), lse.data_ptr(), B, H, H, nq, nkv, d, -1.0, 4)
+    assert fa.fa_fwd_splitkv(*args, ws.data_ptr(), nbytes - 16, fa.FA_LAYOUT_BSND, fa.FA_DTYPE_BF16, None) == 1
+    assert fa.fa_fwd_splitkv(*args, None, 0, fa.FA_LAYOUT_BSND, fa.FA_DTYPE_BF16, None) == 1
+    assert fa.fa_fwd_splitkv(*args, ws.data_ptr() + 4, nbytes - 16, fa.FA_LAYOUT_BSND, fa.FA_DTYPE_BF16, None) == 1
+    assert fa.fa_fwd_splitkv(*args, ws.data_ptr() + 4, nbytes, fa.FA_LAYOUT_BSND, fa.FA_DTYPE_BF16, None) == 3

@@ -24,7 +24,7 @@ import os
 __all__ = [
     "FA_LAYOUT_BHND", "FA_LAYOUT_BSND", "FA_DTYPE_BF16", "FA_DTYPE_FP16", "FA_DTYPE_FP32",
     "FaError", "lib", "lib_path", "fa_fwd", "fa_fwd_gqa", "fa_fwd_band", "fa_fwd_paged", "fa_fwd_noalloc",
-    "fa_status_string",
+    "fa_splitkv_plan", "fa_fwd_splitkv", "fa_fwd_paged_splitkv", "splitkv_plan", "fa_status_string",
     "fa_get_device_status", "fa_set_wait_timeout_us", "fa_debug_set_fault", "fa_abi_version", "forward",
     "forward_paged", "forward_host",
     "HostForward", "HostPipeline", "EXPORTED",
@@ -34,8 +34,8 @@ FA_LAYOUT_BHND, FA_LAYOUT_BSND = 0, 1
 FA_DTYPE_BF16, FA_DTYPE_FP16, FA_DTYPE_FP32 = 0, 1, 2
 FA_OK = 0
 
-EXPORTED = ("fa_fwd", "fa_fwd_gqa", "fa_fwd_band", "fa_fwd_paged", "fa_fwd_noalloc", "fa_status_string",
-            "fa_get_device_status", "fa_set_wait_timeout_us", "fa_debug_set_fault", "fa_abi_version")
+EXPORTED = ("fa_fwd", "fa_fwd_gqa", "fa_fwd_band", "fa_fwd_paged", "fa_fwd_noalloc", "fa_splitkv_plan",
+            "fa_fwd_splitkv", "fa_fwd_paged_splitkv", "fa_status_string", "fa_get_device_status", "fa_set_wait_timeout_us", "fa_debug_set_fault", "fa_abi_version")
 
 _LIB = None
 
@@ -75,6 +75,15 @@ def lib() -> ctypes.CDLL:
     L.fa_fwd_paged.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64, i64, i64, ctypes.c_float,
                                ctypes.c_int, ctypes.c_int, ctypes.c_int, vp]
     L.fa_fwd_paged.restype = ctypes.c_int
+    L.fa_splitkv_plan.argtypes = [i64, i64, i64, i64, i64, ctypes.c_int, ctypes.c_int, ctypes.POINTER(ctypes.c_int),
+                                  ctypes.POINTER(i64)]
+    L.fa_splitkv_plan.restype = ctypes.c_int
+    L.fa_fwd_splitkv.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, ctypes.c_float, ctypes.c_int, vp,
+                                 i64, ctypes.c_int, ctypes.c_int, vp]
+    L.fa_fwd_splitkv.restype = ctypes.c_int
+    L.fa_fwd_paged_splitkv.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64, i64, i64,
+                                       ctypes.c_float, ctypes.c_int, vp, i64, ctypes.c_int, ctypes.c_int, vp]
+    L.fa_fwd_paged_splitkv.restype = ctypes.c_int
     L.fa_status_string.argtypes = [ctypes.c_int]
     L.fa_status_string.restype = ctypes.c_char_p
     L.fa_get_device_status.argtypes = [vp]
@@ -119,6 +128,29 @@ def fa_fwd_paged(q, k_cache, v_cache, block_table, o, lse, B, H, Hkv, Nq, Nkv, d
     Hkv, d] and an int32 block table [B, max_blocks]."""
     return lib().fa_fwd_paged(q, k_cache, v_cache, block_table, o, lse, B, H, Hkv, Nq, Nkv, d, block_size,
                               num_blocks, max_blocks, float(scale), int(causal), int(layout), int(dtype), stream)
+
+
+def fa_splitkv_plan(B, H, Nq, Nkv, d, num_splits, num_sms):
+    """int fa_splitkv_plan(...) -> (status, splits, workspace_bytes)."""
+    sp, wb = ctypes.c_int(0), ctypes.c_int64(0)
+    rc = lib().fa_splitkv_plan(B, H, Nq, Nkv, d, int(num_splits), int(num_sms), ctypes.byref(sp), ctypes.byref(wb))
+    return rc, sp.value, wb.value
+
+
+def fa_fwd_splitkv(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, d, scale, num_splits, workspace, workspace_bytes, layout,
+                   dtype, stream) -> int:
+    """int fa_fwd_splitkv(...): non-causal attention with the key tiles cut into
+    slices, each slice's (O, LSE) in the fp32 workspace, then merged."""
+    return lib().fa_fwd_splitkv(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, d, float(scale), int(num_splits), workspace,
+                                int(workspace_bytes), int(layout), int(dtype), stream)
+
+
+def fa_fwd_paged_splitkv(q, k_cache, v_cache, block_table, o, lse, B, H, Hkv, Nq, Nkv, d, block_size, num_blocks,
+                         max_blocks, scale, num_splits, workspace, workspace_bytes, layout, dtype, stream) -> int:
+    """int fa_fwd_paged_splitkv(...): fa_fwd_splitkv with K/V through a paged cache."""
+    return lib().fa_fwd_paged_splitkv(q, k_cache, v_cache, block_table, o, lse, B, H, Hkv, Nq, Nkv, d, block_size,
+                                      num_blocks, max_blocks, float(scale), int(num_splits), workspace,
+                                      int(workspace_bytes), int(layout), int(dtype), stream)
 
 
 def fa_fwd_noalloc(q, k, v, o, lse, B, H, Nq, Nkv, d, scale, causal, layout, dtype, stream) -> int:
@@ -171,8 +203,33 @@ def _kv_heads(k, layout):
     return k.shape[1] if layout == "BHND" else k.shape[2]
 
 
+def splitkv_plan(B, H, Nq, Nkv, d, num_splits: int = 0, num_sms: int = 0):
+    """(splits, workspace_bytes) of a split-KV call: num_splits <= 0 lets the
+    library choose for num_sms SMs (<= 0: the current device's)."""
+    rc, sp, wb = fa_splitkv_plan(B, H, Nq, Nkv, d, num_splits, num_sms)
+    if rc != FA_OK:
+        raise FaError(rc, "fa_splitkv_plan")
+    return sp, wb
+
+
+def _splitkv_workspace(B, H, Nq, Nkv, d, num_splits, device, stream, user_stream):
+    """Device workspace for a split-KV call (None when the plan has one
+    slice).  Taken from torch's caching allocator; when the call runs on a
+    stream other than the current one, the block is tied to that stream so
+    that it is not reused before the call's kernels finish."""
+    import torch
+
+    _, nbytes = splitkv_plan(B, H, Nq, Nkv, d, num_splits)
+    if nbytes == 0:
+        return None
+    ws = torch.empty(nbytes, dtype=torch.uint8, device=device)
+    if user_stream:
+        ws.record_stream(torch.cuda.ExternalStream(stream, device=device))
+    return ws
+
+
 def forward(q, k, v, causal: bool = False, scale=None, layout: str = "BHND", out=None, lse=None,
-            stream=None, band=None):
+            stream=None, band=None, num_splits=None):
     """O, LSE = softmax(scale Q K^T [+causal]) V on the GPU (returns (o, lse)).
 
     q: [B,H,Nq,d] (BHND) or [B,Nq,H,d] (BSND); k, v the same with Nkv and
@@ -181,6 +238,9 @@ def forward(q, k, v, causal: bool = False, scale=None, layout: str = "BHND", out
     scale None -> 1/sqrt(d).  LSE is fp32 [B, H, Nq].  band = (pre_tokens,
     next_tokens) replaces ``causal``: key j visible to query i iff
     i - pre_tokens <= j <= i + next_tokens (fa_fwd_band; bf16/fp16).
+    num_splits (not None; bf16/fp16, no mask) runs split-KV (fa_fwd_splitkv):
+    the key tiles cut into that many slices, or as many as the library
+    chooses for this device when it is 0.
     """
     import torch
 
@@ -196,12 +256,23 @@ def forward(q, k, v, causal: bool = False, scale=None, layout: str = "BHND", out
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    user_stream = stream is not None
     if stream is None:
         stream = torch.cuda.current_stream(q.device).cuda_stream
     sc = -1.0 if scale is None else float(scale)
     Hkv = _kv_heads(k, layout)
     lay = FA_LAYOUT_BHND if layout == "BHND" else FA_LAYOUT_BSND
     lp = lse.data_ptr() if lse.numel() else None
+    if num_splits is not None:
+        if causal or band is not None:
+            raise ValueError("split-KV takes no mask (causal=False, band=None)")
+        ws = _splitkv_workspace(B, H, Nq, Nkv, d, int(num_splits), q.device, stream, user_stream)
+        rc = fa_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lp, B, H, Hkv, Nq, Nkv, d, sc,
+                            int(num_splits), None if ws is None else ws.data_ptr(), 0 if ws is None else ws.numel(),
+                            lay, _dtype_code(q), stream)
+        if rc != FA_OK:
+            raise FaError(rc, "fa_fwd_splitkv")
+        return out, lse
     if band is not None:
         if causal:
             raise ValueError("give either causal or band")
@@ -223,12 +294,14 @@ def forward(q, k, v, causal: bool = False, scale=None, layout: str = "BHND", out
 
 
 def forward_paged(q, k_cache, v_cache, block_table, seq_len: int, causal: bool = False, scale=None,
-                  layout: str = "BSND", out=None, lse=None, stream=None):
+                  layout: str = "BSND", out=None, lse=None, stream=None, num_splits=None):
     """O, LSE with K and V gathered through a paged cache (returns (o, lse)).
 
     q: [B,H,Nq,d] (BHND) or [B,Nq,H,d] (BSND), bf16 or fp16; k_cache, v_cache:
     [num_blocks, block_size, Hkv, d] of q's dtype; block_table: int32
     [B, max_blocks] CUDA tensor; seq_len: keys per sequence.  All contiguous.
+    num_splits (not None, causal False) runs split-KV (fa_fwd_paged_splitkv),
+    as for forward().
     """
     import torch
 
@@ -250,9 +323,22 @@ def forward_paged(q, k_cache, v_cache, block_table, seq_len: int, causal: bool =
         out = torch.empty_like(q)
     if lse is None:
         lse = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device)
+    user_stream = stream is not None
     if stream is None:
         stream = torch.cuda.current_stream(q.device).cuda_stream
     sc = -1.0 if scale is None else float(scale)
+    if num_splits is not None:
+        if causal:
+            raise ValueError("split-KV takes no mask (causal=False)")
+        ws = _splitkv_workspace(B, H, Nq, int(seq_len), d, int(num_splits), q.device, stream, user_stream)
+        rc = fa_fwd_paged_splitkv(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_table.data_ptr(),
+                                  out.data_ptr(), lse.data_ptr() if lse.numel() else None, B, H, Hkv, Nq, int(seq_len),
+                                  d, block_size, num_blocks, block_table.shape[1], sc, int(num_splits),
+                                  None if ws is None else ws.data_ptr(), 0 if ws is None else ws.numel(),
+                                  FA_LAYOUT_BHND if layout == "BHND" else FA_LAYOUT_BSND, _dtype_code(q), stream)
+        if rc != FA_OK:
+            raise FaError(rc, "fa_fwd_paged_splitkv")
+        return out, lse
     rc = fa_fwd_paged(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), block_table.data_ptr(), out.data_ptr(),
                       lse.data_ptr() if lse.numel() else None, B, H, Hkv, Nq, int(seq_len), d, block_size,
                       num_blocks, block_table.shape[1], sc, int(bool(causal)),

@@ -24,6 +24,7 @@ __device__ unsigned int g_status_word = 0;
 
 #include "fa_fwd_simt.cuh"
 #include "fa_fwd_tc.cuh"
+#include "fa_splitkv_merge.cuh"
 
 namespace {
 
@@ -84,6 +85,14 @@ int device_setup(int dev, DeviceInfo** out) {
       ok &= set_smem_attr(fa::fa_fwd_tc_kernel<128, __nv_bfloat16, false, true>, fa::TcCfg<128>::SMEM_BYTES);
       ok &= set_smem_attr(fa::fa_fwd_tc_kernel<64, __half, false, true>, fa::TcCfg<64>::SMEM_BYTES);
       ok &= set_smem_attr(fa::fa_fwd_tc_kernel<128, __half, false, true>, fa::TcCfg<128>::SMEM_BYTES);
+      ok &= set_smem_attr(fa::fa_fwd_tc_kernel<64, __nv_bfloat16, false, false, true>, fa::TcCfg<64>::SMEM_BYTES);
+      ok &= set_smem_attr(fa::fa_fwd_tc_kernel<128, __nv_bfloat16, false, false, true>, fa::TcCfg<128>::SMEM_BYTES);
+      ok &= set_smem_attr(fa::fa_fwd_tc_kernel<64, __half, false, false, true>, fa::TcCfg<64>::SMEM_BYTES);
+      ok &= set_smem_attr(fa::fa_fwd_tc_kernel<128, __half, false, false, true>, fa::TcCfg<128>::SMEM_BYTES);
+      ok &= set_smem_attr(fa::fa_fwd_tc_kernel<64, __nv_bfloat16, true, false, true>, fa::TcCfg<64>::SMEM_BYTES);
+      ok &= set_smem_attr(fa::fa_fwd_tc_kernel<128, __nv_bfloat16, true, false, true>, fa::TcCfg<128>::SMEM_BYTES);
+      ok &= set_smem_attr(fa::fa_fwd_tc_kernel<64, __half, true, false, true>, fa::TcCfg<64>::SMEM_BYTES);
+      ok &= set_smem_attr(fa::fa_fwd_tc_kernel<128, __half, true, false, true>, fa::TcCfg<128>::SMEM_BYTES);
       ok &= set_smem_attr(fa::fa_fwd_simt_kernel<64>, fa::simt_smem_bytes<64>());
       ok &= set_smem_attr(fa::fa_fwd_simt_kernel<128>, fa::simt_smem_bytes<128>());
       if (!ok) return FA_ERR_LAUNCH;
@@ -165,6 +174,50 @@ struct PagedKV {
   int64_t block_size, num_blocks, max_blocks;
 };
 
+// Split-KV as launch_tc receives it: the plan and the caller's workspace,
+// o_part [n_splits, B, H, Nq, D] then lse_part [n_splits, B, H, Nq], fp32.
+struct SplitKV {
+  int n_splits, split_tiles;
+  float* o_part;
+  float* lse_part;
+};
+
+// The split-KV plan: the KV tiles of every (batch, head, Q-tile pair) cut
+// into n_splits slices of split_tiles tiles, the last possibly shorter and
+// none empty.  requested > 0 asks for that many slices (at most one per KV
+// tile).  requested <= 0 picks the count with a wave model of the persistent
+// grid: base_units * n_splits equal units over num_sms CTAs take
+// ceil(units / num_sms) waves of (split_tiles + 1) tile steps each, the + 1
+// standing for a unit's fixed cost (its Q load, the pipeline's fill and the
+// epilogue); the first count with the lowest cost wins, trying up to about
+// four units per SM.
+void split_plan(int64_t base_units, int64_t kv_tiles, int requested, int num_sms, int* n_splits,
+                int* split_tiles) {
+  int64_t S = 1;
+  if (requested > 0) {
+    S = requested < kv_tiles ? requested : kv_tiles;
+  } else if (base_units > 0 && num_sms > 0) {
+    int64_t smax = (4 * (int64_t)num_sms + base_units - 1) / base_units;
+    if (smax > kv_tiles) smax = kv_tiles;
+    if (smax > 4096) smax = 4096;
+    int64_t best_cost = INT64_MAX;
+    for (int64_t c = 1; c <= smax; ++c) {
+      const int64_t t = (kv_tiles + c - 1) / c;
+      const int64_t sc = (kv_tiles + t - 1) / t;
+      const int64_t waves = (base_units * sc + num_sms - 1) / num_sms;
+      const int64_t cost = waves * (t + 1);
+      if (cost < best_cost) {
+        best_cost = cost;
+        S = c;
+      }
+    }
+  }
+  if (S < 1) S = 1;
+  const int64_t t = (kv_tiles + S - 1) / S;
+  *split_tiles = (int)t;
+  *n_splits = (int)((kv_tiles + t - 1) / t);
+}
+
 // (batch, head) pairs per scheduling chunk: enough that the chunk's K and V
 // (2 * Nkv * D * 2 bytes per K/V head, shared by `group` consecutive query
 // heads) stay within a comfortable share of the 126 MB L2 while every CTA
@@ -181,7 +234,8 @@ int chunk_heads_for(int64_t BH, int64_t Nkv, int64_t D, int64_t group = 1) {
 template <int D, typename T>
 int launch_tc(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
               int64_t Hkv, int64_t Nq, int64_t Nkv, float scale, int causal, bool bsnd, cudaStream_t stream,
-              DeviceInfo& di, const PagedKV* pg = nullptr, const Band* band = nullptr) {
+              DeviceInfo& di, const PagedKV* pg = nullptr, const Band* band = nullptr,
+              const SplitKV* sk = nullptr) {
   constexpr bool BF16 = std::is_same<T, __nv_bfloat16>::value;
   CUtensorMap tq, tk, tv;
   if (!make_tmap(&tq, q, BF16, bsnd, B, H, Nq, D)) return FA_ERR_LAUNCH;
@@ -194,15 +248,15 @@ int launch_tc(const void* q, const void* k, const void* v, void* o, float* lse, 
       return FA_ERR_LAUNCH;
   }
   fa::TcParams p;
-  p.o = o;
-  p.lse = lse;
+  p.o = sk != nullptr ? static_cast<void*>(sk->o_part) : o;  // split: the kernel writes the slices' partials
+  p.lse = sk != nullptr ? sk->lse_part : lse;
   p.B = (int)B; p.H = (int)H; p.Nq = (int)Nq; p.Nkv = (int)Nkv;
   p.bsnd = bsnd ? 1 : 0;
   p.causal = causal;
   p.scale_log2 = scale * 1.4426950408889634f;
   const int64_t qtiles = (Nq + fa::TC_BM - 1) / fa::TC_BM;
   p.n_pairs = (int)((qtiles + 1) / 2);
-  const int64_t units = B * H * (int64_t)p.n_pairs;
+  const int64_t units = B * H * (int64_t)p.n_pairs * (sk != nullptr ? sk->n_splits : 1);
   if (units > INT32_MAX) return FA_ERR_UNSUPPORTED;
   p.n_units = (int)units;
   p.chunk_heads = chunk_heads_for(B * H, Nkv, D, H / Hkv);
@@ -211,8 +265,13 @@ int launch_tc(const void* q, const void* k, const void* v, void* o, float* lse, 
   p.block_size = pg != nullptr ? (int)pg->block_size : 0;
   p.max_blocks = pg != nullptr ? (int)pg->max_blocks : 0;
   p.num_blocks = pg != nullptr ? (int)pg->num_blocks : 0;
-  p.pre_tokens = band != nullptr ? band->pre_tokens : 0;
-  p.next_tokens = band != nullptr ? band->next_tokens : 0;
+  if (sk != nullptr) {
+    p.split.n_splits = sk->n_splits;
+    p.split.split_tiles = sk->split_tiles;
+  } else {
+    p.band.pre_tokens = band != nullptr ? band->pre_tokens : 0;
+    p.band.next_tokens = band != nullptr ? band->next_tokens : 0;
+  }
   p.sched = di.sched + (di.launches.fetch_add(1) % kSchedSlots);
   p.timeout_ns = (uint64_t)g_timeout_us.load() * 1000ull;
   p.fault_mode = g_fault_mode.load();
@@ -220,13 +279,27 @@ int launch_tc(const void* q, const void* k, const void* v, void* o, float* lse, 
   if (band != nullptr)
     fa::fa_fwd_tc_kernel<D, T, false, true><<<grid, fa::TC_THREADS, fa::TcCfg<D>::SMEM_BYTES, stream>>>(
         tq, tk, tv, p, di.status);
+  else if (sk != nullptr && pg == nullptr)
+    fa::fa_fwd_tc_kernel<D, T, false, false, true><<<grid, fa::TC_THREADS, fa::TcCfg<D>::SMEM_BYTES, stream>>>(
+        tq, tk, tv, p, di.status);
+  else if (sk != nullptr)
+    fa::fa_fwd_tc_kernel<D, T, true, false, true><<<grid, fa::TC_THREADS, fa::TcCfg<D>::SMEM_BYTES, stream>>>(
+        tq, tk, tv, p, di.status);
   else if (pg == nullptr)
     fa::fa_fwd_tc_kernel<D, T, false><<<grid, fa::TC_THREADS, fa::TcCfg<D>::SMEM_BYTES, stream>>>(tq, tk, tv, p,
                                                                                                   di.status);
   else
     fa::fa_fwd_tc_kernel<D, T, true><<<grid, fa::TC_THREADS, fa::TcCfg<D>::SMEM_BYTES, stream>>>(tq, tk, tv, p,
                                                                                                  di.status);
-  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  if (sk != nullptr) {  // combine the slices into O and LSE, in stream order
+    const int64_t rows = B * H * Nq;
+    const int64_t blocks = (rows + fa::MERGE_ROWS_PER_CTA - 1) / fa::MERGE_ROWS_PER_CTA;
+    fa::fa_splitkv_merge_kernel<D, T><<<(unsigned int)blocks, fa::MERGE_THREADS, 0, stream>>>(
+        sk->o_part, sk->lse_part, static_cast<T*>(o), lse, (int)B, (int)H, (int)Nq, sk->n_splits, bsnd ? 1 : 0);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  }
+  return FA_OK;
 }
 
 template <int D>
@@ -253,10 +326,6 @@ int launch_simt(const void* q, const void* k, const void* v, void* o, float* lse
 inline bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
 }  // namespace
-
-extern "C" {
-
-}  // extern "C"
 
 namespace {
 
@@ -300,6 +369,71 @@ int fwd_common(const void* q, const void* k, const void* v, void* o, float* lse,
   }
   return d == 64 ? launch_tc<64, __half>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s, *di)
                  : launch_tc<128, __half>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s, *di);
+}
+
+// Bytes of split-KV workspace for n_splits slices (none for one slice).
+int64_t split_workspace_bytes(int64_t B, int64_t H, int64_t Nq, int64_t d, int n_splits) {
+  return n_splits > 1 ? (int64_t)n_splits * B * H * Nq * (d + 1) * 4 : 0;
+}
+
+// fa_fwd_splitkv and fa_fwd_paged_splitkv: validation (in the order the
+// header states), the plan, then the split kernel and the merge, or the plain
+// kernel when the plan has one slice.  pg == nullptr: contiguous K/V.
+int splitkv_common(const void* q, const void* k, const void* v, const PagedKV* pg, void* o, float* lse, int64_t B,
+                   int64_t H, int64_t Hkv, int64_t Nq, int64_t Nkv, int64_t d, float scale, int num_splits,
+                   void* workspace, int64_t workspace_bytes, int layout, int dtype, void* stream) {
+  if (B < 0 || H < 0 || Hkv < 0 || Nq < 0 || Nkv < 0 || d <= 0 || workspace_bytes < 0) return FA_ERR_INVALID_ARG;
+  if (H > 0 && (Hkv < 1 || H % Hkv != 0)) return FA_ERR_INVALID_ARG;
+  if (layout != FA_LAYOUT_BHND && layout != FA_LAYOUT_BSND) return FA_ERR_INVALID_ARG;
+  if (dtype != FA_DTYPE_BF16 && dtype != FA_DTYPE_FP16 && dtype != FA_DTYPE_FP32) return FA_ERR_INVALID_ARG;
+  if (pg != nullptr && (pg->block_size <= 0 || pg->num_blocks < 0 || pg->max_blocks < 0 ||
+                        (pg->block_size & (pg->block_size - 1)) != 0 || pg->block_size < 16))
+    return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (dtype == FA_DTYPE_FP32) return FA_ERR_UNSUPPORTED;  // split-KV is the tensor-core kernel's
+  if (B == 0 || H == 0 || Nq == 0) return FA_OK;          // nothing to compute
+  if (Nkv == 0) return FA_ERR_INVALID_ARG;                // softmax over an empty key set
+  if (pg != nullptr && (pg->num_blocks == 0 || pg->max_blocks < (Nkv + pg->block_size - 1) / pg->block_size))
+    return FA_ERR_INVALID_ARG;
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || (pg != nullptr && pg->block_table == nullptr))
+    return FA_ERR_INVALID_ARG;
+  if (B > INT32_MAX || H > INT32_MAX || B * H > INT32_MAX || Nq > INT32_MAX - 256 || Nkv > INT32_MAX - 256)
+    return FA_ERR_UNSUPPORTED;
+  if (pg != nullptr && (pg->block_size > (1 << 20) || pg->num_blocks > INT32_MAX - 1 ||
+                        pg->max_blocks > INT32_MAX || B * pg->max_blocks > INT32_MAX))
+    return FA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      (lse != nullptr && !aligned(lse, 4)) || (pg != nullptr && !aligned(pg->block_table, 4)))
+    return FA_ERR_MISALIGNED;
+  if (!(scale > 0.f) || std::isinf(scale)) scale = 1.0f / std::sqrt((float)d);
+
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_NO_DEVICE;
+  DeviceInfo* di = nullptr;
+  const int st = device_setup(dev, &di);
+  if (st != FA_OK) return st;
+  const int64_t qtiles = (Nq + fa::TC_BM - 1) / fa::TC_BM;
+  int S = 1, tiles = 0;
+  split_plan(B * H * ((qtiles + 1) / 2), (Nkv + fa::TC_BN - 1) / fa::TC_BN, num_splits, di->num_sms, &S, &tiles);
+  const int64_t need = split_workspace_bytes(B, H, Nq, d, S);
+  if (need > 0) {
+    if (workspace == nullptr || workspace_bytes < need) return FA_ERR_INVALID_ARG;
+    if (!aligned(workspace, 16)) return FA_ERR_MISALIGNED;
+  }
+  const SplitKV sk{S, tiles, static_cast<float*>(workspace),
+                   need > 0 ? reinterpret_cast<float*>(static_cast<char*>(workspace) + (int64_t)S * B * H * Nq * d * 4)
+                            : nullptr};
+  const SplitKV* skp = S > 1 ? &sk : nullptr;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool bsnd = layout == FA_LAYOUT_BSND;
+  if (dtype == FA_DTYPE_BF16)
+    return d == 64 ? launch_tc<64, __nv_bfloat16>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, 0, bsnd, s, *di, pg,
+                                                  nullptr, skp)
+                   : launch_tc<128, __nv_bfloat16>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, 0, bsnd, s, *di, pg,
+                                                   nullptr, skp);
+  return d == 64 ? launch_tc<64, __half>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, 0, bsnd, s, *di, pg, nullptr, skp)
+                 : launch_tc<128, __half>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, 0, bsnd, s, *di, pg, nullptr,
+                                          skp);
 }
 
 }  // namespace
@@ -404,6 +538,47 @@ int fa_fwd_paged(const void* q, const void* k_cache, const void* v_cache, const 
                                           *di, &pg);
 }
 
+int fa_splitkv_plan(int64_t B, int64_t H, int64_t Nq, int64_t Nkv, int64_t d, int num_splits, int num_sms,
+                    int* splits, int64_t* workspace_bytes) {
+  if (B < 0 || H < 0 || Nq < 0 || Nkv < 0 || (d != 64 && d != 128) || splits == nullptr ||
+      workspace_bytes == nullptr)
+    return FA_ERR_INVALID_ARG;
+  if (B > INT32_MAX || H > INT32_MAX || B * H > INT32_MAX || Nq > INT32_MAX - 256 || Nkv > INT32_MAX - 256)
+    return FA_ERR_UNSUPPORTED;
+  if (num_sms <= 0) {
+    int dev = -1;
+    if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_NO_DEVICE;
+    DeviceInfo* di = nullptr;
+    const int st = device_setup(dev, &di);
+    if (st != FA_OK) return st;
+    num_sms = di->num_sms;
+  }
+  int S = 1, tiles = 0;
+  if (B > 0 && H > 0 && Nq > 0 && Nkv > 0) {
+    const int64_t qtiles = (Nq + fa::TC_BM - 1) / fa::TC_BM;
+    split_plan(B * H * ((qtiles + 1) / 2), (Nkv + fa::TC_BN - 1) / fa::TC_BN, num_splits, num_sms, &S, &tiles);
+  }
+  *splits = S;
+  *workspace_bytes = split_workspace_bytes(B, H, Nq, d, S);
+  return FA_OK;
+}
+
+int fa_fwd_splitkv(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
+                   int64_t Hkv, int64_t Nq, int64_t Nkv, int64_t d, float scale, int num_splits, void* workspace,
+                   int64_t workspace_bytes, int layout, int dtype, void* stream) {
+  return splitkv_common(q, k, v, nullptr, o, lse, B, H, Hkv, Nq, Nkv, d, scale, num_splits, workspace,
+                        workspace_bytes, layout, dtype, stream);
+}
+
+int fa_fwd_paged_splitkv(const void* q, const void* k_cache, const void* v_cache, const int* block_table, void* o,
+                         float* lse, int64_t B, int64_t H, int64_t Hkv, int64_t Nq, int64_t Nkv, int64_t d,
+                         int64_t block_size, int64_t num_blocks, int64_t max_blocks, float scale, int num_splits,
+                         void* workspace, int64_t workspace_bytes, int layout, int dtype, void* stream) {
+  const PagedKV pg{block_table, block_size, num_blocks, max_blocks};
+  return splitkv_common(q, k_cache, v_cache, &pg, o, lse, B, H, Hkv, Nq, Nkv, d, scale, num_splits, workspace,
+                        workspace_bytes, layout, dtype, stream);
+}
+
 const char* fa_status_string(int status) {
   switch (status) {
     case FA_OK: return "FA_OK";
@@ -432,7 +607,7 @@ uint32_t fa_set_wait_timeout_us(uint32_t us) {
 
 int fa_debug_set_fault(int mode) { return g_fault_mode.exchange(mode); }
 
-int fa_abi_version(void) { return (1 << 16) | 3; }
+int fa_abi_version(void) { return (1 << 16) | 4; }
 
 #ifdef FA_TRACE_UNITS
 int fa_debug_trace_units_read(unsigned long long* host, int n) {
@@ -552,7 +727,7 @@ int launch_tc_noalloc(const void* q, const void* k, const void* v, void* o, floa
   p.kv_group = 1;        // one K/V head per query head
   p.block_table = nullptr;  // contiguous K/V
   p.block_size = p.max_blocks = p.num_blocks = 0;
-  p.pre_tokens = p.next_tokens = 0;
+  p.band.pre_tokens = p.band.next_tokens = 0;
   p.sched = nd.scratch;  // slot 0 of the static array
   p.timeout_ns = (uint64_t)g_timeout_us.load() * 1000ull;
   p.fault_mode = g_fault_mode.load();

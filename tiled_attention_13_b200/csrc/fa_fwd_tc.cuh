@@ -137,6 +137,10 @@ struct SchedSlot {
 };
 
 struct TcParams {
+  // O and LSE; under split-KV (the kernel's SPLIT instantiation) the fp32
+  // per-slice results instead: o -> o_part [n_splits, B, H, Nq, D] and
+  // lse -> lse_part [n_splits, B, H, Nq], each slice's rows normalised over
+  // that slice alone, combined afterwards by the merge kernel.
   void* o;
   float* lse;
   int B, H, Nq, Nkv;
@@ -153,9 +157,21 @@ struct TcParams {
   // n % block_size.  block_size is a power of two >= 16.
   const int* block_table;
   int block_size, max_blocks, num_blocks;
-  // Band (the kernel's BAND instantiation): key j is visible to query row i
-  // iff i - pre_tokens <= j <= i + next_tokens (and j < Nkv).
-  int pre_tokens, next_tokens;
+  // The one mode-specific pair of ints (the parameter block keeps its size:
+  // a larger one changed the register allocation of every instantiation).
+  //   band (BAND): key j is visible to query row i iff
+  //     i - pre_tokens <= j <= i + next_tokens (and j < Nkv);
+  //   split (SPLIT): the KV tiles are cut into n_splits slices of
+  //     split_tiles tiles (the last may be shorter, none is empty), one unit
+  //     per (batch, head, Q-tile pair, slice).
+  union {
+    struct {
+      int pre_tokens, next_tokens;
+    } band;
+    struct {
+      int n_splits, split_tiles;
+    } split;
+  };
   SchedSlot* sched;  // this launch's work-ticket counter
   uint64_t timeout_ns;
   int fault_mode;
@@ -166,7 +182,7 @@ struct Unit {
   int b, h, qt0;      // qt0 = first Q tile index (even), second = qt0 + 1
   int active1;        // second Q tile has at least one valid row
   int n0, n1;         // KV tiles for tile 0 / tile 1 (0 if inactive)
-  int lo0, s1;        // band: first KV tile of tile 0; tile 1 starts s1 tiles later (else 0, 0)
+  int lo0, s1;        // band / split: first KV tile of tile 0; tile 1 starts s1 tiles later (else 0, 0)
 };
 
 __device__ __forceinline__ int kv_tiles_for(int qt, int Nkv, int causal) {
@@ -204,17 +220,47 @@ __device__ __forceinline__ Unit decode_unit(int t, const TcParams& p) {
 // KV tile range [lo, hi) of Q tile qt under a band: the keys its rows can see,
 // [qt*128 - pre, qt*128 + 127 + next], cut to [0, Nkv).
 __device__ __forceinline__ int band_lo(int qt, const TcParams& p) {
-  const long long k = (long long)qt * TC_BM - p.pre_tokens;
+  const long long k = (long long)qt * TC_BM - p.band.pre_tokens;
   return k <= 0 ? 0 : (int)(k / TC_BN);
 }
 __device__ __forceinline__ int band_hi(int qt, const TcParams& p) {
-  long long k = (long long)qt * TC_BM + TC_BM + p.next_tokens;  // one past the last visible key
+  long long k = (long long)qt * TC_BM + TC_BM + p.band.next_tokens;  // one past the last visible key
   if (k > p.Nkv) k = p.Nkv;
   return (int)((k + TC_BN - 1) / TC_BN);
 }
 
-template <bool BAND>
-__device__ __forceinline__ Unit decode_unit_t(int t, const TcParams& p) {
+// Split-KV ticket t -> unit and its slice index sp.  The (batch, head)
+// chunks are walked as in decode_unit; a head's units are its (Q-tile pair,
+// slice) pairs, the slice index fastest.  Both Q tiles of a pair take the
+// same slice of KV tiles (no mask but the sequence end).
+__device__ __forceinline__ Unit decode_unit_split(int t, const TcParams& p, int& sp) {
+  Unit w;
+  const int BH = p.B * p.H;
+  const int per_chunk = p.chunk_heads * p.n_pairs * p.split.n_splits;  // <= n_units < 2^31
+  const int chunk = t / per_chunk;
+  const int idx = t - chunk * per_chunk;
+  const int h0 = chunk * p.chunk_heads;
+  const int g = (BH - h0 < p.chunk_heads) ? (BH - h0) : p.chunk_heads;
+  const int ps = idx / g;
+  const int bh = h0 + (idx - ps * g);
+  const int pair = ps / p.split.n_splits;
+  sp = ps - pair * p.split.n_splits;
+  w.b = bh / p.H;
+  w.h = bh % p.H;
+  w.qt0 = 2 * pair;
+  w.active1 = ((long long)(w.qt0 + 1) * TC_BM < (long long)p.Nq) ? 1 : 0;
+  const int nt = (p.Nkv + TC_BN - 1) / TC_BN;
+  w.lo0 = sp * p.split.split_tiles;
+  const int n = (nt - w.lo0 < p.split.split_tiles) ? nt - w.lo0 : p.split.split_tiles;
+  w.n0 = n;
+  w.n1 = w.active1 ? n : 0;
+  w.s1 = 0;
+  return w;
+}
+
+template <bool BAND, bool SPLIT>
+__device__ __forceinline__ Unit decode_unit_t(int t, const TcParams& p, int& sp) {
+  if constexpr (SPLIT) return decode_unit_split(t, p, sp);
   Unit w = decode_unit(t, p);
   w.lo0 = 0;
   w.s1 = 0;
@@ -254,11 +300,14 @@ struct Pack<__half> {
   }
 };
 
-template <int D, typename T, bool PAGED = false, bool BAND = false>
+template <int D, typename T, bool PAGED = false, bool BAND = false, bool SPLIT = false>
 __global__ void __launch_bounds__(TC_THREADS, 1)
     fa_fwd_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
                      const __grid_constant__ CUtensorMap tm_v, TcParams p, unsigned int* status_word) {
   using C = TcCfg<D>;
+  static_assert(!(BAND && SPLIT), "a band and split-KV are separate instantiations");
+  // A band or a split walks each unit over its own range of KV tiles.
+  constexpr bool WALK = BAND || SPLIT;
   constexpr bool IS_BF16 = std::is_same<T, __nv_bfloat16>::value;
   extern __shared__ uint8_t smem_raw[];
   // 1024-byte alignment: the 128-byte swizzle pattern is anchored there.
@@ -277,16 +326,18 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
   // Unit ring slot: ticket (-1 = no more work) and the decoded unit.
-  auto ring_put = [&](int slot, int tk, const Unit& w) {
+  // A split's slice index rides in e[9], outside Unit.
+  auto ring_put = [&](int slot, int tk, const Unit& w, int sp) {
     volatile int* e = unit_ring + 16 * slot;
     e[0] = tk; e[1] = w.b; e[2] = w.h; e[3] = w.qt0; e[4] = w.active1; e[5] = w.n0; e[6] = w.n1;
     e[7] = w.lo0; e[8] = w.s1;
+    if constexpr (SPLIT) e[9] = sp;
   };
   auto ring_get = [&](int slot, Unit& w) -> int {
     volatile const int* e = unit_ring + 16 * slot;
     w.b = e[1]; w.h = e[2]; w.qt0 = e[3]; w.active1 = e[4]; w.n0 = e[5]; w.n1 = e[6];
-    w.lo0 = BAND ? e[7] : 0;
-    w.s1 = BAND ? e[8] : 0;
+    w.lo0 = WALK ? e[7] : 0;
+    w.s1 = WALK ? e[8] : 0;
     return e[0];
   };
 
@@ -385,9 +436,10 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         // (decoded here once: its integer divisions stay off the other roles)
         const unsigned int t = atomicAdd(&p.sched->next, 1u);
         const int tk = (t < (unsigned int)p.n_units) ? (int)t : -1;
-        const Unit w = decode_unit_t<BAND>(tk < 0 ? 0 : tk, p);
+        int sp = 0;
+        const Unit w = decode_unit_t<BAND, SPLIT>(tk < 0 ? 0 : tk, p, sp);
         if (!mbar_wait(bar(B_UEMPTY + uslot), uphase ^ 1, wctx)) break;
-        ring_put(uslot, tk, w);
+        ring_put(uslot, tk, w, sp);
         mbar_arrive(bar(B_UFULL + uslot));
         if (++uslot == C::UNIT_SLOTS) { uslot = 0; uphase ^= 1; }
         if (tk < 0) break;
@@ -496,7 +548,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       // Tile i takes part in KV steps [s_[i], s_[i] + n[i]) of the unit's walk
       // over tiles lo0 .. lo0 + N - 1 (s_ = {0, 0} unless a band shifts tile 1).
       const int n[2] = {w.n0, w.n1};
-      const int s_[2] = {0, BAND ? w.s1 : 0};
+      const int s_[2] = {0, WALK ? w.s1 : 0};
       const int N = w.n0 > s_[1] + w.n1 ? w.n0 : s_[1] + w.n1;
       for (int i = 0; i < 2 && ok; ++i) {
         if (n[i] == 0) continue;
@@ -513,11 +565,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         if (j > 0 && !wait_all(B_VFULL + st_prev, ph_prev)) { ok = false; break; }
         FA_TR(lane == 0 && u_first, 17, j, 0);
         tc_fence_after();
-        if (PAGED && j > 0 && ((BAND ? w.lo0 : 0) + j - 1) * TC_BN + TC_BN > p.Nkv) {
+        if (PAGED && j > 0 && ((WALK ? w.lo0 : 0) + j - 1) * TC_BN + TC_BN > p.Nkv) {
           // Rows past Nkv of this V tile hold whatever the cache has there
           // (stale or never written).  Their P is 0, but 0 x NaN would still
           // reach O: clear them before the P V that reads this tile.
-          const int r0 = p.Nkv - ((BAND ? w.lo0 : 0) + j - 1) * TC_BN;
+          const int r0 = p.Nkv - ((WALK ? w.lo0 : 0) + j - 1) * TC_BN;
           const uint32_t vbase = sbase + C::OFF_V + st_prev * C::TILE_BYTES;
           for (int c = 0; c < C::CHUNKS; ++c)
             for (int i = r0 * 8 + lane; i < TC_BN * 8; i += 32)  // 8 x 16 bytes per 128-byte row
@@ -579,7 +631,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
           }
         }
         if (!ok) break;
-        if (BAND && j >= 1) {
+        if (WALK && j >= 1) {
           // a V tile no tile read (cannot happen for adjacent 128-row tiles,
           // whose key ranges overlap or touch): release it all the same
           const bool t0_uses = n[0] > 0 && j - 1 < n[0];
@@ -640,6 +692,7 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       if (!ok) break;
       Unit w;
       const int tk = ring_get(uslot, w);
+      const int sp = SPLIT ? unit_ring[16 * uslot + 9] : 0;  // split-KV: this unit's slice
       mbar_arrive_warp(bar(B_UEMPTY + uslot));
       if (++uslot == C::UNIT_SLOTS) { uslot = 0; uphase ^= 1; }
       if (tk < 0) break;
@@ -660,8 +713,8 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         FA_TRU(warp == 0 && lane == 0 && j == 0, 2, n_units_s, 1);
         s_phase ^= 1;
         tc_fence_after();
-        // KV tile of this step (a band starts the tile's walk at tile kt0)
-        const int kt = (BAND ? w.lo0 + (tile ? w.s1 : 0) : 0) + j;
+        // KV tile of this step (a band or a split starts the tile's walk at lo0 (+ s1))
+        const int kt = (WALK ? w.lo0 + (tile ? w.s1 : 0) : 0) + j;
         const int col0 = kt * TC_BN + 64 * half;
         bool need_mask = (kt * TC_BN + TC_BN > p.Nkv) || (p.causal && kt * TC_BN + TC_BN - 1 > qt * TC_BM);
         // visible keys of this row: [lo_c, lim_c)
@@ -669,11 +722,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         int lo_c = 0;
         if constexpr (BAND) {
           const long long first = (long long)kt * TC_BN, last = first + TC_BN - 1;
-          need_mask = need_mask || first < (long long)qt * TC_BM + TC_BM - 1 - p.pre_tokens ||
-                      last > (long long)qt * TC_BM + p.next_tokens;
-          const long long hi = (long long)row + p.next_tokens + 1;
+          need_mask = need_mask || first < (long long)qt * TC_BM + TC_BM - 1 - p.band.pre_tokens ||
+                      last > (long long)qt * TC_BM + p.band.next_tokens;
+          const long long hi = (long long)row + p.band.next_tokens + 1;
           lim_c = hi < p.Nkv ? (int)hi : p.Nkv;
-          const long long lo = (long long)row - p.pre_tokens;
+          const long long lo = (long long)row - p.band.pre_tokens;
           lo_c = lo > 0 ? (int)lo : 0;
         }
         // This half's 64 scores stay in registers from the row max through the
@@ -886,6 +939,27 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       tc_fence_after();
       const float inv_l = 1.f / l;
       const bool valid = row < p.Nq;
+      if constexpr (SPLIT) {
+        // This slice's normalised half row of O, in fp32, and the row's LSE
+        // over the slice.  The TMEM loads are warp-wide; only the stores
+        // depend on the row.
+        const long long prow = (((long long)sp * p.B + w.b) * p.H + w.h) * p.Nq + row;
+        float* op = static_cast<float*>(p.o) + prow * D + (D / 2) * half;
+#pragma unroll 1
+        for (int c = 0; c < D / 2; c += 32) {
+          float ov[32];
+          tmem_ld32(tO + c, ov);
+          if (valid) {
+#pragma unroll
+            for (int t = 0; t < 8; ++t)
+              *reinterpret_cast<float4*>(op + c + 4 * t) =
+                  make_float4(ov[4 * t] * inv_l, ov[4 * t + 1] * inv_l, ov[4 * t + 2] * inv_l, ov[4 * t + 3] * inv_l);
+          }
+        }
+        if (valid && half == 0) p.lse[prow] = (m_ref + __log2f(l)) * 0.69314718055994530942f;
+        ++n_units_s;
+        continue;
+      }
       // This half row of O as bf16/fp16 pairs: 16-byte chunk k = pk[4k..4k+3].
       constexpr int NC = D / 16;  // chunks per half row: 8 (d=128) or 4 (d=64)
       uint32_t pk[D / 4];

@@ -53,6 +53,7 @@ class Workload:
     Hkv: int = 0  # K/V heads (grouped-query attention); 0 means H
     block_size: int = 0  # > 0: K/V read through a paged cache with blocks of this many keys
     band: tuple = ()  # (pre_tokens, next_tokens): key j visible to query i iff i - pre <= j <= i + next
+    num_splits: int = -1  # >= 0: split-KV with that many slices of the key tiles (0: the library's count)
 
     @property
     def kv_heads(self) -> int:
@@ -116,6 +117,12 @@ WORKLOADS = {
                              band=(2047, 0)),
     "llama13b-8k-gqa8-paged16": _wl("llama13b-8k-gqa8-paged16", 5, B=1, H=40, Hkv=8, Nq=8192, Nkv=8192, d=128,
                                     layout="BSND", causal=True, block_size=16),
+    # one decoding step of the LLaMA-13B shape: the new token's query rows
+    # against an 8192-key cache, batch 1 (online inference), split-KV
+    "llama13b-decode-8k": _wl("llama13b-decode-8k", 6, B=1, H=40, Nq=1, Nkv=8192, d=128, layout="BSND",
+                              num_splits=0),
+    "llama13b-decode-8k-paged16": _wl("llama13b-decode-8k-paged16", 6, B=1, H=40, Nq=1, Nkv=8192, d=128,
+                                      layout="BSND", block_size=16, num_splits=0),
 }
 
 

@@ -22,7 +22,7 @@ Sources (the three surveyed web pages):
   key j is visible to query i iff j <= i; scale = d ** -0.5 by default
   (section 3.1 Config: softmax_scale = -1 means 1/sqrt(d)).
 
-Readings where the pages are silent or garbled (each listed in the design doc):
+Readings where the pages are silent or garbled:
 
 * The page-1 tiling listing divides the block's P by its own sum l_ij inside
   the loop and again by l_prev at the end; the page-2 update divides new_out by

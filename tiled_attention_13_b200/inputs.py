@@ -3,7 +3,7 @@
 This module holds no attention arithmetic: it only draws Q, K and V.  It is the
 one module that both the CUDA-side tests and the CPU oracle checks read.
 
-Recipe (stated in DESIGN.md as well):
+Recipe:
 
 * Q, K, V are i.i.d. N(0, 1) drawn in float32 by ``torch.randn`` from three
   independent generators seeded ``4*seed + 0/1/2`` (Q, K, V), then rounded to
@@ -19,10 +19,12 @@ Recipe (stated in DESIGN.md as well):
   Nkv in each sequence's last block) is NaN, so that any read of them shows.
 * The named workloads are the shapes the surveyed pages benchmark (LLaMA-13B
   self-attention, B=4/H=32/D=128 batched attention, a diffusion cross-attention
-  block, 128K long context), plus a grouped-query variant of the LLaMA-13B
-  shape (8 K/V heads for its 40 query heads).  No dataset, weights or
-  benchmark items are used: every tensor is random and only the shapes follow
-  the pages.
+  block, 128K long context), plus variants of the LLaMA-13B shape that the
+  pages name without sizes: grouped-query (8 K/V heads for its 40 query
+  heads), the same through a paged cache, a 2048-key sliding window (band
+  mask), and one decoding step (one query row per head against an 8192-key
+  cache).  No dataset, weights or benchmark items are used: every tensor is
+  random and only the shapes follow the pages.
 """
 
 from __future__ import annotations

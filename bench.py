@@ -76,6 +76,13 @@ def captured_traffic(workload: str):
     return float(rec["dram_bytes_per_launch"])
 
 
+def roofline_bound(wl, peaks) -> str:
+    """"tensor" when the workload's arithmetic intensity (algorithmic FLOPs
+    per compulsory byte) reaches the measured ridge point, else "hbm"."""
+    ridge = float(peaks["bf16_tflops"]) * 1e12 / (float(peaks["hbm_gbs"]) * 1e9)
+    return "tensor" if wl.flops / wl.bytes_min >= ridge else "hbm"
+
+
 def dist_env():
     ws = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -402,10 +409,7 @@ def run_ours(args, wl):
         kmean = sum(kern_ms) / len(kern_ms)
         traffic = args.traffic if args.traffic is not None else captured_traffic(wl.name)
         achieved = wl.flops / (kmean * 1e-3) / 1e12
-        # the bound: tensor when the work's arithmetic intensity (algorithmic
-        # FLOPs per compulsory byte) is above the measured ridge point
-        ridge = float(peaks["bf16_tflops"]) * 1e12 / (float(peaks["hbm_gbs"]) * 1e9)
-        bound = "tensor" if wl.flops / wl.bytes_min >= ridge else "hbm"
+        bound = roofline_bound(wl, peaks)
         if bound == "tensor":
             peak = float(peaks["bf16_tflops"])
             roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",

@@ -52,3 +52,14 @@ def test_traffic_record_rejected_when_source_changes(tmp_path, monkeypatch):
     (root / "profiles" / "fa_fwd_tc_llama13b_8k.json").write_text(json.dumps(rec))
     monkeypatch.setattr(bench, "ROOT", str(root))
     assert bench.captured_traffic("llama13b-8k") is None
+
+
+def test_roofline_bound_follows_arithmetic_intensity():
+    """Self-attention is tensor-bound at every configured length (intensity
+    about N/2 FLOP per byte against a ridge near 257); the 77-key
+    cross-attention (74 FLOP/B) and a decoding step (1 FLOP/B) are HBM-bound."""
+    peaks = {"bf16_tflops": 1686.0, "hbm_gbs": 6549.1}
+    for name, wl in WORKLOADS.items():
+        want = "hbm" if name in ("cross", "llama13b-decode-8k", "llama13b-decode-8k-paged16") or wl.dtype == "fp32" \
+            else "tensor"
+        assert bench.roofline_bound(wl, peaks) == want, name

@@ -47,6 +47,28 @@ def test_small_bf16(shape, d, causal, layout):
     compare_full(wl)
 
 
+def _random_tiny_cases(n=24, seed=20261202):
+    """Seeded random tiny problems: Nq, Nkv in [1, 300] (every tail length of
+    a 128-row tile is reachable), B in {1, 2}, H in {1, 2, 3}, with head dim,
+    layout and mask cycling so that every combination appears."""
+    import random
+
+    rng = random.Random(seed)
+    cases = []
+    for i in range(n):
+        cases.append((rng.randint(1, 2), rng.randint(1, 3), rng.randint(1, 300), rng.randint(1, 300),
+                      (64, 128)[i % 2], ("BHND", "BSND")[(i // 2) % 2], bool((i // 4) % 2)))
+    return cases
+
+
+@pytest.mark.parametrize("case", _random_tiny_cases(), ids=lambda c: "x".join(map(str, c[:5])) + c[5] + "c" * c[6])
+def test_random_tiny_shapes(case):
+    """Randomized tiny shapes against the oracle, every element."""
+    B, H, nq, nkv, d, layout, causal = case
+    compare_full(Workload("rand", B=B, H=H, Nq=nq, Nkv=nkv, d=d, dtype="bf16", layout=layout, causal=causal,
+                          seed=nq * 301 + nkv))
+
+
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("d", [64, 128])
 @pytest.mark.parametrize("shape", [(2, 3, 300, 333), (1, 2, 513, 1000)], ids=lambda s: "x".join(map(str, s)))

@@ -50,7 +50,9 @@ typedef enum {
   FA_ERR_LAUNCH = 4,       /* the CUDA launch or tensor-map creation failed */
   FA_ERR_TIMEOUT = 5,      /* a bounded device-side wait expired (see fa_get_device_status) */
   FA_ERR_NO_DEVICE = 6,    /* no usable sm_100 device for the current context */
-  FA_ERR_TOO_LARGE = 7     /* fa_fwd_noalloc only: the call needs more than its fixed scratch */
+  FA_ERR_TOO_LARGE = 7,    /* fa_fwd_noalloc only: the call needs more than its fixed scratch */
+  FA_ERR_CHECK = 8         /* debug builds (FA_CHECKS) only: a kernel found a computed index out of
+                              bounds and skipped that access (see fa_get_device_status) */
 } fa_status_t;
 
 /*
@@ -265,10 +267,11 @@ const char* fa_status_string(int status);
 
 /*
  * fa_get_device_status -- synchronise `stream`, then read and clear the
- * current device's status word.  Returns FA_OK, FA_ERR_TIMEOUT if any kernel
- * since the last read gave up on a bounded wait (its outputs are then
- * undefined; the CUDA context stays usable), or FA_ERR_LAUNCH if the stream
- * itself reported an error.
+ * current device's status word.  Returns FA_OK, FA_ERR_CHECK if a kernel of
+ * a debug build (FA_CHECKS) found a computed index out of bounds since the
+ * last read (it skipped that access), FA_ERR_TIMEOUT if any kernel gave up on
+ * a bounded wait (its outputs are then undefined; the CUDA context stays
+ * usable), or FA_ERR_LAUNCH if the stream itself reported an error.
  */
 int fa_get_device_status(void* stream);
 
@@ -293,7 +296,7 @@ uint32_t fa_set_wait_timeout_us(uint32_t us);
 int fa_debug_set_fault(int mode);
 
 /* ABI version of this header, (major << 16) | minor (1.1: fa_fwd_gqa, 1.2: fa_fwd_paged, 1.3: fa_fwd_band,
- * 1.4: fa_splitkv_plan, fa_fwd_splitkv, fa_fwd_paged_splitkv). */
+ * 1.4: fa_splitkv_plan, fa_fwd_splitkv, fa_fwd_paged_splitkv, 1.5: FA_ERR_CHECK). */
 int fa_abi_version(void);
 
 #ifdef __cplusplus

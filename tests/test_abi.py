@@ -31,10 +31,10 @@ def test_library_exports_every_declared_symbol(fa_lib):
 
 
 def test_status_strings_and_version(fa_lib):
-    for code in range(8):
+    for code in range(9):
         assert fa.fa_status_string(code).startswith("FA_")
     assert fa.fa_status_string(99) == "FA_ERR_UNKNOWN"
-    assert fa.fa_abi_version() == (1 << 16) | 4
+    assert fa.fa_abi_version() == (1 << 16) | 5
 
 
 def test_host_settings_roundtrip(fa_lib):

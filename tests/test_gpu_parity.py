@@ -188,6 +188,40 @@ def test_polynomial_exp_option(tmp_path):
     assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout[-2000:] + r.stderr[-2000:]
 
 
+def test_index_checks_build(tmp_path):
+    """The debug build (FA_CHECKS: every computed global index checked on the
+    device, a violation reported as FA_ERR_CHECK) runs the contiguous, fp32,
+    paged, paged split-KV, band and split-KV paths on ragged shapes with a
+    clean status and the usual parity, in a process of its own."""
+    import os
+    import subprocess
+    import sys
+
+    from tiled_attention_13_b200.build import build_variant
+
+    lib = build_variant(str(tmp_path / "libfa_checks.so"), {"FA_CHECKS": 1})
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    code = ("import tiled_attention_13_b200 as fa\n"
+            "from tests.parity import compare_full\n"
+            "from tests import test_gpu_parity as t\n"
+            "from tiled_attention_13_b200.inputs import Workload\n"
+            "for c in (False, True):\n"
+            "    compare_full(Workload('chk', B=2, H=3, Nq=300, Nkv=333, d=128, dtype='bf16', layout='BSND',"
+            " causal=c, seed=7))\n"
+            "compare_full(Workload('chk32', B=1, H=2, Nq=70, Nkv=90, d=64, dtype='fp32', layout='BHND', seed=8))\n"
+            "pw = Workload('chkp', B=2, H=8, Hkv=2, Nq=7, Nkv=4097, d=128, dtype='bf16', layout='BSND', seed=3,"
+            " block_size=16)\n"
+            "t._paged_parity(pw)\n"
+            "t._paged_parity(pw, num_splits=3)\n"
+            "t.test_band_bf16(t.BAND_CASES[1])\n"
+            "t.test_splitkv(t.SPLIT_CASES[1])\n"
+            "assert fa.fa_get_device_status(None) == 0\n"
+            "print('ok')\n")
+    r = subprocess.run([sys.executable, "-c", code], cwd=root, env={**os.environ, "FA_B200_LIB": lib},
+                       capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0 and r.stdout.strip().endswith("ok"), r.stdout[-2000:] + r.stderr[-2000:]
+
+
 # ----------------------------------------------------------------- grouped-query attention
 GQA_SHAPES = [  # (B, H, Hkv, Nq, Nkv)
     (1, 8, 1, 300, 333),

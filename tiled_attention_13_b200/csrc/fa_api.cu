@@ -589,6 +589,7 @@ const char* fa_status_string(int status) {
     case FA_ERR_TIMEOUT: return "FA_ERR_TIMEOUT: a bounded device wait expired";
     case FA_ERR_NO_DEVICE: return "FA_ERR_NO_DEVICE: no usable sm_100 device";
     case FA_ERR_TOO_LARGE: return "FA_ERR_TOO_LARGE: the problem needs more than fa_fwd_noalloc's fixed scratch";
+    case FA_ERR_CHECK: return "FA_ERR_CHECK: a debug build found a computed index out of bounds";
     default: return "FA_ERR_UNKNOWN";
   }
 }
@@ -598,6 +599,7 @@ int fa_get_device_status(void* stream) {
   unsigned int w = 0, zero = 0;
   if (cudaMemcpyFromSymbol(&w, fa::g_status_word, sizeof(w)) != cudaSuccess) return FA_ERR_LAUNCH;
   if (w != 0 && cudaMemcpyToSymbol(fa::g_status_word, &zero, sizeof(zero)) != cudaSuccess) return FA_ERR_LAUNCH;
+  if (w & 2u) return FA_ERR_CHECK;  // bit 1: a debug build's index check failed
   return (w & 1u) ? FA_ERR_TIMEOUT : FA_OK;
 }
 
@@ -607,7 +609,7 @@ uint32_t fa_set_wait_timeout_us(uint32_t us) {
 
 int fa_debug_set_fault(int mode) { return g_fault_mode.exchange(mode); }
 
-int fa_abi_version(void) { return (1 << 16) | 4; }
+int fa_abi_version(void) { return (1 << 16) | 5; }
 
 #ifdef FA_TRACE_UNITS
 int fa_debug_trace_units_read(unsigned long long* host, int n) {

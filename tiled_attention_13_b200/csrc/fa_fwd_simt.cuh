@@ -13,6 +13,8 @@
 // output columns l, l+32, ... and receives p_key by shuffle.
 #pragma once
 
+#include "ptx.cuh"  // FA_INDEX_OK
+
 namespace fa {
 
 constexpr int SIMT_ROWS = 32;   // query rows per CTA
@@ -63,7 +65,9 @@ __global__ void __launch_bounds__(SIMT_THREADS) fa_fwd_simt_kernel(SimtParams p)
   for (int idx = threadIdx.x; idx < SIMT_ROWS * D; idx += SIMT_THREADS) {
     const int r = idx / D, c = idx % D;
     const int n = row0 + r;
-    Qs[r][c] = (n < p.Nq) ? p.q[simt_row(p, b, h, n, p.Nq) * D + c] : 0.f;
+    const long long qi = simt_row(p, b, h, n, p.Nq) * D + c;
+    Qs[r][c] = (n < p.Nq && FA_INDEX_OK(&g_status_word, qi >= 0 && qi < (long long)p.B * p.H * p.Nq * D)) ? p.q[qi]
+                                                                                                        : 0.f;
   }
 
   float m[8], l[8], acc[8][CPL];
@@ -86,8 +90,8 @@ __global__ void __launch_bounds__(SIMT_THREADS) fa_fwd_simt_kernel(SimtParams p)
     for (int idx = threadIdx.x; idx < SIMT_KEYS * D; idx += SIMT_THREADS) {
       const int r = idx / D, c = idx % D;
       const int n = kb + r;
-      const bool in = n < p.Nkv;
-      const long long off = in ? simt_kv_row(p, b, hk, n) * D + c : 0;
+      const long long off = n < p.Nkv ? simt_kv_row(p, b, hk, n) * D + c : 0;
+      const bool in = n < p.Nkv && FA_INDEX_OK(&g_status_word, off >= 0 && off < (long long)p.B * p.Hkv * p.Nkv * D);
       Ks[r][c] = in ? p.k[off] : 0.f;
       Vs[r][c] = in ? p.v[off] : 0.f;
     }
@@ -130,7 +134,9 @@ __global__ void __launch_bounds__(SIMT_THREADS) fa_fwd_simt_kernel(SimtParams p)
     const int grow = row0 + warp * 8 + rr;
     if (grow >= p.Nq) continue;
     const float inv = 1.f / l[rr];
-    float* orow = p.o + simt_row(p, b, h, grow, p.Nq) * D;
+    const long long oi = simt_row(p, b, h, grow, p.Nq) * D;
+    if (!FA_INDEX_OK(&g_status_word, oi >= 0 && oi + D <= (long long)p.B * p.H * p.Nq * D)) continue;
+    float* orow = p.o + oi;
 #pragma unroll
     for (int t = 0; t < CPL; ++t) orow[lane + 32 * t] = acc[rr][t] * inv;
     if (p.lse != nullptr && lane == 0)

@@ -417,7 +417,9 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 #pragma unroll
         for (int u = 0; u < PSUB; ++u) {
           const int lb = (kv0 + u * pbox) / p.block_size;
-          phys[u] = (u * pbox < TC_BN && lb < pvalid) ? p.block_table[(long long)b * p.max_blocks + lb]
+          phys[u] = (u * pbox < TC_BN && lb < pvalid &&
+                     FA_INDEX_OK(status_word, lb < p.max_blocks && b < p.B))
+                        ? p.block_table[(long long)b * p.max_blocks + lb]
                                                       : p.num_blocks;
         }
       };
@@ -945,18 +947,20 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         // depend on the row.
         const long long prow = (((long long)sp * p.B + w.b) * p.H + w.h) * p.Nq + row;
         float* op = static_cast<float*>(p.o) + prow * D + (D / 2) * half;
+        const bool pvalid_row =
+            valid && FA_INDEX_OK(status_word, prow >= 0 && prow < (long long)p.split.n_splits * p.B * p.H * p.Nq);
 #pragma unroll 1
         for (int c = 0; c < D / 2; c += 32) {
           float ov[32];
           tmem_ld32(tO + c, ov);
-          if (valid) {
+          if (pvalid_row) {
 #pragma unroll
             for (int t = 0; t < 8; ++t)
               *reinterpret_cast<float4*>(op + c + 4 * t) =
                   make_float4(ov[4 * t] * inv_l, ov[4 * t + 1] * inv_l, ov[4 * t + 2] * inv_l, ov[4 * t + 3] * inv_l);
           }
         }
-        if (valid && half == 0) p.lse[prow] = (m_ref + __log2f(l)) * 0.69314718055994530942f;
+        if (pvalid_row && half == 0) p.lse[prow] = (m_ref + __log2f(l)) * 0.69314718055994530942f;
         ++n_units_s;
         continue;
       }
@@ -1001,14 +1005,19 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
         T* obase = reinterpret_cast<T*>(p.o) +
                    (p.bsnd ? ((long long)w.b * p.Nq * p.H + w.h) * D : ((long long)w.b * p.H + w.h) * p.Nq * D) +
                    (D / 2) * half + 8 * ci;
+#ifdef FA_CHECKS
+        const long long o_total = (long long)p.B * p.H * p.Nq * D;
+        const long long o_off = obase - reinterpret_cast<T*>(p.o);
+#endif
 #pragma unroll
         for (int k = 0; k < NC; ++k) {
           const int rk = rbase + k;
-          if (rk < p.Nq)
+          if (rk < p.Nq && FA_INDEX_OK(status_word, o_off + rk * rstride >= 0 && o_off + rk * rstride + 8 <= o_total))
             *reinterpret_cast<uint4*>(obase + rk * rstride) = make_uint4(pk[4 * k], pk[4 * k + 1], pk[4 * k + 2], pk[4 * k + 3]);
         }
       }
-      if (valid && half == 0 && p.lse != nullptr) {
+      if (valid && half == 0 && p.lse != nullptr &&
+          FA_INDEX_OK(status_word, ((long long)w.b * p.H + w.h) * p.Nq + row < (long long)p.B * p.H * p.Nq)) {
         p.lse[((long long)w.b * p.H + w.h) * p.Nq + row] = (m_ref + __log2f(l)) * 0.69314718055994530942f;
       }
       FA_TRU(warp == 0 && lane == 0, 2, n_units_s, 4);

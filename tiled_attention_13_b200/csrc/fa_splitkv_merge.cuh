@@ -19,6 +19,8 @@
 
 #include <cstdint>
 
+#include "ptx.cuh"  // FA_INDEX_OK
+
 namespace fa {
 
 constexpr int MERGE_ROWS_PER_CTA = 8;  // one warp per query row
@@ -60,6 +62,7 @@ __global__ void __launch_bounds__(MERGE_THREADS)
   const long long rows = (long long)B * H * Nq;
   const long long r = (long long)blockIdx.x * MERGE_ROWS_PER_CTA + (threadIdx.x >> 5);
   if (r >= rows) return;
+  if (!FA_INDEX_OK(&g_status_word, r >= 0 && n_splits >= 1)) return;
   const int lane = threadIdx.x & 31;
   float m = -INFINITY;
   for (int s = 0; s < n_splits; ++s) m = fmaxf(m, lse_part[(long long)s * rows + r]);

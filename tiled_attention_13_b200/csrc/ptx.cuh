@@ -10,6 +10,16 @@
 
 namespace fa {
 
+// Debug builds (-DFA_CHECKS): every computed global index is checked before
+// its access; a violation sets bit 1 of the device status word (read by
+// fa_get_device_status as FA_ERR_CHECK) and the access is skipped.  No trap,
+// no assert.  Default builds compile each check to `true`.
+#ifdef FA_CHECKS
+#define FA_INDEX_OK(status_ptr, cond) ((cond) ? true : (atomicOr((status_ptr), 2u), false))
+#else
+#define FA_INDEX_OK(status_ptr, cond) true
+#endif
+
 // ---------------------------------------------------------------- addresses
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));

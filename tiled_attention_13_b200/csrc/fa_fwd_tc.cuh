@@ -177,7 +177,9 @@ struct TcParams {
   int fault_mode;
 };
 
-// Per-unit geometry shared by every role (pure integer arithmetic).
+// Per-unit geometry shared by every role (pure integer arithmetic; the
+// decode functions below also compile for the host, where a test checks the
+// schedule's coverage).
 struct Unit {
   int b, h, qt0;      // qt0 = first Q tile index (even), second = qt0 + 1
   int active1;        // second Q tile has at least one valid row
@@ -185,7 +187,7 @@ struct Unit {
   int lo0, s1;        // band / split: first KV tile of tile 0; tile 1 starts s1 tiles later (else 0, 0)
 };
 
-__device__ __forceinline__ int kv_tiles_for(int qt, int Nkv, int causal) {
+__host__ __device__ __forceinline__ int kv_tiles_for(int qt, int Nkv, int causal) {
   int lim = Nkv;
   if (causal) {
     long long e = (long long)(qt + 1) * TC_BM;
@@ -198,7 +200,7 @@ __device__ __forceinline__ int kv_tiles_for(int qt, int Nkv, int causal) {
 // chunk_heads, so the K/V of the heads in flight stay in L2; inside a chunk
 // the heaviest causal Q-tile pairs come first (longest-processing-time order)
 // and the heads of one pair are adjacent.
-__device__ __forceinline__ Unit decode_unit(int t, const TcParams& p) {
+__host__ __device__ __forceinline__ Unit decode_unit(int t, const TcParams& p) {
   Unit w;
   const int BH = p.B * p.H;
   const int per_chunk = p.chunk_heads * p.n_pairs;  // <= n_units < 2^31
@@ -219,11 +221,11 @@ __device__ __forceinline__ Unit decode_unit(int t, const TcParams& p) {
 
 // KV tile range [lo, hi) of Q tile qt under a band: the keys its rows can see,
 // [qt*128 - pre, qt*128 + 127 + next], cut to [0, Nkv).
-__device__ __forceinline__ int band_lo(int qt, const TcParams& p) {
+__host__ __device__ __forceinline__ int band_lo(int qt, const TcParams& p) {
   const long long k = (long long)qt * TC_BM - p.band.pre_tokens;
   return k <= 0 ? 0 : (int)(k / TC_BN);
 }
-__device__ __forceinline__ int band_hi(int qt, const TcParams& p) {
+__host__ __device__ __forceinline__ int band_hi(int qt, const TcParams& p) {
   long long k = (long long)qt * TC_BM + TC_BM + p.band.next_tokens;  // one past the last visible key
   if (k > p.Nkv) k = p.Nkv;
   return (int)((k + TC_BN - 1) / TC_BN);
@@ -233,7 +235,7 @@ __device__ __forceinline__ int band_hi(int qt, const TcParams& p) {
 // chunks are walked as in decode_unit; a head's units are its (Q-tile pair,
 // slice) pairs, the slice index fastest.  Both Q tiles of a pair take the
 // same slice of KV tiles (no mask but the sequence end).
-__device__ __forceinline__ Unit decode_unit_split(int t, const TcParams& p, int& sp) {
+__host__ __device__ __forceinline__ Unit decode_unit_split(int t, const TcParams& p, int& sp) {
   Unit w;
   const int BH = p.B * p.H;
   const int per_chunk = p.chunk_heads * p.n_pairs * p.split.n_splits;  // <= n_units < 2^31
@@ -259,7 +261,7 @@ __device__ __forceinline__ Unit decode_unit_split(int t, const TcParams& p, int&
 }
 
 template <bool BAND, bool SPLIT>
-__device__ __forceinline__ Unit decode_unit_t(int t, const TcParams& p, int& sp) {
+__host__ __device__ __forceinline__ Unit decode_unit_t(int t, const TcParams& p, int& sp) {
   if constexpr (SPLIT) return decode_unit_split(t, p, sp);
   Unit w = decode_unit(t, p);
   w.lo0 = 0;

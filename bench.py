@@ -36,6 +36,7 @@ sys.path.insert(0, ROOT)
 METRIC = "attention fwd TFLOP/s (and % of B200 dense BF16 peak) and ms/call at 1 GPU"
 UNIT = "TFLOP/s"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+DATASHEET_BF16_TFLOPS = 2250.0  # B200 dense BF16 (the vendor's figure without sparsity), context only
 
 
 def load_peaks():
@@ -74,6 +75,13 @@ def captured_traffic(workload: str):
     if rec.get("kernel_source_sha256") != sha or rec.get("workload") != workload:
         return None
     return float(rec["dram_bytes_per_launch"])
+
+
+def step_percentiles(ms):
+    """p10 / median / p90 of per-step durations (nearest rank)."""
+    xs = sorted(ms)
+    pick = lambda q: xs[min(len(xs) - 1, max(0, int(round(q * (len(xs) - 1)))))]
+    return {"p10": pick(0.1), "median": pick(0.5), "p90": pick(0.9)}
 
 
 def roofline_bound(wl, peaks) -> str:
@@ -440,6 +448,8 @@ def run_ours(args, wl):
             "gpu_launches": args.steps * launches_per_step, "clocks": clocks, "timing": "cuda-graph replay of the K steps" if use_graph
             else "eager launches",
             "pct_of_measured_bf16_peak": 100.0 * (value / ws) / float(peaks["bf16_tflops"]),
+            "pct_of_datasheet_bf16_peak": 100.0 * (value / ws) / DATASHEET_BF16_TFLOPS,
+            "kernel_ms_percentiles": step_percentiles(kern_ms),
         }
         if s_used is not None:
             line["config"]["splits_used"] = s_used

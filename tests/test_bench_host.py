@@ -63,3 +63,10 @@ def test_roofline_bound_follows_arithmetic_intensity():
         want = "hbm" if name in ("cross", "llama13b-decode-8k", "llama13b-decode-8k-paged16") or wl.dtype == "fp32" \
             else "tensor"
         assert bench.roofline_bound(wl, peaks) == want, name
+
+
+def test_step_percentiles():
+    """Nearest-rank p10 / median / p90 of the per-step kernel times."""
+    ms = [float(x) for x in range(1, 12)]  # 1 .. 11
+    assert bench.step_percentiles(ms) == {"p10": 2.0, "median": 6.0, "p90": 10.0}
+    assert bench.step_percentiles([3.5]) == {"p10": 3.5, "median": 3.5, "p90": 3.5}

@@ -238,11 +238,12 @@ int fa_fwd_paged_splitkv(const void* q, const void* k_cache, const void* v_cache
  * of the library, not of the method.)
  *
  * fa_fwd's tile scheduler keeps its per-launch work counters in 8 KB that it
- * allocates on its first call on a device.  This entry point keeps its single
- * counter in a fixed 256-byte static device array instead, which every GPU
- * that loads the library holds until the process exits; no call allocates
- * or frees anything.  The counter is cleared (cudaMemsetAsync on `stream`)
- * before each launch.
+ * allocates on its first call on a device.  This entry point keeps them in a
+ * fixed 256-byte static device array instead, which every GPU that loads the
+ * library holds until the process exits; no call allocates or frees
+ * anything.  Slot 0 of the array (8 bytes: the work-ticket counter and the
+ * finished-CTA counter) is cleared with cudaMemsetAsync on `stream` before
+ * each launch; the rest of the array is unused padding.
  *
  *   - The first call on a device looks up the array's device address
  *     (cudaGetSymbolAddress) and sets kernel attributes; make that first call
@@ -250,7 +251,7 @@ int fa_fwd_paged_splitkv(const void* q, const void* k_cache, const void* v_cache
  *   - Every call on a device shares the array and it keeps the last call's
  *     contents: calls that overlap on the GPU (other streams, other threads)
  *     race on the counter and may compute wrong results.  Serialise them.
- *   - Limit: the scratch holds one 32-bit work-ticket counter, so a bf16/fp16
+ *   - Limit: the work-ticket counter is 32-bit, so a bf16/fp16
  *     call may have at most 2^31 - 1025 work units (a unit is a pair of
  *     128-row query tiles of one batch and head); larger calls return
  *     FA_ERR_TOO_LARGE before anything is launched.  fp32 inputs use no

@@ -18,7 +18,6 @@ overlapping the computation (separate copy streams, two device buffer sets).
 from __future__ import annotations
 
 import ctypes
-import math
 import os
 
 __all__ = [
@@ -460,6 +459,3 @@ def forward_host(q_host, k_host, v_host, causal=False, scale=None, layout="BHND"
     torch.cuda.current_stream(hf.dev).synchronize()
     return o.clone(), lse.clone()
 
-
-def default_scale(d: int) -> float:
-    return 1.0 / math.sqrt(d)

@@ -646,9 +646,11 @@ namespace fa {
 constexpr int kNoAllocScratchBytes = 256;
 constexpr int kNoAllocScratchSlots = kNoAllocScratchBytes / (int)sizeof(SchedSlot);
 // One copy per device that loads the library, held until the process exits.
-// Every call of fa_fwd_noalloc on a device uses slot 0; see the header for why
-// overlapping calls race.
+// Every call of fa_fwd_noalloc on a device uses slot 0 (its work-ticket
+// counter and its finished-CTA counter, 8 bytes); the rest of the 256 bytes
+// is unused padding.  See the header for why overlapping calls race.
 static __device__ __align__(256) SchedSlot g_noalloc_scratch[kNoAllocScratchSlots];
+static_assert(sizeof(SchedSlot) <= kNoAllocScratchBytes, "the fixed scratch must hold one scheduler slot");
 }  // namespace fa
 
 namespace {
@@ -760,10 +762,9 @@ extern "C" int fa_fwd_noalloc(const void* q, const void* k, const void* v, void*
   if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
       (lse != nullptr && !aligned(lse, 4)))
     return FA_ERR_MISALIGNED;
-  // The fixed scratch holds one 32-bit work-ticket counter: a call fits when
-  // the counter can number all its work units (pairs of 128-row query tiles
+  // Slot 0 of the fixed scratch holds the 32-bit work-ticket counter: a call
+  // fits when it can number all its work units (pairs of 128-row query tiles
   // over every batch and head) plus one closing ticket per CTA.
-  if ((int)sizeof(fa::SchedSlot) > fa::kNoAllocScratchBytes) return FA_ERR_TOO_LARGE;
   const int64_t units = B * H * (((Nq + fa::TC_BM - 1) / fa::TC_BM + 1) / 2);
   if (dtype != FA_DTYPE_FP32 && units > (int64_t)INT32_MAX - 1024) return FA_ERR_TOO_LARGE;
   if (!(scale > 0.f) || std::isinf(scale)) scale = 1.0f / std::sqrt((float)d);

@@ -8,7 +8,8 @@ text).  The kernel reduces x = n + f with n = round(x) (adding and subtracting
 1.5 * 2^23 rounds to the nearest integer in fp32), evaluates p(f) by Horner's
 rule and adds n to the exponent field.  The coefficients are rounded to fp32
 and the error is re-measured in fp32 arithmetic.  The printed constants are
-the ones in fa_fwd_tc.cuh; tests/test_exp2_poly.py re-runs this fit.
+the ones in ptx.cuh (exp2_poly_x2); tests/test_exp2_poly.py re-runs this fit
+and checks them and their error bound.
 """
 
 from __future__ import annotations

@@ -61,20 +61,23 @@ def max_over_ranks(x: float, device=None) -> float:
 
 def captured_traffic(workload: str):
     """DRAM bytes per launch from the committed ncu capture of this workload's
-    kernel (profiles/fa_fwd_tc_<workload>.json), or None when there is none or
-    the kernel source has changed since the counters were taken."""
+    kernel (a profiles/*.json record whose "workload" is this one), or None
+    when there is none or the kernel's source files (the record's
+    "source_files", by default fa_fwd_tc.cuh and ptx.cuh) have changed since
+    the counters were taken."""
+    import glob
     import hashlib
 
-    path = os.path.join(ROOT, "profiles", f"fa_fwd_tc_{workload.replace('-', '_')}.json")
-    if not os.path.exists(path):
-        return None
-    rec = json.load(open(path))
     csrc = os.path.join(ROOT, "tiled_attention_13_b200", "csrc")
-    sha = hashlib.sha256(b"".join(open(os.path.join(csrc, f), "rb").read()
-                                  for f in ("fa_fwd_tc.cuh", "ptx.cuh"))).hexdigest()
-    if rec.get("kernel_source_sha256") != sha or rec.get("workload") != workload:
-        return None
-    return float(rec["dram_bytes_per_launch"])
+    for path in sorted(glob.glob(os.path.join(ROOT, "profiles", "*.json"))):
+        rec = json.load(open(path))
+        if rec.get("workload") != workload or "dram_bytes_per_launch" not in rec:
+            continue
+        files = rec.get("source_files", ["fa_fwd_tc.cuh", "ptx.cuh"])
+        sha = hashlib.sha256(b"".join(open(os.path.join(csrc, f), "rb").read() for f in files)).hexdigest()
+        if rec.get("kernel_source_sha256") == sha:
+            return float(rec["dram_bytes_per_launch"])
+    return None
 
 
 def step_percentiles(ms):
@@ -164,11 +167,38 @@ def oracle_sample(wl, rows_budget_s: float = 12.0, seed: int = 0):
     import torch
     from threadpoolctl import threadpool_info
 
-    from oracle import attention, attention_masked, band_mask
-    from tiled_attention_13_b200.inputs import make_qkv
+    from oracle import attention, attention_masked, band_mask, block_sparse_mask
+    from tiled_attention_13_b200.inputs import make_block_mask, make_qkv
 
     one = wl.with_(B=1, H=1, Hkv=0)
+    if wl.backward:  # the backward oracle on the first n positions of one head, repeated up to the budget
+        from oracle import attention_backward
+        from tiled_attention_13_b200.inputs import make_dout
+
+        n = min(wl.Nq, wl.Nkv, 2048)
+        small = one.with_(Nq=n, Nkv=n)
+        q, k, v = make_qkv(small, device="cpu")
+        do = make_dout(small, device="cpu")
+        sl = (lambda t: t[0, :, 0]) if wl.layout == "BSND" else (lambda t: t[0, 0])
+        q, k, v, do = (sl(t).to(torch.float64).numpy() for t in (q, k, v, do))
+        flops, reps = 0.0, 0
+        t0 = time.perf_counter()
+        while True:
+            attention_backward(q, k, v, do, causal=wl.causal)
+            flops += small.flops
+            reps += 1
+            if time.perf_counter() - t0 > rows_budget_s:
+                break
+        el = time.perf_counter() - t0
+        threads = max([p.get("num_threads", 1) for p in threadpool_info()] + [1])
+        return flops / el / 1e12, (f"{reps} x the backward of the first {n} positions of one head of {wl.name}, "
+                                   "float64 numpy oracle"), threads, el
     q, k, v = make_qkv(one, device="cpu")
+    bmask = None
+    if wl.block_density > 0:  # this head's block mask, expanded and cut to the causal range
+        bmask = block_sparse_mask(make_block_mask(wl)[0, 0].numpy(), 128, 128, wl.Nq, wl.Nkv)
+        if wl.causal:
+            bmask &= np.tril(np.ones((wl.Nq, wl.Nkv), dtype=bool))
     if wl.layout == "BSND":
         q, k, v = q[0, :, 0], k[0, :, 0], v[0, :, 0]
     else:
@@ -186,6 +216,15 @@ def oracle_sample(wl, rows_budget_s: float = 12.0, seed: int = 0):
     rng.shuffle(starts)
     for r0 in [r for _ in range(wl.B * wl.H) for r in starts]:
         r1 = min(wl.Nq, r0 + block)
+        if bmask is not None:
+            mk = bmask[r0:r1]
+            keep = mk.any(axis=1)
+            attention_masked(qn[r0:r1][keep], kn, vn, mk[keep])
+            flops += 4.0 * wl.d * float(mk.sum())
+            rows_done += r1 - r0
+            if time.perf_counter() - t0 > rows_budget_s:
+                break
+            continue
         if wl.band:
             mask = band_mask(wl.Nq, wl.Nkv, wl.band[0], wl.band[1])[r0:r1]
             attention_masked(qn[r0:r1], kn, vn, mask)
@@ -260,6 +299,8 @@ def _config(wl, ws):
             **({"kv_cache": f"paged, {wl.block_size}-key blocks in shuffled order"} if wl.block_size > 0 else {}),
             **({"band": {"pre_tokens": wl.band[0], "next_tokens": wl.band[1]}} if wl.band else {}),
             **({"num_splits": wl.num_splits} if wl.num_splits >= 0 else {}),
+            **({"block_sparse": f"128x128 blocks, density {wl.block_density} per head plus the diagonal"
+                + (", intersected with the causal mask" if wl.causal else "")} if wl.block_density > 0 else {}),
             "parallelism": f"independent replicas x{ws} (no collective)",
             "l2": (f"{n} input sets of {wl.bytes_min / 1e6:.1f} MB (Q, K, V, O, LSE) rotate between steps, "
                    f"{n * wl.bytes_min / 1e6:.0f} MB in all > 2x the 126 MB L2"),
@@ -295,21 +336,47 @@ def run_ours(args, wl):
 
             paged = make_paged_kv(wl.with_(seed=wl.seed + s), k, v)
         sets.append((q, k, v, o, lse, paged))
+    bmask = None
+    if wl.block_density > 0:
+        from tiled_attention_13_b200.inputs import make_block_mask
+
+        bmask = make_block_mask(wl, device=dev)
+    bwd = []  # backward: per input set the forward's O and LSE, dO, the gradients and the workspace
+    if wl.backward:
+        from tiled_attention_13_b200.inputs import make_dout
+
+        _, nbytes = fa.fa_bwd_workspace_size(wl.B, wl.H, wl.Nq, wl.d)
+        for s_i, (q, k, v, o, lse, _) in enumerate(sets):
+            fa.forward(q, k, v, causal=wl.causal, layout=wl.layout, out=o, lse=lse)
+            bwd.append((make_dout(wl.with_(seed=wl.seed + s_i), device=dev), torch.empty_like(q), torch.empty_like(k),
+                        torch.empty_like(v), torch.empty(nbytes, dtype=torch.uint8, device=dev)))
     torch.cuda.synchronize()
 
     splits = wl.num_splits if wl.num_splits >= 0 else None
     # kernels per step: the split kernel and the merge when the plan has
     # more than one slice, else the one attention kernel
     launches_per_step, s_used = 1, None
+    if wl.backward:
+        launches_per_step = 3  # row statistics, the gradient kernel, dQ conversion (plus one memset)
     if splits is not None:
         s_used, _ = fa.splitkv_plan(wl.B, wl.H, wl.Nq, wl.Nkv, wl.d, splits)
         launches_per_step = 2 if s_used > 1 else 1
 
     def step(i):
         q, k, v, o, lse, paged = sets[i % n_sets]
+        if wl.backward:
+            do, dq, dk, dv, ws = bwd[i % n_sets]
+            rc = fa.fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(),
+                           dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), ws.numel(), wl.B, wl.H,
+                           wl.kv_heads, wl.Nq, wl.Nkv, wl.d, -1.0, int(wl.causal),
+                           fa.FA_LAYOUT_BHND if wl.layout == "BHND" else fa.FA_LAYOUT_BSND, fa.FA_DTYPE_BF16,
+                           torch.cuda.current_stream().cuda_stream)
+            if rc != 0:
+                raise RuntimeError(f"fa_bwd: {fa.fa_status_string(rc)}")
+            return
         if paged is None:
             fa.forward(q, k, v, causal=wl.causal, layout=wl.layout, out=o, lse=lse, band=wl.band or None,
-                       num_splits=splits)
+                       num_splits=splits, block_mask=bmask)
         else:
             kc, vc, table = paged
             fa.forward_paged(q, kc, vc, table, wl.Nkv, causal=wl.causal, layout=wl.layout, out=o, lse=lse,
@@ -376,14 +443,45 @@ def run_ours(args, wl):
     if rc != 0:
         raise RuntimeError(f"device status after timing: {fa.fa_status_string(rc)}")
 
+    # ---- steady state: the same K steps replayed back to back for about
+    # --sustain-s seconds after the timed region, once the 1 kW power cap has
+    # had time to act; reported beside (not in place of) the burst figure
+    sustained = None
+    if args.sustain_s > 0 and use_graph:
+        reps = max(1, int(args.sustain_s * 1e3 / max(total_ms, 1e-3)))
+        ssamp = ClockSampler(sampler.gpu)
+        if rank == 0:
+            ssamp.start()
+            time.sleep(0.3)
+        a_ev, b_ev = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if ws > 1:
+            dist.barrier()
+        ts0 = time.time()
+        a_ev.record(stream)
+        for _ in range(reps):
+            graph.replay()
+        b_ev.record(stream)
+        torch.cuda.synchronize()
+        ts1 = time.time()
+        if rank == 0:
+            time.sleep(0.1)
+            ssamp.stop()
+        rc = fa.fa_get_device_status(stream.cuda_stream)
+        if rc != 0:
+            raise RuntimeError(f"device status after the steady-state run: {fa.fa_status_string(rc)}")
+        ms_s = max_over_ranks(a_ev.elapsed_time(b_ev), dev) / (reps * args.steps)
+        sustained = {"seconds": reps * args.steps * ms_s / 1e3, "steps": reps * args.steps, "ms_per_step": ms_s,
+                     "value": ws * wl.flops / (ms_s * 1e-3) / 1e12, "unit": UNIT,
+                     "clocks": ssamp.summary(ts0, ts1) if rank == 0 else None}
+
     ms_step = max_over_ranks(total_ms, dev) / args.steps
     value = ws * wl.flops / (ms_step * 1e-3) / 1e12
 
     # ---- end-to-end through the public API: pinned host in, host out
     e2e = None
-    if not args.no_e2e and (wl.block_size > 0 or wl.band or splits is not None):
-        e2e = {"value": None, "unit": UNIT, "skipped": "HostPipeline takes contiguous K/V without a band or "
-               "split-KV; this path is measured on the device only"}
+    if not args.no_e2e and (wl.block_size > 0 or wl.band or splits is not None or bmask is not None or wl.backward):
+        e2e = {"value": None, "unit": UNIT, "skipped": "HostPipeline runs the plain forward (contiguous K/V, no band, "
+               "block mask or split-KV); this path is measured on the device only"}
     elif not args.no_e2e:
         # Every step copies its inputs from pinned host memory and reads its
         # O and LSE back; HostPipeline overlaps step i+1's upload and step
@@ -430,7 +528,19 @@ def run_ours(args, wl):
             roof = {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s", "frac": gbs / peak,
                     "traffic": traffic, "peak_source": f"{src} hbm_gbs", "kernel_ms_mean": kmean,
                     "kernel_ms_min": min(kern_ms), "algorithmic_bytes": wl.bytes_min}
-        if launches_per_step > 1:
+        if sustained is not None:
+            if bound == "tensor":
+                sp = float(peaks.get("bf16_tflops_sustained", peaks["bf16_tflops"]))
+                sustained.update({"peak": sp, "peak_source": f"{src} bf16_tflops_sustained",
+                                  "frac": (sustained["value"] / ws) / sp})
+            else:
+                gbs = wl.bytes_min / (sustained["ms_per_step"] * 1e-3) / 1e9
+                sustained.update({"achieved_gbs": gbs, "peak": float(peaks["hbm_gbs"]),
+                                  "peak_source": f"{src} hbm_gbs", "frac": gbs / float(peaks["hbm_gbs"])})
+        if launches_per_step > 1 and wl.backward:
+            roof["timed"] = ("each step's event pair spans the accumulator clear and the three backward kernels; "
+                             "achieved counts the backward's algorithmic FLOPs (2.5x the forward's)")
+        elif launches_per_step > 1:
             roof["timed"] = ("each step's event pair spans both kernels (split kernel and merge); achieved "
                              "counts the compulsory bytes only")
         cpu = None
@@ -450,6 +560,7 @@ def run_ours(args, wl):
             "pct_of_measured_bf16_peak": 100.0 * (value / ws) / float(peaks["bf16_tflops"]),
             "pct_of_datasheet_bf16_peak": 100.0 * (value / ws) / DATASHEET_BF16_TFLOPS,
             "kernel_ms_percentiles": step_percentiles(kern_ms),
+            "steady_state": sustained,
         }
         if s_used is not None:
             line["config"]["splits_used"] = s_used
@@ -474,6 +585,9 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget-s", type=float, default=12.0)
     ap.add_argument("--ref-step-s", type=float, default=2.0)
+    ap.add_argument("--sustain-s", type=float, default=1.0,
+                    help="after the timed region, replay the timed steps for about this many seconds and report "
+                         "the steady-state figure beside the burst one (0: skip)")
     ap.add_argument("--traffic", type=float, default=None,
                     help="DRAM bytes per launch from an ncu capture of the same kernel (else null)")
     args = ap.parse_args()

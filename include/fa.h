@@ -45,7 +45,7 @@ typedef enum { FA_DTYPE_BF16 = 0, FA_DTYPE_FP16 = 1, FA_DTYPE_FP32 = 2 } fa_dtyp
 typedef enum {
   FA_OK = 0,
   FA_ERR_INVALID_ARG = 1,  /* null pointer, negative size, bad enum, Nkv == 0 with Nq > 0 */
-  FA_ERR_UNSUPPORTED = 2,  /* head dim not in {64, 128}, or a size beyond the index range */
+  FA_ERR_UNSUPPORTED = 2,  /* head dim not supported by the entry point, or a size beyond the index range */
   FA_ERR_MISALIGNED = 3,   /* q, k, v, o not 16-byte aligned, or lse not 4-byte aligned */
   FA_ERR_LAUNCH = 4,       /* the CUDA launch or tensor-map creation failed */
   FA_ERR_TIMEOUT = 5,      /* a bounded device-side wait expired (see fa_get_device_status) */
@@ -63,7 +63,8 @@ typedef enum {
  *   o      same shape, layout and dtype as q, device memory, written
  *   lse    [B,H,Nq] fp32 device memory (head-major whatever the layout),
  *          written; may be NULL, in which case no LSE is written
- *   d      head dimension, 64 or 128
+ *   d      head dimension, 64, 128 or 256 (256: bf16/fp16 only; page 1,
+ *          section 分块 Tiling 的计算骨架, gives head dims of 64-256)
  *   scale  softmax scale; scale <= 0 or NaN selects 1/sqrt(d)
  *   causal 0 or 1.  Causal masking is top-left aligned: query row i sees key j
  *          iff j <= i (page 3, section 6.1: triu(ones(Nq, Nkv), diagonal=1)
@@ -108,6 +109,82 @@ int fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
 int fa_fwd_gqa(const void* q, const void* k, const void* v, void* o, float* lse,
                int64_t B, int64_t H, int64_t Hkv, int64_t Nq, int64_t Nkv, int64_t d,
                float scale, int causal, int layout, int dtype, void* stream);
+
+/*
+ * fa_bwd_workspace_size -- bytes of device workspace fa_bwd needs for B, H,
+ * Nq and d (0 when B * H * Nq == 0): an fp32 dQ accumulator of B*H*Nq*d
+ * values and two fp32 row arrays of B*H*ceil(Nq/128)*128 values, each part
+ * rounded up to 256 bytes.  Returns FA_OK, FA_ERR_INVALID_ARG (negative size,
+ * d not 64 or 128, NULL out pointer) or FA_ERR_UNSUPPORTED (sizes beyond the
+ * index range).  Needs no GPU.
+ */
+int fa_bwd_workspace_size(int64_t B, int64_t H, int64_t Nq, int64_t d, int64_t* workspace_bytes);
+
+/*
+ * fa_bwd -- the gradients dQ, dK, dV of fa_fwd_gqa's O with respect to q, k
+ * and v, given dO (page 1, "CANN ops-transformer FlashAttentionScore",
+ * section 反向传播的重算策略及其合理性: the backward keeps no N x N matrix; it
+ * recomputes each tile of P from Q, K and the forward's row statistics).  With
+ * S = scale Q K^T [+ causal mask] and P = exp(S - LSE):
+ *     dV = P^T dO,  dP = dO V^T,  dS = P o (dP - D),  D_i = sum_c dO_ic O_ic,
+ *     dQ = scale dS K,  dK = scale dS^T Q.
+ * Under grouped K/V heads a K/V head's gradient is the sum over the query
+ * heads that read it.
+ *
+ *   q, k, v, o, lse   the forward's inputs, output and LSE (fa_fwd_gqa with
+ *                     the same scale, causal flag, layout and dtype); lse
+ *                     must not be NULL
+ *   dout              dO, q's shape, layout and dtype
+ *   dq                written, q's shape, layout and dtype
+ *   dk, dv            written, k's shape, layout and dtype
+ *   workspace         caller-owned device memory of at least
+ *                     fa_bwd_workspace_size() bytes, 256-byte aligned; its
+ *                     contents on entry do not matter, and it is in use until
+ *                     the stream has finished the call
+ *   d                 64 or 128; dtype bf16 or fp16 (fp32 returns
+ *                     FA_ERR_UNSUPPORTED)
+ *
+ * Errors: as for fa_fwd_gqa, plus FA_ERR_INVALID_ARG for a missing or too
+ * small workspace and FA_ERR_MISALIGNED for a misaligned one, both before
+ * any launch.  The call clears the accumulator (cudaMemsetAsync) and
+ * launches three kernels on `stream`; Nq == 0 only clears dk and dv.  The
+ * first-call allocation is fa_fwd's.
+ */
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+           void* dq, void* dk, void* dv, void* workspace, int64_t workspace_bytes,
+           int64_t B, int64_t H, int64_t Hkv, int64_t Nq, int64_t Nkv, int64_t d,
+           float scale, int causal, int layout, int dtype, void* stream);
+
+/*
+ * fa_fwd_block_sparse -- fa_fwd_gqa with a block-sparse mask: query tile qt
+ * (rows [128 qt, 128 qt + 128)) of batch entry b and head h sees key tile kt
+ * (keys [128 kt, 128 kt + 128)) iff
+ *     block_mask[b * mask_batch_stride + h * mask_head_stride + qt * KT + kt] != 0,
+ * KT = ceil(Nkv / 128); with causal = 1 the causal mask applies as well.  Key
+ * tiles a query tile does not see are skipped (page 1, "CANN ops-transformer
+ * FlashAttentionScore", section 总结: SparseFlashAttention skips the key
+ * blocks a sparse mask marks as not needed).
+ *
+ *   block_mask         uint8 device memory, [.., .., ceil(Nq/128), KT] with the
+ *                      last two dimensions dense; read only
+ *   mask_batch_stride, mask_head_stride
+ *                      element strides of the batch and head dimensions of
+ *                      block_mask (>= 0; 0 shares one mask across that
+ *                      dimension)
+ *   d                  64, 128 or 256
+ *   dtype              bf16 or fp16 (fp32 returns FA_ERR_UNSUPPORTED)
+ *
+ * A query row with no visible key (all of its tile's mask entries zero, or
+ * zero within its causal range) gets O = 0 and LSE = -inf: softmax over an
+ * empty set is not defined, and these are the limits of an empty sum.  KT may
+ * be at most 4096 (Nkv <= 524288), else FA_ERR_UNSUPPORTED.  The mask must be
+ * readable for every (b, h, qt, kt) the strides address.  Other arguments,
+ * ownership, the first-call allocation and errors are as for fa_fwd_gqa.
+ */
+int fa_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, float* lse,
+                        const uint8_t* block_mask, int64_t mask_batch_stride, int64_t mask_head_stride,
+                        int64_t B, int64_t H, int64_t Hkv, int64_t Nq, int64_t Nkv, int64_t d,
+                        float scale, int causal, int layout, int dtype, void* stream);
 
 /*
  * fa_fwd_band -- fa_fwd_gqa with a band mask in place of the causal flag:
@@ -253,8 +330,9 @@ int fa_fwd_paged_splitkv(const void* q, const void* k_cache, const void* v_cache
  *     race on the counter and may compute wrong results.  Serialise them.
  *   - Limit: the work-ticket counter is 32-bit, so a bf16/fp16
  *     call may have at most 2^31 - 1025 work units (a unit is a pair of
- *     128-row query tiles of one batch and head); larger calls return
- *     FA_ERR_TOO_LARGE before anything is launched.  fp32 inputs use no
+ *     128-row query tiles of one batch and head, or one such tile at
+ *     d = 256); larger calls return FA_ERR_TOO_LARGE before anything is
+ *     launched.  fp32 inputs, and calls with at most 128 keys, use no
  *     scratch.
  *
  * Other arguments, ownership and errors are as for fa_fwd.
@@ -297,7 +375,8 @@ uint32_t fa_set_wait_timeout_us(uint32_t us);
 int fa_debug_set_fault(int mode);
 
 /* ABI version of this header, (major << 16) | minor (1.1: fa_fwd_gqa, 1.2: fa_fwd_paged, 1.3: fa_fwd_band,
- * 1.4: fa_splitkv_plan, fa_fwd_splitkv, fa_fwd_paged_splitkv, 1.5: FA_ERR_CHECK). */
+ * 1.4: fa_splitkv_plan, fa_fwd_splitkv, fa_fwd_paged_splitkv, 1.5: FA_ERR_CHECK, 1.6: d = 256 in fa_fwd,
+ * fa_fwd_gqa and fa_fwd_noalloc; fa_fwd_block_sparse, 1.7: fa_bwd_workspace_size, fa_bwd). */
 int fa_abi_version(void);
 
 #ifdef __cplusplus

@@ -7,6 +7,7 @@
 #include <utility>
 #include <vector>
 
+#include "fa_fwd_short.cuh"
 #include "fa_fwd_tc.cuh"
 
 using fa::TcParams;
@@ -135,7 +136,46 @@ static void check_split(int B, int H, int Nq, int Nkv, int S_req, int chunk) {
           covered[i]);
 }
 
+// The short-key kernel's static schedule: CTA c of G takes query tiles
+// [t0, t1); the ranges tile [0, n_tiles) exactly, none is empty and their
+// sizes differ by at most one; every tile decodes to a distinct (b, h, qt)
+// inside the problem with the K/V head h / (H / Hkv).
+static void check_short(int B, int H, int Hkv, int Nq, int G) {
+  fa::ShParams p{};
+  p.B = B; p.H = H; p.Nq = Nq;
+  p.qtiles = cdiv(Nq, 128);
+  p.n_tiles = B * H * p.qtiles;
+  p.kv_group = H / Hkv;
+  if (G > p.n_tiles) G = p.n_tiles;
+  std::vector<int> seen((size_t)p.n_tiles, 0);
+  int expect = 0, lo = 1 << 30, hi = 0;
+  for (int c = 0; c < G; ++c) {
+    int t0, t1;
+    fa::sh_range(c, G, p.n_tiles, t0, t1);
+    CHECK(t0 == expect && t1 > t0, "short B%d H%d Nq%d G%d: CTA %d range [%d, %d)", B, H, Nq, G, c, t0, t1);
+    expect = t1;
+    lo = t1 - t0 < lo ? t1 - t0 : lo;
+    hi = t1 - t0 > hi ? t1 - t0 : hi;
+    for (int t = t0; t < t1; ++t) {
+      const fa::ShTile x = fa::sh_decode(t, p);
+      CHECK(x.b >= 0 && x.b < B && x.h >= 0 && x.h < H && x.qt >= 0 && x.qt < p.qtiles,
+            "short: tile %d decodes outside the problem", t);
+      CHECK(x.kv == x.b * Hkv + x.h / (H / Hkv), "short: tile %d K/V key %d", t, x.kv);
+      if (x.b >= 0 && x.b < B && x.h >= 0 && x.h < H && x.qt >= 0 && x.qt < p.qtiles)
+        seen[((size_t)x.b * H + x.h) * p.qtiles + x.qt]++;
+    }
+  }
+  CHECK(expect == p.n_tiles && hi - lo <= 1, "short B%d H%d Nq%d G%d: ranges end at %d, sizes %d..%d", B, H, Nq, G,
+        expect, lo, hi);
+  for (size_t i = 0; i < seen.size(); ++i) CHECK(seen[i] == 1, "short: tile %zu scheduled %d times", i, seen[i]);
+}
+
 int main() {
+  const int short_shapes[][4] = {{1, 1, 1, 1}, {2, 8, 8, 4096}, {4, 32, 32, 4096}, {5, 200, 100, 100},
+                                 {1, 8, 2, 2000}, {3, 7, 7, 129}};
+  for (const auto& s : short_shapes)
+    for (int G : {1, 7, 148, 1 << 20}) check_short(s[0], s[1], s[2], s[3], G);
+
   const int shapes[][4] = {{1, 1, 1, 1}, {1, 2, 300, 333}, {2, 3, 129, 127}, {1, 40, 1024, 1024},
                            {2, 5, 777, 2000}, {3, 7, 4096, 77}, {1, 1, 8192, 8192}};
   for (const auto& s : shapes) {

@@ -34,7 +34,7 @@ def test_status_strings_and_version(fa_lib):
     for code in range(9):
         assert fa.fa_status_string(code).startswith("FA_")
     assert fa.fa_status_string(99) == "FA_ERR_UNKNOWN"
-    assert fa.fa_abi_version() == (1 << 16) | 5
+    assert fa.fa_abi_version() == (1 << 16) | 7
 
 
 def test_host_settings_roundtrip(fa_lib):
@@ -51,7 +51,7 @@ A16 = 1 << 20  # a 16-byte aligned fake address (never dereferenced)
 @pytest.mark.parametrize("kw,code", [
     (dict(B=-1), 1), (dict(H=-2), 1), (dict(Nq=-1), 1), (dict(Nkv=-5), 1), (dict(d=0), 1),
     (dict(layout=2), 1), (dict(dtype=3), 1), (dict(causal=2), 1),
-    (dict(d=96), 2), (dict(d=256), 2),
+    (dict(d=96), 2), (dict(d=512), 2), (dict(d=256, dtype=2), 2),
     (dict(Nkv=0), 1),
     (dict(q=None), 1), (dict(o=None), 1),
     (dict(q=A16 + 8), 3), (dict(v=A16 + 4), 3), (dict(lse=A16 + 2), 3),
@@ -237,3 +237,38 @@ def test_binding_rejects_host_tensors_and_bad_tables(fa_lib):
         fa.forward_paged(q, kc, kc, table, 40)
     with pytest.raises(ValueError):
         fa.forward(q, q.float(), q)
+
+
+def test_bwd_workspace_size_and_argument_checks(fa_lib):
+    """fa_bwd_workspace_size needs no GPU: an fp32 dQ accumulator plus two
+    padded fp32 row arrays, each part rounded up to 256 bytes.  fa_bwd
+    refuses bad arguments before touching the device (fake, never
+    dereferenced pointers)."""
+    up = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    for B, H, Nq, d in [(1, 1, 1, 64), (2, 3, 300, 128), (1, 40, 8192, 128)]:
+        rc, nb = fa.fa_bwd_workspace_size(B, H, Nq, d)
+        pad = -(-Nq // 128) * 128
+        assert rc == 0 and nb == up(B * H * Nq * d * 4) + 2 * up(B * H * pad * 4)
+    assert fa.fa_bwd_workspace_size(1, 1, 0, 64) == (0, 0)
+    assert fa.fa_bwd_workspace_size(1, 1, 10, 96)[0] == 1
+    assert fa.fa_bwd_workspace_size(-1, 1, 10, 64)[0] == 1
+    a = A16
+    base = [a] * 9 + [a, 1 << 30]  # q k v o dout lse dq dk dv, workspace, bytes
+
+    def call(**kw):
+        args = dict(B=1, H=2, Hkv=2, Nq=300, Nkv=300, d=64, scale=-1.0, causal=0, layout=0, dtype=0)
+        args.update(kw)
+        ptrs = list(base)
+        for i, name in enumerate(["q", "k", "v", "o", "dout", "lse", "dq", "dk", "dv", "ws"]):
+            if name in kw:
+                ptrs[i] = kw.pop(name)
+                args.pop(name, None)
+        return fa.fa_bwd(*ptrs, args["B"], args["H"], args["Hkv"], args["Nq"], args["Nkv"], args["d"], args["scale"],
+                         args["causal"], args["layout"], args["dtype"], None)
+
+    assert call(d=256) == 2 and call(dtype=2) == 2            # unsupported head dim, fp32
+    assert call(Hkv=3) == 1 and call(causal=2) == 1 and call(Nkv=0) == 1
+    assert call(lse=None) == 1 and call(dout=None) == 1
+    assert call(q=A16 + 8) == 3 and call(lse=A16 + 2) == 3
+    assert call(ws=A16 + 16) == 3                             # workspace must be 256-byte aligned
+    assert call(B=0) == 0

@@ -70,3 +70,24 @@ def test_step_percentiles():
     ms = [float(x) for x in range(1, 12)]  # 1 .. 11
     assert bench.step_percentiles(ms) == {"p10": 2.0, "median": 6.0, "p90": 10.0}
     assert bench.step_percentiles([3.5]) == {"p10": 3.5, "median": 3.5, "p90": 3.5}
+
+
+def test_traffic_record_names_its_kernel_sources(tmp_path, monkeypatch):
+    """A record lists the source files of the kernel it captured; it is used
+    while their hash matches, whatever the file name of the record."""
+    import hashlib
+
+    root = tmp_path
+    (root / "profiles").mkdir()
+    csrc = root / "tiled_attention_13_b200" / "csrc"
+    csrc.mkdir(parents=True)
+    (csrc / "fa_fwd_short.cuh").write_text("short kernel\n")
+    (csrc / "ptx.cuh").write_text("helpers\n")
+    sha = hashlib.sha256(b"short kernel\nhelpers\n").hexdigest()
+    rec = {"workload": "cross", "source_files": ["fa_fwd_short.cuh", "ptx.cuh"], "kernel_source_sha256": sha,
+           "dram_bytes_per_launch": 17.0e6}
+    (root / "profiles" / "fa_fwd_short_cross.json").write_text(json.dumps(rec))
+    monkeypatch.setattr(bench, "ROOT", str(root))
+    assert bench.captured_traffic("cross") == 17.0e6
+    (csrc / "ptx.cuh").write_text("helpers v2\n")
+    assert bench.captured_traffic("cross") is None

@@ -459,3 +459,64 @@ def test_splitkv_rejects_a_short_workspace():
     assert fa.fa_fwd_splitkv(*args, None, 0, fa.FA_LAYOUT_BSND, fa.FA_DTYPE_BF16, None) == 1
     assert fa.fa_fwd_splitkv(*args, ws.data_ptr() + 4, nbytes - 16, fa.FA_LAYOUT_BSND, fa.FA_DTYPE_BF16, None) == 1
     assert fa.fa_fwd_splitkv(*args, ws.data_ptr() + 4, nbytes, fa.FA_LAYOUT_BSND, fa.FA_DTYPE_BF16, None) == 3
+
+
+# ----------------------------------------------------------------- short keys (Nkv <= 128)
+# Calls whose keys fit one KV tile run the short-key kernel: one softmax pass
+# per query tile, a static contiguous schedule of query tiles per CTA, K/V
+# loaded again only when the (batch, K/V head) changes, O written by TMA
+# stores from the tile's own Q stage.
+SHORT_CASES = [  # (B, H, Hkv, Nq, Nkv, d, layout, causal, dtype)
+    (1, 1, 1, 1, 1, 64, "BHND", False, "bf16"),
+    (1, 1, 1, 1, 1, 128, "BSND", True, "bf16"),
+    (1, 2, 2, 300, 16, 64, "BHND", False, "bf16"),
+    (1, 2, 2, 300, 17, 128, "BSND", True, "bf16"),
+    (2, 3, 3, 257, 33, 64, "BSND", False, "fp16"),
+    (1, 2, 1, 129, 64, 128, "BHND", True, "fp16"),
+    (2, 4, 2, 500, 96, 64, "BSND", True, "bf16"),
+    (1, 3, 3, 1000, 127, 128, "BHND", False, "bf16"),
+    (2, 2, 2, 640, 128, 64, "BHND", True, "bf16"),
+    (1, 4, 4, 90, 128, 128, "BSND", False, "fp16"),
+    (2, 8, 8, 1024, 77, 64, "BHND", False, "bf16"),
+    (1, 8, 2, 2000, 77, 128, "BSND", False, "bf16"),
+]
+
+
+@pytest.mark.parametrize("case", SHORT_CASES, ids=lambda c: "x".join(map(str, c[:6])) + c[6] + "c" * c[7] + c[8])
+def test_short_keys(case):
+    B, H, Hkv, Nq, Nkv, d, layout, causal, dtype = case
+    compare_full(Workload("short", B=B, H=H, Hkv=Hkv, Nq=Nq, Nkv=Nkv, d=d, dtype=dtype, layout=layout,
+                          causal=causal, seed=Nq * 7 + Nkv))
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_short_keys_many_tiles_per_cta_and_head_switches(d):
+    """Enough query tiles that every CTA wraps its Q ring several times
+    (B4 H32 Nq4096: 4096 tiles on <= 148 CTAs), and single-tile heads so that
+    a CTA changes K/V head on every tile and reuses both K/V slots; checked on
+    sampled rows of several heads."""
+    wl = Workload("short-many", B=4, H=32, Nq=4096, Nkv=77, d=d, dtype="bf16", layout="BHND", causal=False, seed=9)
+    compare_sampled(wl, [(0, 0), (3, 31), (1, 17), (2, 5)], rows_per_head=40)
+    wl = Workload("short-heads", B=5, H=200, Hkv=100, Nq=100, Nkv=120, d=d, dtype="fp16", layout="BSND",
+                  causal=True, seed=10)
+    compare_sampled(wl, [(0, 0), (4, 199), (2, 101), (3, 50), (1, 1)], rows_per_head=20)
+
+
+def test_short_keys_bounded_wait_expires_and_context_survives():
+    """The failure hook on the short-key kernel: P is never signalled, the MMA
+    warp's bounded wait expires, every role leaves its loop and the status
+    word reads FA_ERR_TIMEOUT; the next normal call is correct."""
+    wl = Workload("short-fault", B=2, H=8, Nq=1024, Nkv=77, d=64, dtype="bf16", layout="BHND", causal=False, seed=4)
+    q, k, v = (t.cuda() for t in make_qkv(wl))
+    assert fa.fa_get_device_status(None) == 0
+    prev_t = fa.fa_set_wait_timeout_us(50_000)
+    prev_f = fa.fa_debug_set_fault(1)
+    try:
+        fa.forward(q, k, v)
+        rc = fa.fa_get_device_status(None)
+    finally:
+        fa.fa_debug_set_fault(prev_f)
+        fa.fa_set_wait_timeout_us(prev_t)
+    assert rc == 5, fa.fa_status_string(rc)  # FA_ERR_TIMEOUT
+    assert fa.fa_get_device_status(None) == 0
+    compare_full(wl)

@@ -35,3 +35,29 @@ def test_named_workloads():
     w = WORKLOADS["llama13b-8k"]
     assert w.flops == 4 * 40 * 8192 * 8192 * 128 / 2
     assert WORKLOADS["cross"].bytes_min == 2 * 2 * 8 * 64 * (2 * 4096 + 2 * 77) + 4 * 2 * 8 * 4096
+
+
+def test_block_mask_recipe_and_visible_pairs():
+    """The block-sparse workloads' mask: seeded, diagonal always visible, and
+    the FLOP count's visible-pair total equals a brute-force count over the
+    element mask (block mask expanded, intersected with the causal mask)."""
+    import numpy as np
+
+    from oracle import block_sparse_mask
+    from tiled_attention_13_b200.inputs import Workload, make_block_mask, visible_pairs_block
+
+    for causal in (False, True):
+        wl = Workload("bsp", B=2, H=3, Nq=300, Nkv=260, d=64, causal=causal, block_density=0.4, seed=5)
+        m = make_block_mask(wl)
+        assert m.dtype == torch.uint8 and tuple(m.shape) == (2, 3, 3, 3)
+        assert torch.equal(m, make_block_mask(wl))
+        assert all(int(m[b, h, i, i]) == 1 for b in range(2) for h in range(3) for i in range(3))
+        total = 0
+        for b in range(2):
+            for h in range(3):
+                em = block_sparse_mask(m[b, h].numpy(), 128, 128, wl.Nq, wl.Nkv)
+                if causal:
+                    em &= np.tril(np.ones((wl.Nq, wl.Nkv), dtype=bool))
+                total += int(em.sum())
+        assert visible_pairs_block(wl) == total
+        assert wl.flops == 4.0 * wl.d * total

@@ -22,7 +22,8 @@ import os
 
 __all__ = [
     "FA_LAYOUT_BHND", "FA_LAYOUT_BSND", "FA_DTYPE_BF16", "FA_DTYPE_FP16", "FA_DTYPE_FP32",
-    "FaError", "lib", "lib_path", "fa_fwd", "fa_fwd_gqa", "fa_fwd_band", "fa_fwd_paged", "fa_fwd_noalloc",
+    "FaError", "lib", "lib_path", "fa_fwd", "fa_fwd_gqa", "fa_fwd_band", "fa_fwd_block_sparse", "fa_fwd_paged",
+    "fa_fwd_noalloc", "fa_bwd_workspace_size", "fa_bwd", "backward",
     "fa_splitkv_plan", "fa_fwd_splitkv", "fa_fwd_paged_splitkv", "splitkv_plan", "fa_status_string",
     "fa_get_device_status", "fa_set_wait_timeout_us", "fa_debug_set_fault", "fa_abi_version", "forward",
     "forward_paged", "forward_host",
@@ -33,7 +34,8 @@ FA_LAYOUT_BHND, FA_LAYOUT_BSND = 0, 1
 FA_DTYPE_BF16, FA_DTYPE_FP16, FA_DTYPE_FP32 = 0, 1, 2
 FA_OK = 0
 
-EXPORTED = ("fa_fwd", "fa_fwd_gqa", "fa_fwd_band", "fa_fwd_paged", "fa_fwd_noalloc", "fa_splitkv_plan",
+EXPORTED = ("fa_fwd", "fa_fwd_gqa", "fa_fwd_band", "fa_fwd_block_sparse", "fa_bwd_workspace_size", "fa_bwd",
+            "fa_fwd_paged", "fa_fwd_noalloc", "fa_splitkv_plan",
             "fa_fwd_splitkv", "fa_fwd_paged_splitkv", "fa_status_string", "fa_get_device_status", "fa_set_wait_timeout_us", "fa_debug_set_fault", "fa_abi_version")
 
 _LIB = None
@@ -71,6 +73,14 @@ def lib() -> ctypes.CDLL:
     L.fa_fwd_band.argtypes = [vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, ctypes.c_float, i64, i64, ctypes.c_int,
                               ctypes.c_int, vp]
     L.fa_fwd_band.restype = ctypes.c_int
+    L.fa_fwd_block_sparse.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64, i64, ctypes.c_float,
+                                      ctypes.c_int, ctypes.c_int, ctypes.c_int, vp]
+    L.fa_fwd_block_sparse.restype = ctypes.c_int
+    L.fa_bwd_workspace_size.argtypes = [i64, i64, i64, i64, ctypes.POINTER(i64)]
+    L.fa_bwd_workspace_size.restype = ctypes.c_int
+    L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64, ctypes.c_float,
+                         ctypes.c_int, ctypes.c_int, ctypes.c_int, vp]
+    L.fa_bwd.restype = ctypes.c_int
     L.fa_fwd_paged.argtypes = [vp, vp, vp, vp, vp, vp, i64, i64, i64, i64, i64, i64, i64, i64, i64, ctypes.c_float,
                                ctypes.c_int, ctypes.c_int, ctypes.c_int, vp]
     L.fa_fwd_paged.restype = ctypes.c_int
@@ -119,6 +129,60 @@ def fa_fwd_band(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, d, scale, pre_tokens, next_
     i + next_tokens."""
     return lib().fa_fwd_band(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, d, float(scale), int(pre_tokens), int(next_tokens),
                              int(layout), int(dtype), stream)
+
+
+def fa_fwd_block_sparse(q, k, v, o, lse, block_mask, mask_batch_stride, mask_head_stride, B, H, Hkv, Nq, Nkv, d,
+                        scale, causal, layout, dtype, stream) -> int:
+    """int fa_fwd_block_sparse(...): query tile qt of (b, h) sees key tile kt
+    iff block_mask[b * mask_batch_stride + h * mask_head_stride + qt * KT + kt]
+    != 0 (uint8, 128 x 128 blocks, KT = ceil(Nkv / 128))."""
+    return lib().fa_fwd_block_sparse(q, k, v, o, lse, block_mask, int(mask_batch_stride), int(mask_head_stride), B,
+                                     H, Hkv, Nq, Nkv, d, float(scale), int(causal), int(layout), int(dtype), stream)
+
+
+def fa_bwd_workspace_size(B, H, Nq, d):
+    """int fa_bwd_workspace_size(...) -> (status, workspace_bytes)."""
+    wb = ctypes.c_int64(0)
+    rc = lib().fa_bwd_workspace_size(B, H, Nq, d, ctypes.byref(wb))
+    return rc, wb.value
+
+
+def fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, workspace, workspace_bytes, B, H, Hkv, Nq, Nkv, d, scale, causal, layout,
+           dtype, stream) -> int:
+    """int fa_bwd(...): dQ, dK, dV of the forward, recomputing P tile by tile
+    from q, k and the forward's LSE."""
+    return lib().fa_bwd(q, k, v, o, dout, lse, dq, dk, dv, workspace, int(workspace_bytes), B, H, Hkv, Nq, Nkv, d,
+                        float(scale), int(causal), int(layout), int(dtype), stream)
+
+
+def backward(q, k, v, o, lse, dout, causal: bool = False, scale=None, layout: str = "BHND", stream=None):
+    """(dq, dk, dv) of ``forward(q, k, v, causal, scale, layout)`` for the
+    upstream gradient ``dout`` (o and lse are that forward's outputs).  The
+    workspace comes from torch's caching allocator."""
+    import torch
+
+    for t in (q, k, v, o, dout, lse):
+        if not t.is_cuda or not t.is_contiguous():
+            raise ValueError("q, k, v, o, dout and lse must be contiguous CUDA tensors")
+    B, H, Nq, Nkv, d = _dims(q, k, layout)
+    Hkv = _kv_heads(k, layout)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    rc, nbytes = fa_bwd_workspace_size(B, H, Nq, d)
+    if rc != FA_OK:
+        raise FaError(rc, "fa_bwd_workspace_size")
+    user_stream = stream is not None
+    if stream is None:
+        stream = torch.cuda.current_stream(q.device).cuda_stream
+    ws = torch.empty(max(nbytes, 256), dtype=torch.uint8, device=q.device)
+    if user_stream:
+        ws.record_stream(torch.cuda.ExternalStream(stream, device=q.device))
+    rc = fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), dout.data_ptr(), lse.data_ptr(), dq.data_ptr(),
+                dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), ws.numel(), B, H, Hkv, Nq, Nkv, d,
+                -1.0 if scale is None else float(scale), int(bool(causal)),
+                FA_LAYOUT_BHND if layout == "BHND" else FA_LAYOUT_BSND, _dtype_code(q), stream)
+    if rc != FA_OK:
+        raise FaError(rc, "fa_bwd")
+    return dq, dk, dv
 
 
 def fa_fwd_paged(q, k_cache, v_cache, block_table, o, lse, B, H, Hkv, Nq, Nkv, d, block_size, num_blocks,
@@ -228,18 +292,23 @@ def _splitkv_workspace(B, H, Nq, Nkv, d, num_splits, device, stream, user_stream
 
 
 def forward(q, k, v, causal: bool = False, scale=None, layout: str = "BHND", out=None, lse=None,
-            stream=None, band=None, num_splits=None):
+            stream=None, band=None, num_splits=None, block_mask=None):
     """O, LSE = softmax(scale Q K^T [+causal]) V on the GPU (returns (o, lse)).
 
     q: [B,H,Nq,d] (BHND) or [B,Nq,H,d] (BSND); k, v the same with Nkv and
     Hkv heads (Hkv dividing H: grouped-query attention when Hkv < H); all
-    contiguous CUDA tensors of one dtype (bf16, fp16 or fp32); d in {64, 128}.
+    contiguous CUDA tensors of one dtype (bf16, fp16 or fp32); d in {64, 128},
+    or 256 for bf16/fp16.
     scale None -> 1/sqrt(d).  LSE is fp32 [B, H, Nq].  band = (pre_tokens,
     next_tokens) replaces ``causal``: key j visible to query i iff
     i - pre_tokens <= j <= i + next_tokens (fa_fwd_band; bf16/fp16).
     num_splits (not None; bf16/fp16, no mask) runs split-KV (fa_fwd_splitkv):
     the key tiles cut into that many slices, or as many as the library
-    chooses for this device when it is 0.
+    chooses for this device when it is 0.  block_mask (a uint8 CUDA tensor of
+    shape [B or 1, H or 1, ceil(Nq/128), ceil(Nkv/128)], bf16/fp16) runs
+    fa_fwd_block_sparse: query tile qt sees key tile kt iff the entry is
+    nonzero (and causal still applies when set); a size-1 batch or head
+    dimension is shared.
     """
     import torch
 
@@ -263,14 +332,32 @@ def forward(q, k, v, causal: bool = False, scale=None, layout: str = "BHND", out
     lay = FA_LAYOUT_BHND if layout == "BHND" else FA_LAYOUT_BSND
     lp = lse.data_ptr() if lse.numel() else None
     if num_splits is not None:
-        if causal or band is not None:
-            raise ValueError("split-KV takes no mask (causal=False, band=None)")
+        if causal or band is not None or block_mask is not None:
+            raise ValueError("split-KV takes no mask (causal=False, band=None, block_mask=None)")
         ws = _splitkv_workspace(B, H, Nq, Nkv, d, int(num_splits), q.device, stream, user_stream)
         rc = fa_fwd_splitkv(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lp, B, H, Hkv, Nq, Nkv, d, sc,
                             int(num_splits), None if ws is None else ws.data_ptr(), 0 if ws is None else ws.numel(),
                             lay, _dtype_code(q), stream)
         if rc != FA_OK:
             raise FaError(rc, "fa_fwd_splitkv")
+        return out, lse
+    if block_mask is not None:
+        if band is not None:
+            raise ValueError("give either band or block_mask")
+        import torch as _t
+
+        if block_mask.dtype != _t.uint8 or block_mask.dim() != 4 or not block_mask.is_cuda:
+            raise ValueError("block_mask must be a 4-D uint8 CUDA tensor")
+        qt, kt = -(-Nq // 128), -(-Nkv // 128)
+        if tuple(block_mask.shape[2:]) != (qt, kt) or block_mask.shape[0] not in (1, B) or \
+                block_mask.shape[1] not in (1, H) or block_mask.stride(3) != 1 or block_mask.stride(2) != kt:
+            raise ValueError(f"block_mask must be [B or 1, H or 1, {qt}, {kt}] with dense last two dims")
+        sb = 0 if block_mask.shape[0] == 1 else block_mask.stride(0)
+        sh = 0 if block_mask.shape[1] == 1 else block_mask.stride(1)
+        rc = fa_fwd_block_sparse(q.data_ptr(), k.data_ptr(), v.data_ptr(), out.data_ptr(), lp, block_mask.data_ptr(),
+                                 sb, sh, B, H, Hkv, Nq, Nkv, d, sc, int(bool(causal)), lay, _dtype_code(q), stream)
+        if rc != FA_OK:
+            raise FaError(rc, "fa_fwd_block_sparse")
         return out, lse
     if band is not None:
         if causal:

@@ -22,8 +22,11 @@ namespace fa {
 __device__ unsigned int g_status_word = 0;
 }  // namespace fa
 
+#include "fa_fwd_short.cuh"
 #include "fa_fwd_simt.cuh"
 #include "fa_fwd_tc.cuh"
+#include "fa_fwd_tile1.cuh"
+#include "fa_bwd.cuh"
 #include "fa_splitkv_merge.cuh"
 
 namespace {
@@ -54,6 +57,48 @@ EncodeTiledFn g_encode = nullptr;
 template <typename K>
 bool set_smem_attr(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
+}
+
+// Shared-memory attributes of the short-key kernels.
+bool set_short_attrs() {
+  bool ok = true;
+  ok &= set_smem_attr(fa::fa_fwd_short_kernel<64, __nv_bfloat16>, fa::ShCfg<64>::SMEM_BYTES);
+  ok &= set_smem_attr(fa::fa_fwd_short_kernel<128, __nv_bfloat16>, fa::ShCfg<128>::SMEM_BYTES);
+  ok &= set_smem_attr(fa::fa_fwd_short_kernel<64, __half>, fa::ShCfg<64>::SMEM_BYTES);
+  ok &= set_smem_attr(fa::fa_fwd_short_kernel<128, __half>, fa::ShCfg<128>::SMEM_BYTES);
+  return ok;
+}
+
+// Shared-memory attributes of the one-tile kernels (d = 256, block-sparse).
+template <typename T>
+bool set_t1_attrs_t() {
+  bool ok = true;
+  ok &= set_smem_attr(fa::fa_fwd_t1_kernel<256, T, false>, fa::T1Cfg<256>::SMEM_BYTES);
+  ok &= set_smem_attr(fa::fa_fwd_t1_kernel<64, T, true>, fa::T1Cfg<64>::SMEM_BYTES);
+  ok &= set_smem_attr(fa::fa_fwd_t1_kernel<128, T, true>, fa::T1Cfg<128>::SMEM_BYTES);
+  ok &= set_smem_attr(fa::fa_fwd_t1_kernel<256, T, true>, fa::T1Cfg<256>::SMEM_BYTES);
+  return ok;
+}
+bool set_t1_attrs() {
+#ifdef FA_T1_DENSE
+  // build option: plain d = 64 / 128 calls on the one-tile kernel as well
+  if (!set_smem_attr(fa::fa_fwd_t1_kernel<64, __nv_bfloat16, false>, fa::T1Cfg<64>::SMEM_BYTES) ||
+      !set_smem_attr(fa::fa_fwd_t1_kernel<128, __nv_bfloat16, false>, fa::T1Cfg<128>::SMEM_BYTES) ||
+      !set_smem_attr(fa::fa_fwd_t1_kernel<64, __half, false>, fa::T1Cfg<64>::SMEM_BYTES) ||
+      !set_smem_attr(fa::fa_fwd_t1_kernel<128, __half, false>, fa::T1Cfg<128>::SMEM_BYTES))
+    return false;
+#endif
+  return set_t1_attrs_t<__nv_bfloat16>() && set_t1_attrs_t<__half>();
+}
+
+// Shared-memory attributes of the backward kernels.
+bool set_bwd_attrs() {
+  bool ok = true;
+  ok &= set_smem_attr(fa::fa_bwd_kernel<64, __nv_bfloat16>, fa::BwdCfg<64>::SMEM_BYTES);
+  ok &= set_smem_attr(fa::fa_bwd_kernel<128, __nv_bfloat16>, fa::BwdCfg<128>::SMEM_BYTES);
+  ok &= set_smem_attr(fa::fa_bwd_kernel<64, __half>, fa::BwdCfg<64>::SMEM_BYTES);
+  ok &= set_smem_attr(fa::fa_bwd_kernel<128, __half>, fa::BwdCfg<128>::SMEM_BYTES);
+  return ok;
 }
 
 // Per-device one-time set-up with that device current: properties, the
@@ -95,6 +140,9 @@ int device_setup(int dev, DeviceInfo** out) {
       ok &= set_smem_attr(fa::fa_fwd_tc_kernel<128, __half, true, false, true>, fa::TcCfg<128>::SMEM_BYTES);
       ok &= set_smem_attr(fa::fa_fwd_simt_kernel<64>, fa::simt_smem_bytes<64>());
       ok &= set_smem_attr(fa::fa_fwd_simt_kernel<128>, fa::simt_smem_bytes<128>());
+      ok &= set_short_attrs();
+      ok &= set_t1_attrs();
+      ok &= set_bwd_attrs();
       if (!ok) return FA_ERR_LAUNCH;
       // The tile scheduler's ticket counters: one slot per launch in flight,
       // each put back to zero by the last CTA of its launch.
@@ -302,6 +350,136 @@ int launch_tc(const void* q, const void* k, const void* v, void* o, float* lse, 
   return FA_OK;
 }
 
+// Keys fit one KV tile (Nkv <= 128): the short-key kernel, one pass of
+// softmax per query tile, a static schedule and no work counter.  Plain
+// (contiguous, causal or not, grouped or not) bf16/fp16 calls.
+template <int D, typename T>
+int launch_short(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
+                 int64_t Hkv, int64_t Nq, int64_t Nkv, float scale, int causal, bool bsnd, cudaStream_t stream,
+                 int num_sms, unsigned int* status) {
+  constexpr bool BF16 = std::is_same<T, __nv_bfloat16>::value;
+  CUtensorMap tq, tk, tv, to;
+  if (!make_tmap(&tq, q, BF16, bsnd, B, H, Nq, D) || !make_tmap(&tk, k, BF16, bsnd, B, Hkv, Nkv, D) ||
+      !make_tmap(&tv, v, BF16, bsnd, B, Hkv, Nkv, D) || !make_tmap(&to, o, BF16, bsnd, B, H, Nq, D))
+    return FA_ERR_LAUNCH;
+  fa::ShParams p;
+  p.lse = lse;
+  p.B = (int)B; p.H = (int)H; p.Nq = (int)Nq; p.Nkv = (int)Nkv;
+  p.bsnd = bsnd ? 1 : 0;
+  p.causal = causal;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.qtiles = (int)((Nq + 127) / 128);
+  const int64_t tiles = B * H * (int64_t)p.qtiles;
+  if (tiles > INT32_MAX) return FA_ERR_UNSUPPORTED;
+  p.n_tiles = (int)tiles;
+  p.kv_group = (int)(H / Hkv);
+  p.n_s = (int)((Nkv + 15) / 16) * 16;
+  p.kv_steps = (int)((Nkv + 15) / 16);
+  p.timeout_ns = (uint64_t)g_timeout_us.load() * 1000ull;
+  p.fault_mode = g_fault_mode.load();
+  const int grid = (int)(tiles < num_sms ? tiles : num_sms);
+  fa::fa_fwd_short_kernel<D, T><<<grid, fa::SH_THREADS, fa::ShCfg<D>::SMEM_BYTES, stream>>>(tq, tk, tv, to, p,
+                                                                                            status);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+// A block-sparse mask as fa_fwd_block_sparse receives it.
+struct BlockMask {
+  const uint8_t* mask;  // [.., .., ceil(Nq/128), ceil(Nkv/128)]
+  int64_t batch_stride, head_stride;
+};
+
+// The one-tile kernel: d = 256 (BLOCK false) or a block-sparse mask (BLOCK
+// true, bm the mask).
+template <int D, typename T, bool BLOCK>
+int launch_t1(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H, int64_t Hkv,
+              int64_t Nq, int64_t Nkv, float scale, int causal, bool bsnd, cudaStream_t stream, int num_sms,
+              unsigned int* status, fa::SchedSlot* sched, const BlockMask* bm) {
+  constexpr bool BF16 = std::is_same<T, __nv_bfloat16>::value;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap(&tq, q, BF16, bsnd, B, H, Nq, D) || !make_tmap(&tk, k, BF16, bsnd, B, Hkv, Nkv, D) ||
+      !make_tmap(&tv, v, BF16, bsnd, B, Hkv, Nkv, D))
+    return FA_ERR_LAUNCH;
+  fa::T1Params p;
+  p.o = o;
+  p.lse = lse;
+  p.B = (int)B; p.H = (int)H; p.Nq = (int)Nq; p.Nkv = (int)Nkv;
+  p.bsnd = bsnd ? 1 : 0;
+  p.causal = causal;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.qtiles = (int)((Nq + 127) / 128);
+  p.kvtiles = (int)((Nkv + 127) / 128);
+  const int64_t units = B * H * (int64_t)p.qtiles;
+  if (units > INT32_MAX - 1024) return FA_ERR_UNSUPPORTED;
+  p.n_units = (int)units;
+  p.chunk_heads = chunk_heads_for(B * H, Nkv, D, H / Hkv);
+  p.kv_group = (int)(H / Hkv);
+  p.block_mask = bm != nullptr ? bm->mask : nullptr;
+  p.mask_sb = bm != nullptr ? (long long)bm->batch_stride : 0;
+  p.mask_sh = bm != nullptr ? (long long)bm->head_stride : 0;
+  p.sched = sched;
+  p.timeout_ns = (uint64_t)g_timeout_us.load() * 1000ull;
+  p.fault_mode = g_fault_mode.load();
+  const int grid = (int)(units < num_sms ? units : num_sms);
+  fa::fa_fwd_t1_kernel<D, T, BLOCK><<<grid, fa::T1_THREADS, fa::T1Cfg<D>::SMEM_BYTES, stream>>>(tq, tk, tv, p, status);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
+// The backward workspace: the fp32 dQ accumulator [B, H, Nq, d], then
+// LSE * log2(e) and D = rowsum(dO o O), each [B, H, nq_pad] fp32 with nq_pad
+// = Nq rounded up to 128; each part starts on a 256-byte boundary.
+struct BwdLayout {
+  int64_t nq_pad, off_lse2, off_delta, bytes;
+};
+BwdLayout bwd_layout(int64_t B, int64_t H, int64_t Nq, int64_t d) {
+  BwdLayout L;
+  auto up = [](int64_t x) { return (x + 255) / 256 * 256; };
+  L.nq_pad = (Nq + 127) / 128 * 128;
+  L.off_lse2 = up(B * H * Nq * d * 4);
+  L.off_delta = L.off_lse2 + up(B * H * L.nq_pad * 4);
+  L.bytes = L.off_delta + up(B * H * L.nq_pad * 4);
+  return L;
+}
+
+template <int D, typename T>
+int launch_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,
+               void* dq, void* dk, void* dv, void* ws, int64_t B, int64_t H, int64_t Hkv, int64_t Nq, int64_t Nkv,
+               float scale, int causal, bool bsnd, cudaStream_t stream, unsigned int* status) {
+  constexpr bool BF16 = std::is_same<T, __nv_bfloat16>::value;
+  CUtensorMap tq, tk, tv, tdo;
+  if (!make_tmap(&tq, q, BF16, bsnd, B, H, Nq, D) || !make_tmap(&tk, k, BF16, bsnd, B, Hkv, Nkv, D) ||
+      !make_tmap(&tv, v, BF16, bsnd, B, Hkv, Nkv, D) || !make_tmap(&tdo, dout, BF16, bsnd, B, H, Nq, D))
+    return FA_ERR_LAUNCH;
+  const BwdLayout L = bwd_layout(B, H, Nq, D);
+  fa::BwdParams p;
+  p.o = o; p.dout = dout; p.lse = lse;
+  p.dq_acc = static_cast<float*>(ws);
+  p.lse2 = reinterpret_cast<float*>(static_cast<char*>(ws) + L.off_lse2);
+  p.delta = reinterpret_cast<float*>(static_cast<char*>(ws) + L.off_delta);
+  p.dq = dq; p.dk = dk; p.dv = dv;
+  p.B = (int)B; p.H = (int)H; p.Hkv = (int)Hkv; p.Nq = (int)Nq; p.Nkv = (int)Nkv;
+  p.bsnd = bsnd ? 1 : 0;
+  p.causal = causal;
+  p.scale = scale;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.qtiles = (int)((Nq + 127) / 128);
+  p.kvtiles = (int)((Nkv + 127) / 128);
+  p.nq_pad = (int)L.nq_pad;
+  p.timeout_ns = (uint64_t)g_timeout_us.load() * 1000ull;
+  const int64_t ctas = (int64_t)p.kvtiles * B * Hkv;
+  const int64_t pre_rows = B * H * L.nq_pad, post_items = B * H * Nq * (D / 8);
+  if (ctas > INT32_MAX || pre_rows > (int64_t)INT32_MAX * 256 || post_items > (int64_t)INT32_MAX * 256)
+    return FA_ERR_UNSUPPORTED;
+  if (cudaMemsetAsync(p.dq_acc, 0, (size_t)(B * H * Nq * D * 4), stream) != cudaSuccess) return FA_ERR_LAUNCH;
+  fa::fa_bwd_pre_kernel<D, T><<<(unsigned int)((pre_rows + 255) / 256), 256, 0, stream>>>(p);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  fa::fa_bwd_kernel<D, T><<<(unsigned int)ctas, fa::BWD_THREADS, fa::BwdCfg<D>::SMEM_BYTES, stream>>>(tq, tk, tv, tdo,
+                                                                                                    p, status);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  fa::fa_bwd_post_kernel<D, T><<<(unsigned int)((post_items + 255) / 256), 256, 0, stream>>>(p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
 template <int D>
 int launch_simt(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
                 int64_t Hkv, int64_t Nq, int64_t Nkv, float scale, int causal, bool bsnd, cudaStream_t stream) {
@@ -339,7 +517,8 @@ int fwd_common(const void* q, const void* k, const void* v, void* o, float* lse,
   if (layout != FA_LAYOUT_BHND && layout != FA_LAYOUT_BSND) return FA_ERR_INVALID_ARG;
   if (dtype != FA_DTYPE_BF16 && dtype != FA_DTYPE_FP16 && dtype != FA_DTYPE_FP32) return FA_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  if (d == 256 && dtype == FA_DTYPE_FP32) return FA_ERR_UNSUPPORTED;  // d = 256 is the one-tile kernel's
   if (B == 0 || H == 0 || Nq == 0) return FA_OK;  // nothing to compute
   if (Nkv == 0) return FA_ERR_INVALID_ARG;         // softmax over an empty key set
   if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return FA_ERR_INVALID_ARG;
@@ -358,9 +537,42 @@ int fwd_common(const void* q, const void* k, const void* v, void* o, float* lse,
 
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool bsnd = layout == FA_LAYOUT_BSND;
+#ifdef FA_T1_DENSE
+  if (dtype != FA_DTYPE_FP32 && d != 256 && Nkv > fa::SH_MAX_NKV) {
+    fa::SchedSlot* slot = di->sched + (di->launches.fetch_add(1) % kSchedSlots);
+    if (dtype == FA_DTYPE_BF16)
+      return d == 64 ? launch_t1<64, __nv_bfloat16, false>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s,
+                                                           di->num_sms, di->status, slot, nullptr)
+                     : launch_t1<128, __nv_bfloat16, false>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd,
+                                                            s, di->num_sms, di->status, slot, nullptr);
+    return d == 64 ? launch_t1<64, __half, false>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s,
+                                                  di->num_sms, di->status, slot, nullptr)
+                   : launch_t1<128, __half, false>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s,
+                                                   di->num_sms, di->status, slot, nullptr);
+  }
+#endif
+  if (d == 256) {
+    fa::SchedSlot* slot = di->sched + (di->launches.fetch_add(1) % kSchedSlots);
+    return dtype == FA_DTYPE_BF16
+               ? launch_t1<256, __nv_bfloat16, false>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s,
+                                               di->num_sms, di->status, slot, nullptr)
+               : launch_t1<256, __half, false>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s, di->num_sms,
+                                        di->status, slot, nullptr);
+  }
   if (dtype == FA_DTYPE_FP32) {
     return d == 64 ? launch_simt<64>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s)
                    : launch_simt<128>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s);
+  }
+  if (Nkv <= fa::SH_MAX_NKV) {  // one KV tile per query tile
+    if (dtype == FA_DTYPE_BF16)
+      return d == 64 ? launch_short<64, __nv_bfloat16>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s,
+                                                       di->num_sms, di->status)
+                     : launch_short<128, __nv_bfloat16>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s,
+                                                        di->num_sms, di->status);
+    return d == 64 ? launch_short<64, __half>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s,
+                                              di->num_sms, di->status)
+                   : launch_short<128, __half>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s,
+                                               di->num_sms, di->status);
   }
   if (dtype == FA_DTYPE_BF16) {
     return d == 64
@@ -492,6 +704,111 @@ int fa_fwd_band(const void* q, const void* k, const void* v, void* o, float* lse
                                           &band);
 }
 
+int fa_bwd_workspace_size(int64_t B, int64_t H, int64_t Nq, int64_t d, int64_t* workspace_bytes) {
+  if (B < 0 || H < 0 || Nq < 0 || (d != 64 && d != 128) || workspace_bytes == nullptr) return FA_ERR_INVALID_ARG;
+  if (B > INT32_MAX || H > INT32_MAX || B * H > INT32_MAX || Nq > INT32_MAX - 256) return FA_ERR_UNSUPPORTED;
+  *workspace_bytes = (B == 0 || H == 0 || Nq == 0) ? 0 : bwd_layout(B, H, Nq, d).bytes;
+  return FA_OK;
+}
+
+int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse, void* dq,
+           void* dk, void* dv, void* workspace, int64_t workspace_bytes, int64_t B, int64_t H, int64_t Hkv,
+           int64_t Nq, int64_t Nkv, int64_t d, float scale, int causal, int layout, int dtype, void* stream) {
+  if (B < 0 || H < 0 || Hkv < 0 || Nq < 0 || Nkv < 0 || d <= 0 || workspace_bytes < 0) return FA_ERR_INVALID_ARG;
+  if (H > 0 && (Hkv < 1 || H % Hkv != 0)) return FA_ERR_INVALID_ARG;
+  if (layout != FA_LAYOUT_BHND && layout != FA_LAYOUT_BSND) return FA_ERR_INVALID_ARG;
+  if (dtype != FA_DTYPE_BF16 && dtype != FA_DTYPE_FP16 && dtype != FA_DTYPE_FP32) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (dtype == FA_DTYPE_FP32) return FA_ERR_UNSUPPORTED;  // the backward is the tensor-core kernel's
+  if (B == 0 || H == 0 || (Nq == 0 && Nkv == 0)) return FA_OK;
+  if (Nkv == 0) return FA_ERR_INVALID_ARG;  // the forward was not defined
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || dout == nullptr || lse == nullptr ||
+      dq == nullptr || dk == nullptr || dv == nullptr)
+    return FA_ERR_INVALID_ARG;
+  if (B > INT32_MAX || H > INT32_MAX || B * H > INT32_MAX || Nq > INT32_MAX - 256 || Nkv > INT32_MAX - 256)
+    return FA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) || !aligned(dout, 16) ||
+      !aligned(dq, 16) || !aligned(dk, 16) || !aligned(dv, 16) || !aligned(lse, 4))
+    return FA_ERR_MISALIGNED;
+  if (Nq > 0) {
+    if (workspace == nullptr || workspace_bytes < bwd_layout(B, H, Nq, d).bytes) return FA_ERR_INVALID_ARG;
+    if (!aligned(workspace, 256)) return FA_ERR_MISALIGNED;
+  }
+  if (!(scale > 0.f) || std::isinf(scale)) scale = 1.0f / std::sqrt((float)d);
+
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_NO_DEVICE;
+  DeviceInfo* di = nullptr;
+  const int st = device_setup(dev, &di);
+  if (st != FA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool bsnd = layout == FA_LAYOUT_BSND;
+  if (Nq == 0) {  // no query: dK = dV = 0
+    const size_t nb = (size_t)(B * Hkv * Nkv * d * 2);
+    if (cudaMemsetAsync(dk, 0, nb, s) != cudaSuccess || cudaMemsetAsync(dv, 0, nb, s) != cudaSuccess)
+      return FA_ERR_LAUNCH;
+    return FA_OK;
+  }
+  if (dtype == FA_DTYPE_BF16)
+    return d == 64 ? launch_bwd<64, __nv_bfloat16>(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, Nq, Nkv,
+                                                   scale, causal, bsnd, s, di->status)
+                   : launch_bwd<128, __nv_bfloat16>(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, Nq, Nkv,
+                                                    scale, causal, bsnd, s, di->status);
+  return d == 64 ? launch_bwd<64, __half>(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, Nq, Nkv, scale,
+                                          causal, bsnd, s, di->status)
+                 : launch_bwd<128, __half>(q, k, v, o, dout, lse, dq, dk, dv, workspace, B, H, Hkv, Nq, Nkv, scale,
+                                           causal, bsnd, s, di->status);
+}
+
+int fa_fwd_block_sparse(const void* q, const void* k, const void* v, void* o, float* lse, const uint8_t* block_mask,
+                        int64_t mask_batch_stride, int64_t mask_head_stride, int64_t B, int64_t H, int64_t Hkv,
+                        int64_t Nq, int64_t Nkv, int64_t d, float scale, int causal, int layout, int dtype,
+                        void* stream) {
+  if (B < 0 || H < 0 || Hkv < 0 || Nq < 0 || Nkv < 0 || d <= 0 || mask_batch_stride < 0 || mask_head_stride < 0)
+    return FA_ERR_INVALID_ARG;
+  if (H > 0 && (Hkv < 1 || H % Hkv != 0)) return FA_ERR_INVALID_ARG;
+  if (layout != FA_LAYOUT_BHND && layout != FA_LAYOUT_BSND) return FA_ERR_INVALID_ARG;
+  if (dtype != FA_DTYPE_BF16 && dtype != FA_DTYPE_FP16 && dtype != FA_DTYPE_FP32) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  if (dtype == FA_DTYPE_FP32) return FA_ERR_UNSUPPORTED;  // the block-sparse path is the tensor-core kernel's
+  if (B == 0 || H == 0 || Nq == 0) return FA_OK;          // nothing to compute
+  if (Nkv == 0) return FA_ERR_INVALID_ARG;                // softmax over an empty key set
+  if (q == nullptr || k == nullptr || v == nullptr || o == nullptr || block_mask == nullptr) return FA_ERR_INVALID_ARG;
+  if (B > INT32_MAX || H > INT32_MAX || B * H > INT32_MAX || Nq > INT32_MAX - 256 || Nkv > INT32_MAX - 256 ||
+      (Nkv + 127) / 128 > 32 * fa::T1_MAX_WORDS)
+    return FA_ERR_UNSUPPORTED;
+  if (!aligned(q, 16) || !aligned(k, 16) || !aligned(v, 16) || !aligned(o, 16) ||
+      (lse != nullptr && !aligned(lse, 4)))
+    return FA_ERR_MISALIGNED;
+  if (!(scale > 0.f) || std::isinf(scale)) scale = 1.0f / std::sqrt((float)d);
+
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) return FA_ERR_NO_DEVICE;
+  DeviceInfo* di = nullptr;
+  const int st = device_setup(dev, &di);
+  if (st != FA_OK) return st;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool bsnd = layout == FA_LAYOUT_BSND;
+  const BlockMask bm{block_mask, mask_batch_stride, mask_head_stride};
+  fa::SchedSlot* slot = di->sched + (di->launches.fetch_add(1) % kSchedSlots);
+  const int n = di->num_sms;
+  unsigned int* sw = di->status;
+  if (dtype == FA_DTYPE_BF16) {
+    if (d == 64)
+      return launch_t1<64, __nv_bfloat16, true>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s, n, sw, slot, &bm);
+    if (d == 128)
+      return launch_t1<128, __nv_bfloat16, true>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s, n, sw, slot, &bm);
+    return launch_t1<256, __nv_bfloat16, true>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s, n, sw, slot, &bm);
+  }
+  if (d == 64)
+    return launch_t1<64, __half, true>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s, n, sw, slot, &bm);
+  if (d == 128)
+    return launch_t1<128, __half, true>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s, n, sw, slot, &bm);
+  return launch_t1<256, __half, true>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s, n, sw, slot, &bm);
+}
+
 int fa_fwd_paged(const void* q, const void* k_cache, const void* v_cache, const int* block_table, void* o,
                  float* lse, int64_t B, int64_t H, int64_t Hkv, int64_t Nq, int64_t Nkv, int64_t d,
                  int64_t block_size, int64_t num_blocks, int64_t max_blocks, float scale, int causal, int layout,
@@ -609,7 +926,7 @@ uint32_t fa_set_wait_timeout_us(uint32_t us) {
 
 int fa_debug_set_fault(int mode) { return g_fault_mode.exchange(mode); }
 
-int fa_abi_version(void) { return (1 << 16) | 5; }
+int fa_abi_version(void) { return (1 << 16) | 7; }
 
 #ifdef FA_TRACE_UNITS
 int fa_debug_trace_units_read(unsigned long long* host, int n) {
@@ -691,6 +1008,8 @@ int noalloc_setup(int dev, NoAllocDevice** out) {
       ok &= set_smem_attr(fa::fa_fwd_tc_kernel<128, __half>, fa::TcCfg<128>::SMEM_BYTES);
       ok &= set_smem_attr(fa::fa_fwd_simt_kernel<64>, fa::simt_smem_bytes<64>());
       ok &= set_smem_attr(fa::fa_fwd_simt_kernel<128>, fa::simt_smem_bytes<128>());
+      ok &= set_short_attrs();
+      ok &= set_t1_attrs();
       if (!ok) return FA_ERR_LAUNCH;
       if (g_encode == nullptr) {
         void* fn = nullptr;
@@ -753,7 +1072,8 @@ extern "C" int fa_fwd_noalloc(const void* q, const void* k, const void* v, void*
   if (layout != FA_LAYOUT_BHND && layout != FA_LAYOUT_BSND) return FA_ERR_INVALID_ARG;
   if (dtype != FA_DTYPE_BF16 && dtype != FA_DTYPE_FP16 && dtype != FA_DTYPE_FP32) return FA_ERR_INVALID_ARG;
   if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
-  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  if (d == 256 && dtype == FA_DTYPE_FP32) return FA_ERR_UNSUPPORTED;
   if (B == 0 || H == 0 || Nq == 0) return FA_OK;
   if (Nkv == 0) return FA_ERR_INVALID_ARG;
   if (q == nullptr || k == nullptr || v == nullptr || o == nullptr) return FA_ERR_INVALID_ARG;
@@ -765,7 +1085,8 @@ extern "C" int fa_fwd_noalloc(const void* q, const void* k, const void* v, void*
   // Slot 0 of the fixed scratch holds the 32-bit work-ticket counter: a call
   // fits when it can number all its work units (pairs of 128-row query tiles
   // over every batch and head) plus one closing ticket per CTA.
-  const int64_t units = B * H * (((Nq + fa::TC_BM - 1) / fa::TC_BM + 1) / 2);
+  const int64_t qtiles = (Nq + fa::TC_BM - 1) / fa::TC_BM;
+  const int64_t units = B * H * (d == 256 ? qtiles : (qtiles + 1) / 2);  // d = 256: one query tile per unit
   if (dtype != FA_DTYPE_FP32 && units > (int64_t)INT32_MAX - 1024) return FA_ERR_TOO_LARGE;
   if (!(scale > 0.f) || std::isinf(scale)) scale = 1.0f / std::sqrt((float)d);
 
@@ -780,6 +1101,25 @@ extern "C" int fa_fwd_noalloc(const void* q, const void* k, const void* v, void*
   if (dtype == FA_DTYPE_FP32) {  // this kernel uses no scratch at all
     return d == 64 ? launch_simt<64>(q, k, v, o, lse, B, H, H, Nq, Nkv, scale, causal, bsnd, s)
                    : launch_simt<128>(q, k, v, o, lse, B, H, H, Nq, Nkv, scale, causal, bsnd, s);
+  }
+  if (d == 256) {  // the one-tile kernel, its ticket counter in slot 0 of the fixed scratch
+    if (cudaMemsetAsync(nd->scratch, 0, sizeof(fa::SchedSlot), s) != cudaSuccess) return FA_ERR_LAUNCH;
+    return dtype == FA_DTYPE_BF16
+               ? launch_t1<256, __nv_bfloat16, false>(q, k, v, o, lse, B, H, H, Nq, Nkv, scale, causal, bsnd, s, nd->num_sms,
+                                               nd->status, nd->scratch, nullptr)
+               : launch_t1<256, __half, false>(q, k, v, o, lse, B, H, H, Nq, Nkv, scale, causal, bsnd, s, nd->num_sms,
+                                        nd->status, nd->scratch, nullptr);
+  }
+  if (Nkv <= fa::SH_MAX_NKV) {  // the short-key kernel uses no scratch at all
+    if (dtype == FA_DTYPE_BF16)
+      return d == 64 ? launch_short<64, __nv_bfloat16>(q, k, v, o, lse, B, H, H, Nq, Nkv, scale, causal, bsnd, s,
+                                                       nd->num_sms, nd->status)
+                     : launch_short<128, __nv_bfloat16>(q, k, v, o, lse, B, H, H, Nq, Nkv, scale, causal, bsnd, s,
+                                                        nd->num_sms, nd->status);
+    return d == 64 ? launch_short<64, __half>(q, k, v, o, lse, B, H, H, Nq, Nkv, scale, causal, bsnd, s, nd->num_sms,
+                                              nd->status)
+                   : launch_short<128, __half>(q, k, v, o, lse, B, H, H, Nq, Nkv, scale, causal, bsnd, s, nd->num_sms,
+                                               nd->status);
   }
   if (dtype == FA_DTYPE_BF16) {
     return d == 64 ? launch_tc_noalloc<64, __nv_bfloat16>(q, k, v, o, lse, B, H, Nq, Nkv, scale, causal, bsnd, s, *nd)

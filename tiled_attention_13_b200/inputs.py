@@ -17,13 +17,20 @@ Recipe:
   drawn by ``torch.randperm`` on a CPU generator seeded ``10**9 + seed``;
   every cache element no block-table entry points at (spare blocks, rows past
   Nkv in each sequence's last block) is NaN, so that any read of them shows.
+* Block-sparse masks (``block_density > 0``): a uint8 mask [B, H, ceil(Nq/128),
+  ceil(Nkv/128)] of 128 x 128 blocks, each entry 1 with probability
+  ``block_density`` (``torch.rand`` on a CPU generator seeded
+  ``2 * 10**9 + seed``), and the diagonal blocks (kt == qt) always 1, so that
+  every row of a causal call sees a key.
 * The named workloads are the shapes the surveyed pages benchmark (LLaMA-13B
   self-attention, B=4/H=32/D=128 batched attention, a diffusion cross-attention
   block, 128K long context), plus variants of the LLaMA-13B shape that the
   pages name without sizes: grouped-query (8 K/V heads for its 40 query
   heads), the same through a paged cache, a 2048-key sliding window (band
-  mask), and one decoding step (one query row per head against an 8192-key
-  cache).  No dataset, weights or benchmark items are used: every tensor is
+  mask), one decoding step (one query row per head against an 8192-key
+  cache), a block-sparse mask over it, and head dim 256 at the same model
+  width (20 heads of 256).  The pages give head dims up to 256 and name
+  SparseFlashAttention without a pattern or density.  No dataset, weights or benchmark items are used: every tensor is
   random and only the shapes follow the pages.
 """
 
@@ -56,6 +63,8 @@ class Workload:
     block_size: int = 0  # > 0: K/V read through a paged cache with blocks of this many keys
     band: tuple = ()  # (pre_tokens, next_tokens): key j visible to query i iff i - pre <= j <= i + next
     num_splits: int = -1  # >= 0: split-KV with that many slices of the key tiles (0: the library's count)
+    block_density: float = 0.0  # > 0: block-sparse mask of 128 x 128 blocks with this density (plus the diagonal)
+    backward: bool = False  # the step is the backward pass (dQ, dK, dV for a seeded dO), not the forward
 
     @property
     def kv_heads(self) -> int:
@@ -63,8 +72,14 @@ class Workload:
 
     @property
     def flops(self) -> float:
-        """Algorithmic FLOPs: 4*B*H*Nq*Nkv*d, halved when causal; with a band,
-        4*B*H*d times the number of visible (query, key) pairs."""
+        """Algorithmic FLOPs: 4*B*H*Nq*Nkv*d, halved when causal; with a band
+        or a block-sparse mask, 4*d times the number of visible (query, key)
+        pairs.  The backward's five products (S, dP, dV, dK, dQ) against the
+        forward's two count 2.5 times the forward's."""
+        if self.backward:
+            return 2.5 * self.with_(backward=False).flops
+        if self.block_density > 0:
+            return 4.0 * self.d * float(visible_pairs_block(self))
         if self.band:
             pre, nxt = self.band
             i = torch.arange(self.Nq, dtype=torch.float64)
@@ -77,8 +92,12 @@ class Workload:
 
     @property
     def bytes_min(self) -> int:
-        """Compulsory HBM bytes: read Q, K, V once, write O and the fp32 LSE."""
+        """Compulsory HBM bytes: read Q, K, V once, write O and the fp32 LSE
+        (backward: read Q, K, V, O, dO and the LSE, write dQ, dK, dV)."""
         es = 4 if self.dtype == "fp32" else 2
+        if self.backward:
+            return (es * self.B * self.d * (4 * self.H * self.Nq + 4 * self.kv_heads * self.Nkv)
+                    + 4 * self.B * self.H * self.Nq)
         return (es * self.B * self.d * (2 * self.H * self.Nq + 2 * self.kv_heads * self.Nkv)
                 + 4 * self.B * self.H * self.Nq)
 
@@ -125,6 +144,15 @@ WORKLOADS = {
                               num_splits=0),
     "llama13b-decode-8k-paged16": _wl("llama13b-decode-8k-paged16", 6, B=1, H=40, Nq=1, Nkv=8192, d=128,
                                       layout="BSND", block_size=16, num_splits=0),
+    # the LLaMA-13B 8K causal shape with a block-sparse mask: half of the
+    # 128 x 128 blocks of each head (plus the diagonal) visible
+    "llama13b-8k-bsp50": _wl("llama13b-8k-bsp50", 7, B=1, H=40, Nq=8192, Nkv=8192, d=128, layout="BSND",
+                             causal=True, block_density=0.5),
+    # head dim 256 at the LLaMA-13B model width (20 heads x 256 = 5120), 8K causal
+    "d256-8k": _wl("d256-8k", 8, B=1, H=20, Nq=8192, Nkv=8192, d=256, layout="BSND", causal=True),
+    # the backward pass of the LLaMA-13B 8K causal forward, for a seeded N(0, 1) dO
+    "llama13b-8k-bwd": _wl("llama13b-8k-bwd", 1, B=1, H=40, Nq=8192, Nkv=8192, d=128, layout="BSND", causal=True,
+                           backward=True),
 }
 
 
@@ -141,6 +169,44 @@ def outlier_positions(wl: Workload) -> torch.Tensor:
         return torch.zeros((0,), dtype=torch.int64)
     perm = torch.randperm(wl.Nkv, generator=_gen(4 * wl.seed + 3, "cpu"))
     return torch.sort(perm[:n]).values
+
+
+def make_block_mask(wl: Workload, device="cpu") -> torch.Tensor:
+    """The block-sparse mask of ``wl``: uint8 [B, H, ceil(Nq/128), ceil(Nkv/128)]."""
+    qt, kt = -(-wl.Nq // 128), -(-wl.Nkv // 128)
+    m = torch.rand((wl.B, wl.H, qt, kt), generator=_gen(2 * 10**9 + wl.seed, "cpu")) < wl.block_density
+    d = torch.arange(min(qt, kt))
+    m[:, :, d, d] = True
+    return m.to(torch.uint8).to(device)
+
+
+def visible_pairs_block(wl: Workload) -> int:
+    """(query, key) pairs a block-sparse workload's mask leaves visible
+    (intersected with the causal mask when the workload is causal)."""
+    m = make_block_mask(wl).to(torch.int64)
+    qt, kt = m.shape[2], m.shape[3]
+    rows = torch.clamp(wl.Nq - torch.arange(qt) * 128, max=128)
+    if not wl.causal:
+        cols = torch.clamp(wl.Nkv - torch.arange(kt) * 128, max=128)
+        per = rows.view(-1, 1) * cols.view(1, -1)
+    else:  # pairs (i, j) with j <= i inside each block, summed exactly
+        i = torch.arange(wl.Nq).view(-1, 1)
+        lim = torch.clamp(i + 1, max=wl.Nkv)  # keys [0, lim) per row
+        k0 = (torch.arange(kt) * 128).view(1, -1)
+        cnt = torch.clamp(torch.minimum(lim, k0 + 128) - k0, min=0)  # [Nq, kt]
+        per = torch.zeros((qt, kt), dtype=torch.int64).index_add_(0, torch.arange(wl.Nq) // 128, cnt)
+    return int((m * per.view(1, 1, qt, kt)).sum())
+
+
+def make_dout(wl: Workload, device="cpu"):
+    """The upstream gradient dO of a backward workload: i.i.d. N(0, 1) in q's
+    shape, drawn in fp32 from a generator seeded 7 * seed + 1, rounded to the
+    storage dtype."""
+    dev = torch.device(device)
+    gdev = "cuda" if dev.type == "cuda" else "cpu"
+    with torch.cuda.device(dev) if dev.type == "cuda" else _null():
+        g = torch.randn(wl.q_shape(), generator=_gen(7 * wl.seed + 1, gdev), device=dev, dtype=torch.float32)
+    return g.to(_DTYPES[wl.dtype])
 
 
 def make_qkv(wl: Workload, device="cpu"):

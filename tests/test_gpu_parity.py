@@ -407,6 +407,10 @@ SPLIT_CASES = [  # (B, H, Hkv, Nq, Nkv, d, layout, dtype, num_splits); 0 = the l
     (1, 2, 2, 129, 9000, 64, "BHND", "bf16", 71),   # one key tile per slice, two Q tiles
     (1, 6, 3, 5, 3000, 128, "BHND", "fp16", 0),     # fp16
     (1, 40, 40, 1, 8192, 128, "BSND", "bf16", 0),   # the LLaMA-13B decode step's shape
+    (2, 8, 2, 2, 3001, 64, "BSND", "bf16", 0),      # decode-shaped with 8 rows per K/V head (the most)
+    (1, 8, 1, 1, 2000, 128, "BHND", "fp16", 2),     # multi-query decode, fp16, two slices
+    (3, 4, 4, 3, 77, 64, "BHND", "bf16", 1),        # decode-shaped, one short slice, final O written directly
+    (1, 2, 2, 1, 100000, 128, "BSND", "bf16", 0),   # a long cache: many chunks per warp, ring wrap-around
 ]
 
 

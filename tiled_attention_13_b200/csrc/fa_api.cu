@@ -27,6 +27,7 @@ __device__ unsigned int g_status_word = 0;
 #include "fa_fwd_tc.cuh"
 #include "fa_fwd_tile1.cuh"
 #include "fa_bwd.cuh"
+#include "fa_decode.cuh"
 #include "fa_splitkv_merge.cuh"
 
 namespace {
@@ -94,6 +95,10 @@ bool set_t1_attrs() {
 // Shared-memory attributes of the backward kernels.
 bool set_bwd_attrs() {
   bool ok = true;
+  ok &= set_smem_attr(fa::fa_decode_kernel<64, __nv_bfloat16>, fa::DecCfg<64>::SMEM_BYTES);
+  ok &= set_smem_attr(fa::fa_decode_kernel<128, __nv_bfloat16>, fa::DecCfg<128>::SMEM_BYTES);
+  ok &= set_smem_attr(fa::fa_decode_kernel<64, __half>, fa::DecCfg<64>::SMEM_BYTES);
+  ok &= set_smem_attr(fa::fa_decode_kernel<128, __half>, fa::DecCfg<128>::SMEM_BYTES);
   ok &= set_smem_attr(fa::fa_bwd_kernel<64, __nv_bfloat16>, fa::BwdCfg<64>::SMEM_BYTES);
   ok &= set_smem_attr(fa::fa_bwd_kernel<128, __nv_bfloat16>, fa::BwdCfg<128>::SMEM_BYTES);
   ok &= set_smem_attr(fa::fa_bwd_kernel<64, __half>, fa::BwdCfg<64>::SMEM_BYTES);
@@ -171,21 +176,21 @@ int device_setup(int dev, DeviceInfo** out) {
 }
 
 // 4-D tensor map over a [B, H, N, D] (BHND) or [B, N, H, D] (BSND) 16-bit
-// tensor, box = 64 columns x 128 rows of one (b, h), 128-byte swizzle,
+// tensor, box = 64 columns x box_rows rows of one (b, h), 128-byte swizzle,
 // out-of-range rows read as zero.
 bool make_tmap(CUtensorMap* tm, const void* base, bool bf16, bool bsnd, int64_t B, int64_t H, int64_t N,
-               int64_t D) {
+               int64_t D, uint32_t box_rows = 128) {
   cuuint64_t dims[4], strides[3];
   cuuint32_t box[4], estr[4] = {1, 1, 1, 1};
   const cuuint64_t es = 2;
   if (!bsnd) {
     dims[0] = D; dims[1] = N; dims[2] = H; dims[3] = B;
     strides[0] = D * es; strides[1] = N * D * es; strides[2] = H * N * D * es;
-    box[0] = 64; box[1] = 128; box[2] = 1; box[3] = 1;
+    box[0] = 64; box[1] = box_rows; box[2] = 1; box[3] = 1;
   } else {
     dims[0] = D; dims[1] = H; dims[2] = N; dims[3] = B;
     strides[0] = D * es; strides[1] = H * D * es; strides[2] = N * H * D * es;
-    box[0] = 64; box[1] = 1; box[2] = 128; box[3] = 1;
+    box[0] = 64; box[1] = 1; box[2] = box_rows; box[3] = 1;
   }
   CUresult r = g_encode(tm, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
                         const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
@@ -480,6 +485,43 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
+// Decoding-shaped split-KV (at most fa::DEC_ROWS query rows per batch and
+// K/V head, contiguous K/V): the CUDA-core decode kernel over the plan's
+// slices, then the merge when there is more than one slice.
+template <int D, typename T>
+int launch_decode(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
+                  int64_t Hkv, int64_t Nq, int64_t Nkv, float scale, bool bsnd, cudaStream_t stream,
+                  unsigned int* status, const SplitKV* sk) {
+  constexpr bool BF16 = std::is_same<T, __nv_bfloat16>::value;
+  CUtensorMap tk, tv;
+  if (!make_tmap(&tk, k, BF16, bsnd, B, Hkv, Nkv, D, fa::DEC_CHUNK) ||
+      !make_tmap(&tv, v, BF16, bsnd, B, Hkv, Nkv, D, fa::DEC_CHUNK))
+    return FA_ERR_LAUNCH;
+  fa::DecParams p;
+  p.q = q;
+  p.o = sk != nullptr ? static_cast<void*>(sk->o_part) : o;
+  p.lse = sk != nullptr ? sk->lse_part : lse;
+  p.B = (int)B; p.H = (int)H; p.Hkv = (int)Hkv; p.Nq = (int)Nq; p.Nkv = (int)Nkv;
+  p.bsnd = bsnd ? 1 : 0;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.n_splits = sk != nullptr ? sk->n_splits : 1;
+  p.split_keys = sk != nullptr ? sk->split_tiles * fa::TC_BN : (int)((Nkv + fa::TC_BN - 1) / fa::TC_BN) * fa::TC_BN;
+  p.timeout_ns = (uint64_t)g_timeout_us.load() * 1000ull;
+  const int64_t ctas = (int64_t)p.n_splits * B * Hkv;
+  if (ctas > INT32_MAX) return FA_ERR_UNSUPPORTED;
+  fa::fa_decode_kernel<D, T><<<(unsigned int)ctas, fa::DEC_THREADS, fa::DecCfg<D>::SMEM_BYTES, stream>>>(tk, tv, p,
+                                                                                                       status);
+  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  if (sk != nullptr) {
+    const int64_t rows = B * H * Nq;
+    const int64_t blocks = (rows + fa::MERGE_ROWS_PER_CTA - 1) / fa::MERGE_ROWS_PER_CTA;
+    fa::fa_splitkv_merge_kernel<D, T><<<(unsigned int)blocks, fa::MERGE_THREADS, 0, stream>>>(
+        sk->o_part, sk->lse_part, static_cast<T*>(o), lse, (int)B, (int)H, (int)Nq, sk->n_splits, bsnd ? 1 : 0);
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  }
+  return FA_OK;
+}
+
 template <int D>
 int launch_simt(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
                 int64_t Hkv, int64_t Nq, int64_t Nkv, float scale, int causal, bool bsnd, cudaStream_t stream) {
@@ -638,6 +680,15 @@ int splitkv_common(const void* q, const void* k, const void* v, const PagedKV* p
   const SplitKV* skp = S > 1 ? &sk : nullptr;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool bsnd = layout == FA_LAYOUT_BSND;
+  if (pg == nullptr && Nq * (H / Hkv) <= fa::DEC_ROWS) {  // decoding-shaped: the CUDA-core kernel
+    if (dtype == FA_DTYPE_BF16)
+      return d == 64 ? launch_decode<64, __nv_bfloat16>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, bsnd, s,
+                                                        di->status, skp)
+                     : launch_decode<128, __nv_bfloat16>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, bsnd, s,
+                                                         di->status, skp);
+    return d == 64 ? launch_decode<64, __half>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, bsnd, s, di->status, skp)
+                   : launch_decode<128, __half>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, bsnd, s, di->status, skp);
+  }
   if (dtype == FA_DTYPE_BF16)
     return d == 64 ? launch_tc<64, __nv_bfloat16>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, 0, bsnd, s, *di, pg,
                                                   nullptr, skp)

@@ -454,8 +454,9 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     if (ok && n > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DKDV), 0, wctx));
     if (ok) {
       tc_fence_after();
-      const bool store = key < p.Nkv;
       const long long off = bwd_row(p.bsnd, b, hk, key < p.Nkv ? key : 0, p.Hkv, p.Nkv, D);
+      const bool store =
+          key < p.Nkv && FA_INDEX_OK(status_word, off >= 0 && off + D <= (long long)p.B * p.Hkv * p.Nkv * D);
       T* dvp = static_cast<T*>(p.dv) + off;
       T* dkp = static_cast<T*>(p.dk) + off;
 #pragma unroll 1

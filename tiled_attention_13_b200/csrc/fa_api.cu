@@ -26,6 +26,7 @@ __device__ unsigned int g_status_word = 0;
 #include "fa_fwd_simt.cuh"
 #include "fa_fwd_tc.cuh"
 #include "fa_fwd_tile1.cuh"
+#include "fa_fwd_tc2.cuh"
 #include "fa_bwd.cuh"
 #include "fa_decode.cuh"
 #include "fa_splitkv_merge.cuh"
@@ -95,6 +96,12 @@ bool set_t1_attrs() {
 // Shared-memory attributes of the backward kernels.
 bool set_bwd_attrs() {
   bool ok = true;
+#ifdef FA_TC2
+  ok &= set_smem_attr(fa::fa_fwd_tc2_kernel<64, __nv_bfloat16>, fa::T2Cfg<64>::SMEM_BYTES);
+  ok &= set_smem_attr(fa::fa_fwd_tc2_kernel<128, __nv_bfloat16>, fa::T2Cfg<128>::SMEM_BYTES);
+  ok &= set_smem_attr(fa::fa_fwd_tc2_kernel<64, __half>, fa::T2Cfg<64>::SMEM_BYTES);
+  ok &= set_smem_attr(fa::fa_fwd_tc2_kernel<128, __half>, fa::T2Cfg<128>::SMEM_BYTES);
+#endif
   ok &= set_smem_attr(fa::fa_decode_kernel<64, __nv_bfloat16>, fa::DecCfg<64>::SMEM_BYTES);
   ok &= set_smem_attr(fa::fa_decode_kernel<128, __nv_bfloat16>, fa::DecCfg<128>::SMEM_BYTES);
   ok &= set_smem_attr(fa::fa_decode_kernel<64, __half>, fa::DecCfg<64>::SMEM_BYTES);
@@ -485,6 +492,41 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
+// The one-row-per-thread two-tile kernel (plain calls: contiguous K/V, causal
+// or not, grouped K/V heads).
+template <int D, typename T>
+int launch_tc2(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H, int64_t Hkv,
+               int64_t Nq, int64_t Nkv, float scale, int causal, bool bsnd, cudaStream_t stream, DeviceInfo& di) {
+  constexpr bool BF16 = std::is_same<T, __nv_bfloat16>::value;
+  CUtensorMap tq, tk, tv;
+  if (!make_tmap(&tq, q, BF16, bsnd, B, H, Nq, D) || !make_tmap(&tk, k, BF16, bsnd, B, Hkv, Nkv, D) ||
+      !make_tmap(&tv, v, BF16, bsnd, B, Hkv, Nkv, D))
+    return FA_ERR_LAUNCH;
+  fa::TcParams p;
+  p.o = o;
+  p.lse = lse;
+  p.B = (int)B; p.H = (int)H; p.Nq = (int)Nq; p.Nkv = (int)Nkv;
+  p.bsnd = bsnd ? 1 : 0;
+  p.causal = causal;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  const int64_t qtiles = (Nq + fa::TC_BM - 1) / fa::TC_BM;
+  p.n_pairs = (int)((qtiles + 1) / 2);
+  const int64_t units = B * H * (int64_t)p.n_pairs;
+  if (units > INT32_MAX - 1024) return FA_ERR_UNSUPPORTED;
+  p.n_units = (int)units;
+  p.chunk_heads = chunk_heads_for(B * H, Nkv, D, H / Hkv);
+  p.kv_group = (int)(H / Hkv);
+  p.block_table = nullptr;
+  p.block_size = p.max_blocks = p.num_blocks = 0;
+  p.band.pre_tokens = p.band.next_tokens = 0;
+  p.sched = di.sched + (di.launches.fetch_add(1) % kSchedSlots);
+  p.timeout_ns = (uint64_t)g_timeout_us.load() * 1000ull;
+  p.fault_mode = g_fault_mode.load();
+  const int grid = (int)(units < di.num_sms ? units : di.num_sms);
+  fa::fa_fwd_tc2_kernel<D, T><<<grid, fa::T2_THREADS, fa::T2Cfg<D>::SMEM_BYTES, stream>>>(tq, tk, tv, p, di.status);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
 // Decoding-shaped split-KV (at most fa::DEC_ROWS query rows per batch and
 // K/V head, contiguous K/V): the CUDA-core decode kernel over the plan's
 // slices, then the merge when there is more than one slice.
@@ -616,6 +658,13 @@ int fwd_common(const void* q, const void* k, const void* v, void* o, float* lse,
                    : launch_short<128, __half>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s,
                                                di->num_sms, di->status);
   }
+#ifdef FA_TC2
+  if (dtype == FA_DTYPE_BF16)
+    return d == 64 ? launch_tc2<64, __nv_bfloat16>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s, *di)
+                   : launch_tc2<128, __nv_bfloat16>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s, *di);
+  return d == 64 ? launch_tc2<64, __half>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s, *di)
+                 : launch_tc2<128, __half>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s, *di);
+#endif
   if (dtype == FA_DTYPE_BF16) {
     return d == 64
                ? launch_tc<64, __nv_bfloat16>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s, *di)

@@ -170,9 +170,9 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
     const uint32_t kb = ring + st * C::STAGE_BYTES, vb = kb + C::KV_BYTES;
     const int key = k0 + (warp + j * DEC_WARPS) * DEC_CHUNK + lane;  // this lane's key
     // scores: lane = key
-    float s[DEC_ROWS];
+    float s[DEC_ROWS], s2[DEC_ROWS];  // two partial sums per row: shorter FMA chains
 #pragma unroll
-    for (int r = 0; r < DEC_ROWS; ++r) s[r] = 0.f;
+    for (int r = 0; r < DEC_ROWS; ++r) s[r] = s2[r] = 0.f;
 #pragma unroll
     for (int c = 0; c < C::SUB; ++c) {
 #pragma unroll
@@ -188,15 +188,16 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
           if (r < R) {
             const float4 qa = *reinterpret_cast<const float4*>(qs + r * D + c * 64 + pc * 8);
             const float4 qb = *reinterpret_cast<const float4*>(qs + r * D + c * 64 + pc * 8 + 4);
-            s[r] = fmaf(qa.x, kf[0], s[r]); s[r] = fmaf(qa.y, kf[1], s[r]);
-            s[r] = fmaf(qa.z, kf[2], s[r]); s[r] = fmaf(qa.w, kf[3], s[r]);
-            s[r] = fmaf(qb.x, kf[4], s[r]); s[r] = fmaf(qb.y, kf[5], s[r]);
-            s[r] = fmaf(qb.z, kf[6], s[r]); s[r] = fmaf(qb.w, kf[7], s[r]);
+            s[r] = fmaf(qa.x, kf[0], s[r]); s2[r] = fmaf(qa.y, kf[1], s2[r]);
+            s[r] = fmaf(qa.z, kf[2], s[r]); s2[r] = fmaf(qa.w, kf[3], s2[r]);
+            s[r] = fmaf(qb.x, kf[4], s[r]); s2[r] = fmaf(qb.y, kf[5], s2[r]);
+            s[r] = fmaf(qb.z, kf[6], s[r]); s2[r] = fmaf(qb.w, kf[7], s2[r]);
           }
         }
       }
     }
-    // this lane's V columns of the 32 keys are read below; the stage's K is done
+#pragma unroll
+    for (int r = 0; r < DEC_ROWS; ++r) s[r] += s2[r];
     const bool live = key < k1;
     float pr[DEC_ROWS];
 #pragma unroll

@@ -93,6 +93,15 @@ bool set_t1_attrs() {
   return set_t1_attrs_t<__nv_bfloat16>() && set_t1_attrs_t<__half>();
 }
 
+// Shared-memory attributes of the decode kernels (every row count).
+template <int D, typename T>
+bool set_decode_attrs() {
+  return set_smem_attr(fa::fa_decode_kernel<D, T, 1>, fa::DecCfg<D>::SMEM_BYTES) &&
+         set_smem_attr(fa::fa_decode_kernel<D, T, 2>, fa::DecCfg<D>::SMEM_BYTES) &&
+         set_smem_attr(fa::fa_decode_kernel<D, T, 4>, fa::DecCfg<D>::SMEM_BYTES) &&
+         set_smem_attr(fa::fa_decode_kernel<D, T, 8>, fa::DecCfg<D>::SMEM_BYTES);
+}
+
 // Shared-memory attributes of the backward kernels.
 bool set_bwd_attrs() {
   bool ok = true;
@@ -102,10 +111,8 @@ bool set_bwd_attrs() {
   ok &= set_smem_attr(fa::fa_fwd_tc2_kernel<64, __half>, fa::T2Cfg<64>::SMEM_BYTES);
   ok &= set_smem_attr(fa::fa_fwd_tc2_kernel<128, __half>, fa::T2Cfg<128>::SMEM_BYTES);
 #endif
-  ok &= set_smem_attr(fa::fa_decode_kernel<64, __nv_bfloat16>, fa::DecCfg<64>::SMEM_BYTES);
-  ok &= set_smem_attr(fa::fa_decode_kernel<128, __nv_bfloat16>, fa::DecCfg<128>::SMEM_BYTES);
-  ok &= set_smem_attr(fa::fa_decode_kernel<64, __half>, fa::DecCfg<64>::SMEM_BYTES);
-  ok &= set_smem_attr(fa::fa_decode_kernel<128, __half>, fa::DecCfg<128>::SMEM_BYTES);
+  ok &= set_decode_attrs<64, __nv_bfloat16>() && set_decode_attrs<128, __nv_bfloat16>();
+  ok &= set_decode_attrs<64, __half>() && set_decode_attrs<128, __half>();
   ok &= set_smem_attr(fa::fa_bwd_kernel<64, __nv_bfloat16>, fa::BwdCfg<64>::SMEM_BYTES);
   ok &= set_smem_attr(fa::fa_bwd_kernel<128, __nv_bfloat16>, fa::BwdCfg<128>::SMEM_BYTES);
   ok &= set_smem_attr(fa::fa_bwd_kernel<64, __half>, fa::BwdCfg<64>::SMEM_BYTES);
@@ -551,8 +558,17 @@ int launch_decode(const void* q, const void* k, const void* v, void* o, float* l
   p.timeout_ns = (uint64_t)g_timeout_us.load() * 1000ull;
   const int64_t ctas = (int64_t)p.n_splits * B * Hkv;
   if (ctas > INT32_MAX) return FA_ERR_UNSUPPORTED;
-  fa::fa_decode_kernel<D, T><<<(unsigned int)ctas, fa::DEC_THREADS, fa::DecCfg<D>::SMEM_BYTES, stream>>>(tk, tv, p,
-                                                                                                       status);
+  const int64_t R = Nq * (H / Hkv);  // rows per (batch, K/V head), at most fa::DEC_ROWS
+  const dim3 grid((unsigned int)ctas);
+  const int sm = fa::DecCfg<D>::SMEM_BYTES;
+  if (R <= 1)
+    fa::fa_decode_kernel<D, T, 1><<<grid, fa::DEC_THREADS, sm, stream>>>(tk, tv, p, status);
+  else if (R <= 2)
+    fa::fa_decode_kernel<D, T, 2><<<grid, fa::DEC_THREADS, sm, stream>>>(tk, tv, p, status);
+  else if (R <= 4)
+    fa::fa_decode_kernel<D, T, 4><<<grid, fa::DEC_THREADS, sm, stream>>>(tk, tv, p, status);
+  else
+    fa::fa_decode_kernel<D, T, 8><<<grid, fa::DEC_THREADS, sm, stream>>>(tk, tv, p, status);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
   if (sk != nullptr) {
     const int64_t rows = B * H * Nq;

@@ -14,7 +14,7 @@
 //   fa_bwd_pre_kernel    D and LSE * log2(e) per query row, into the caller's
 //                        workspace, padded to whole 128-row tiles (padding:
 //                        LSE = +inf, so P = 0 there, and D = 0).
-//   fa_bwd_kernel        one CTA per (batch, K/V head, 128-key tile), keeping
+//   fa_bwd_kernel        one CTA per (batch, K/V head, 128-key tile), head-major, keeping
 //                        that tile's K and V in shared memory and its dK and
 //                        dV in tensor memory while it walks every query tile
 //                        of every query head that reads this K/V head (under
@@ -37,7 +37,8 @@
 //               then dS^T = P^T o (dP^T - D); P^T and dS^T go back to tensor
 //               memory as 16-bit pairs, dS^T also to shared memory in the
 //               128-byte-swizzled layout; then the thread reads one query row
-//               of dQ and adds it to the accumulator.  After the last step it
+//               of dQ and adds it to the accumulator (a bulk reduction of
+//               each 32-column piece, staged through the dS tile).  After the last step it
 //               writes its key row of dV and scale * dK.
 //
 // TMEM (512 columns): R_S [0, 128), R_DP [128, 256), dV [256, 256 + D),
@@ -56,6 +57,12 @@
 
 namespace fa {
 
+#ifndef FA_BWD_BULK_DQ
+#define FA_BWD_BULK_DQ 1
+#endif
+// 1: dQ rows reach the accumulator as bulk reductions from shared memory (one
+// per thread and 32 columns); 0: as per-thread 16-byte vector reductions.
+constexpr int BWD_BULK_DQ = FA_BWD_BULK_DQ;
 constexpr int BWD_WARP_MMA = 4;
 constexpr int BWD_WARP_TMA = 5;
 constexpr int BWD_THREADS = 32 * 6;
@@ -192,10 +199,11 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // This CTA's key tile: the heaviest (first) key tiles of a causal call go first.
-  const int BHk = p.B * p.Hkv;
-  const int kt = blockIdx.x / BHk;
-  const int bhk = blockIdx.x - kt * BHk;
+  // This CTA's (batch, K/V head) and key tile: head-major, so that the CTAs
+  // in flight share a few heads' Q, dO and dQ accumulator in L2; within a
+  // head the heaviest key tiles (the first, under a causal mask) go first.
+  const int bhk = blockIdx.x / p.kvtiles;
+  const int kt = blockIdx.x - bhk * p.kvtiles;
   const int b = bhk / p.Hkv, hk = bhk - b * p.Hkv;
   const int group = p.H / p.Hkv;
   const int qt0 = p.causal ? kt : 0;  // query i sees key j iff j <= i: tiles before kt see none of these keys
@@ -435,21 +443,48 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       tc_fence_after();
       const int qrow = qt * 128 + r;
       float* acc = p.dq_acc + (bh * p.Nq + qrow) * D;
+      const bool qvalid = qrow < p.Nq && FA_INDEX_OK(status_word, (bh * p.Nq + qrow) < (long long)p.B * p.H * p.Nq);
+      if constexpr (BWD_BULK_DQ) {
+        // 32 columns at a time through the dS tile (free: dQ's MMA has read
+        // it): this thread's 128 bytes at a row stride of 144 bytes (eight
+        // consecutive rows then fall on different banks), then one bulk add
+        // of them into the accumulator row.
+        const uint32_t rowb = sbase + C::OFF_DS + r * 144;
 #pragma unroll 1
-      for (int c = 0; c < D; c += 32) {
-        float v[32];
-        tmem_ld32(tl + C::R_DQ + c, v);
-        if (qrow < p.Nq && FA_INDEX_OK(status_word, (bh * p.Nq + qrow) < (long long)p.B * p.H * p.Nq)) {
+        for (int c0 = 0; c0 < D; c0 += 32) {
+          float v[32];
+          tmem_ld32(tl + C::R_DQ + c0, v);
+          if (c0 > 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
 #pragma unroll
-          for (int t = 0; t < 8; ++t)
-            asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(acc + c + 4 * t), "f"(v[4 * t]),
-                         "f"(v[4 * t + 1]), "f"(v[4 * t + 2]), "f"(v[4 * t + 3])
+          for (int j = 0; j < 8; ++j)
+            st_shared_v4(rowb + j * 16, __float_as_uint(v[4 * j]), __float_as_uint(v[4 * j + 1]),
+                         __float_as_uint(v[4 * j + 2]), __float_as_uint(v[4 * j + 3]));
+          fence_proxy_async_smem();
+          if (qvalid)
+            asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], 128;" ::"l"(acc + c0),
+                         "r"(rowb)
                          : "memory");
+          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
+        }
+        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");  // the dS tile is written again next step
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < D; c += 32) {
+          float v[32];
+          tmem_ld32(tl + C::R_DQ + c, v);
+          if (qvalid) {
+#pragma unroll
+            for (int t = 0; t < 8; ++t)
+              asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(acc + c + 4 * t), "f"(v[4 * t]),
+                           "f"(v[4 * t + 1]), "f"(v[4 * t + 2]), "f"(v[4 * t + 3])
+                           : "memory");
+          }
         }
       }
       tc_fence_before();
       mbar_arrive_warp(bar(B_DQFREE));
     }
+    if constexpr (BWD_BULK_DQ) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");  // dQ adds complete
     // ---------------------------------------------------------- dK, dV of this key row
     if (ok && n > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DKDV), 0, wctx));
     if (ok) {

@@ -88,7 +88,10 @@ __device__ __forceinline__ void dec_unpack8(uint4 w, float (&f)[8]) {
   }
 }
 
-template <int D, typename T>
+// RR: the rows a CTA computes, R rounded up to a power of two (1, 2, 4 or 8),
+// a compile-time count so that no per-row work is predicated off; rows past R
+// have q = 0 and are not stored.
+template <int D, typename T, int RR>
 __global__ void __launch_bounds__(DEC_THREADS, 1)
     fa_decode_kernel(const __grid_constant__ CUtensorMap tm_k, const __grid_constant__ CUtensorMap tm_v,
                      DecParams p, unsigned int* status_word) {
@@ -154,9 +157,9 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
     for (int j = 0; j < DEC_ST && j < mine; ++j) issue(j);
   __syncwarp();
 
-  float m[DEC_ROWS], l[DEC_ROWS], acc[DEC_ROWS][E];
+  float m[RR], l[RR], acc[RR][E];
 #pragma unroll
-  for (int r = 0; r < DEC_ROWS; ++r) {
+  for (int r = 0; r < RR; ++r) {
     m[r] = -INFINITY;
     l[r] = 0.f;
 #pragma unroll
@@ -170,9 +173,9 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
     const uint32_t kb = ring + st * C::STAGE_BYTES, vb = kb + C::KV_BYTES;
     const int key = k0 + (warp + j * DEC_WARPS) * DEC_CHUNK + lane;  // this lane's key
     // scores: lane = key
-    float s[DEC_ROWS], s2[DEC_ROWS];  // two partial sums per row: shorter FMA chains
+    float s[RR], s2[RR];  // two partial sums per row: shorter FMA chains
 #pragma unroll
-    for (int r = 0; r < DEC_ROWS; ++r) s[r] = s2[r] = 0.f;
+    for (int r = 0; r < RR; ++r) s[r] = s2[r] = 0.f;
 #pragma unroll
     for (int c = 0; c < C::SUB; ++c) {
 #pragma unroll
@@ -184,8 +187,8 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
         float kf[8];
         dec_unpack8<T>(w, kf);
 #pragma unroll
-        for (int r = 0; r < DEC_ROWS; ++r) {
-          if (r < R) {
+        for (int r = 0; r < RR; ++r) {
+          {
             const float4 qa = *reinterpret_cast<const float4*>(qs + r * D + c * 64 + pc * 8);
             const float4 qb = *reinterpret_cast<const float4*>(qs + r * D + c * 64 + pc * 8 + 4);
             s[r] = fmaf(qa.x, kf[0], s[r]); s2[r] = fmaf(qa.y, kf[1], s2[r]);
@@ -197,12 +200,11 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
       }
     }
 #pragma unroll
-    for (int r = 0; r < DEC_ROWS; ++r) s[r] += s2[r];
+    for (int r = 0; r < RR; ++r) s[r] += s2[r];
     const bool live = key < k1;
-    float pr[DEC_ROWS];
+    float pr[RR];
 #pragma unroll
-    for (int r = 0; r < DEC_ROWS; ++r) {
-      if (r >= R) { pr[r] = 0.f; continue; }
+    for (int r = 0; r < RR; ++r) {
       const float x = live ? s[r] * sl2 : -INFINITY;
       float mx = x;
 #pragma unroll
@@ -232,12 +234,10 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
         dec_unpack8<T>(make_uint4(w0, 0u, 0u, 0u), vf);
       }
 #pragma unroll
-      for (int r = 0; r < DEC_ROWS; ++r) {
-        if (r < R) {
-          const float pk = __shfl_sync(0xffffffffu, pr[r], kk);
+      for (int r = 0; r < RR; ++r) {
+        const float pk = __shfl_sync(0xffffffffu, pr[r], kk);
 #pragma unroll
-          for (int e = 0; e < E; ++e) acc[r][e] = fmaf(pk, vf[e], acc[r][e]);
-        }
+        for (int e = 0; e < E; ++e) acc[r][e] = fmaf(pk, vf[e], acc[r][e]);
       }
     }
     __syncwarp();
@@ -254,7 +254,7 @@ __global__ void __launch_bounds__(DEC_THREADS, 1)
   // this warp's state into shared memory: m, l (summed over lanes), O
   float* rw = red + warp * C::RED_FLOATS;
 #pragma unroll
-  for (int r = 0; r < DEC_ROWS; ++r) {
+  for (int r = 0; r < RR; ++r) {
     float lt = l[r];
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) lt += __shfl_xor_sync(0xffffffffu, lt, o);

@@ -136,17 +136,20 @@ __device__ __forceinline__ void sh_bulk_commit() { asm volatile("cp.async.bulk.c
 __device__ __forceinline__ void sh_bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
 __device__ __forceinline__ void sh_bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
 
-// Non-blocking test of an mbarrier phase (mbarrier.test_wait returns at once;
-// try_wait may first suspend the thread for a while), for issue loops that
-// poll several barriers and must not sit on one that is not ready yet.
-__device__ __forceinline__ bool mbar_test(uint32_t bar, uint32_t parity) {
+// Poll of an mbarrier phase for issue loops that watch several barriers:
+// the waiting thread may be suspended for at most a few tens of nanoseconds
+// (the suspend-time hint), so a barrier that is not ready yet neither holds
+// up the others for long (a plain try_wait may suspend for a
+// system-dependent time) nor lets the poll spin on issue slots the softmax
+// warps of the same sub-partition need.
+__device__ __forceinline__ bool mbar_poll(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2;\n\t"
+      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(40u)
       : "memory");
   return ok != 0;
 }
@@ -300,7 +303,7 @@ __global__ void __launch_bounds__(SH_THREADS, 1)
     // a CTA's MMAs in issue order, so S(js) overwrites P(js - 2) only after it
     // was read).  P V comes first when both are ready.  Polls are warp-wide;
     // a stretch with nothing ready is bounded like every other wait.
-    auto ready = [&](int b, uint32_t ph) { return __all_sync(0xffffffffu, mbar_test(bar(b), ph)); };
+    auto ready = [&](int b, uint32_t ph) { return __all_sync(0xffffffffu, mbar_poll(bar(b), ph)); };
     int js = 0, jp = 0;
     int s_kv = -1, s_loads = 0;  // K/V slot bookkeeping of the S side
     int v_kv = -1, v_loads = 0;  // and of the P V side
@@ -354,9 +357,7 @@ __global__ void __launch_bounds__(SH_THREADS, 1)
         idle_since = 0;
         continue;
       }
-      // nothing was ready: back off briefly (the polls do not block), and give
-      // up on abort or after the wait limit
-      __nanosleep(32);
+      // nothing was ready: give up on abort or after the wait limit
       const uint64_t now = globaltimer_ns();
       if (idle_since == 0) idle_since = now;
       const int give_up = __shfl_sync(0xffffffffu, (*abort_flag != 0 || now - idle_since > p.timeout_ns) ? 1 : 0, 0);

@@ -373,7 +373,7 @@ __global__ void __launch_bounds__(T1_THREADS, 1)
     const uint64_t dK0 = smem_desc_sw128(sbase + C::OFF_K, 16, 1024);
     const uint64_t dV0 = smem_desc_sw128(sbase + C::OFF_V, C::CHUNK_BYTES, 1024);
     const uint32_t tO = tmem + 256;
-    auto ready = [&](int b, uint32_t ph) { return __all_sync(0xffffffffu, mbar_test(bar(b), ph)); };
+    auto ready = [&](int b, uint32_t ph) { return __all_sync(0xffffffffu, mbar_poll(bar(b), ph)); };
     int uslot = 0;
     uint32_t uphase = 0;
     int gs = 0, gp = 0, gq = 0;  // S steps, P V steps and query tiles so far (all units)
@@ -432,7 +432,6 @@ __global__ void __launch_bounds__(T1_THREADS, 1)
           idle_since = 0;
           continue;
         }
-        __nanosleep(32);  // nothing was ready: back off briefly (the polls do not block)
         const uint64_t now = globaltimer_ns();
         if (idle_since == 0) idle_since = now;
         const int give_up = __shfl_sync(0xffffffffu, (*abort_flag != 0 || now - idle_since > p.timeout_ns) ? 1 : 0, 0);

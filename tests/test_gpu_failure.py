@@ -18,8 +18,13 @@ from .parity import compare_full
 pytestmark = pytest.mark.gpu
 
 
-def test_bounded_wait_expires_and_context_survives(fa_lib):
-    wl = Workload("fault", B=1, H=2, Nq=256, Nkv=300, d=128, dtype="bf16", layout="BHND", causal=False, seed=4)
+@pytest.mark.parametrize("causal,d", [(False, 128), (True, 128), (False, 64), (True, 256)],
+                         ids=["one-row-kernel", "two-tile-kernel", "two-tile-kernel-d64", "one-tile-kernel-d256"])
+def test_bounded_wait_expires_and_context_survives(fa_lib, causal, d):
+    """Every kernel family behind fa_fwd: the non-causal d = 128 call runs the
+    one-row-per-thread kernel, causal and d = 64 calls the two-tile kernel,
+    d = 256 the one-tile kernel."""
+    wl = Workload("fault", B=1, H=2, Nq=256, Nkv=300, d=d, dtype="bf16", layout="BHND", causal=causal, seed=4)
     q = torch.randn(wl.q_shape(), device="cuda").to(torch.bfloat16)
     k = torch.randn(wl.kv_shape(), device="cuda").to(torch.bfloat16)
     v = torch.randn(wl.kv_shape(), device="cuda").to(torch.bfloat16)
@@ -27,7 +32,7 @@ def test_bounded_wait_expires_and_context_survives(fa_lib):
     prev_t = fa.fa_set_wait_timeout_us(50_000)
     prev_f = fa.fa_debug_set_fault(1)
     try:
-        fa.forward(q, k, v)
+        fa.forward(q, k, v, causal=causal)
         rc = fa.fa_get_device_status(None)
     finally:
         fa.fa_debug_set_fault(prev_f)

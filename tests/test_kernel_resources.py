@@ -50,3 +50,31 @@ def test_contiguous_kernel_resources(tmp_path):
             cur = None
     for d, want in EXPECTED.items():
         assert tuple(found.get(d, ())) == want, (d, found.get(d))
+
+
+@pytest.mark.skipif(not os.path.exists(NVCC) and shutil.which("nvcc") is None, reason="needs nvcc")
+def test_other_kernels_do_not_spill(tmp_path):
+    """The short-key, one-tile, backward, decode and merge kernels keep their
+    working set in registers: ptxas reports no spill stores or loads for any
+    of their instantiations (a spill in their inner loops would show up as a
+    slowdown first and be hard to trace)."""
+    nvcc = NVCC if os.path.exists(NVCC) else shutil.which("nvcc")
+    cmd = [nvcc, "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",
+           "--expt-relaxed-constexpr", "-I", os.path.join(ROOT, "include"),
+           "-I", os.path.join(ROOT, "tiled_attention_13_b200", "csrc"), "-cubin", "-Xptxas", "-v",
+           "-o", str(tmp_path / "all.cubin"), os.path.join(ROOT, "tiled_attention_13_b200", "csrc", "fa_api.cu")]
+    r = subprocess.run(cmd, capture_output=True, text=True, timeout=900)
+    assert r.returncode == 0, r.stderr[-2000:]
+    cur, seen = None, set()
+    for line in r.stderr.splitlines():
+        m = re.search(r"Compiling entry function '(_ZN2fa\w+)'", line)
+        if m:
+            cur = m.group(1)
+            continue
+        m = re.search(r"(\d+) bytes spill stores, (\d+) bytes spill loads", line)
+        if m and cur is not None:
+            if re.search(r"fa_fwd_short|fa_fwd_t1|fa_bwd|fa_decode|splitkv_merge", cur):
+                seen.add(cur)
+                assert (int(m.group(1)), int(m.group(2))) == (0, 0), (cur, line)
+            cur = None
+    assert len(seen) >= 20, sorted(seen)

@@ -105,12 +105,8 @@ bool set_decode_attrs() {
 // Shared-memory attributes of the backward kernels.
 bool set_bwd_attrs() {
   bool ok = true;
-#ifdef FA_TC2
-  ok &= set_smem_attr(fa::fa_fwd_tc2_kernel<64, __nv_bfloat16>, fa::T2Cfg<64>::SMEM_BYTES);
   ok &= set_smem_attr(fa::fa_fwd_tc2_kernel<128, __nv_bfloat16>, fa::T2Cfg<128>::SMEM_BYTES);
-  ok &= set_smem_attr(fa::fa_fwd_tc2_kernel<64, __half>, fa::T2Cfg<64>::SMEM_BYTES);
   ok &= set_smem_attr(fa::fa_fwd_tc2_kernel<128, __half>, fa::T2Cfg<128>::SMEM_BYTES);
-#endif
   ok &= set_decode_attrs<64, __nv_bfloat16>() && set_decode_attrs<128, __nv_bfloat16>();
   ok &= set_decode_attrs<64, __half>() && set_decode_attrs<128, __half>();
   ok &= set_smem_attr(fa::fa_bwd_kernel<64, __nv_bfloat16>, fa::BwdCfg<64>::SMEM_BYTES);
@@ -503,7 +499,8 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
 // or not, grouped K/V heads).
 template <int D, typename T>
 int launch_tc2(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H, int64_t Hkv,
-               int64_t Nq, int64_t Nkv, float scale, int causal, bool bsnd, cudaStream_t stream, DeviceInfo& di) {
+               int64_t Nq, int64_t Nkv, float scale, int causal, bool bsnd, cudaStream_t stream, int num_sms,
+               unsigned int* status, fa::SchedSlot* slot) {
   constexpr bool BF16 = std::is_same<T, __nv_bfloat16>::value;
   CUtensorMap tq, tk, tv;
   if (!make_tmap(&tq, q, BF16, bsnd, B, H, Nq, D) || !make_tmap(&tk, k, BF16, bsnd, B, Hkv, Nkv, D) ||
@@ -526,11 +523,11 @@ int launch_tc2(const void* q, const void* k, const void* v, void* o, float* lse,
   p.block_table = nullptr;
   p.block_size = p.max_blocks = p.num_blocks = 0;
   p.band.pre_tokens = p.band.next_tokens = 0;
-  p.sched = di.sched + (di.launches.fetch_add(1) % kSchedSlots);
+  p.sched = slot;
   p.timeout_ns = (uint64_t)g_timeout_us.load() * 1000ull;
   p.fault_mode = g_fault_mode.load();
-  const int grid = (int)(units < di.num_sms ? units : di.num_sms);
-  fa::fa_fwd_tc2_kernel<D, T><<<grid, fa::T2_THREADS, fa::T2Cfg<D>::SMEM_BYTES, stream>>>(tq, tk, tv, p, di.status);
+  const int grid = (int)(units < num_sms ? units : num_sms);
+  fa::fa_fwd_tc2_kernel<D, T><<<grid, fa::T2_THREADS, fa::T2Cfg<D>::SMEM_BYTES, stream>>>(tq, tk, tv, p, status);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
 }
 
@@ -674,13 +671,14 @@ int fwd_common(const void* q, const void* k, const void* v, void* o, float* lse,
                    : launch_short<128, __half>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s,
                                                di->num_sms, di->status);
   }
-#ifdef FA_TC2
-  if (dtype == FA_DTYPE_BF16)
-    return d == 64 ? launch_tc2<64, __nv_bfloat16>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s, *di)
-                   : launch_tc2<128, __nv_bfloat16>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s, *di);
-  return d == 64 ? launch_tc2<64, __half>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s, *di)
-                 : launch_tc2<128, __half>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s, *di);
-#endif
+  if (d == 128 && !causal) {  // the one-row-per-thread kernel: measured faster without a mask
+    fa::SchedSlot* slot = di->sched + (di->launches.fetch_add(1) % kSchedSlots);
+    return dtype == FA_DTYPE_BF16
+               ? launch_tc2<128, __nv_bfloat16>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s,
+                                                di->num_sms, di->status, slot)
+               : launch_tc2<128, __half>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s, di->num_sms,
+                                         di->status, slot);
+  }
   if (dtype == FA_DTYPE_BF16) {
     return d == 64
                ? launch_tc<64, __nv_bfloat16>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s, *di)
@@ -1044,6 +1042,16 @@ int fa_debug_set_fault(int mode) { return g_fault_mode.exchange(mode); }
 
 int fa_abi_version(void) { return (1 << 16) | 7; }
 
+#ifdef FA_TRACE_SHORT
+int fa_debug_short_trace_read(unsigned long long* host, int n) {
+  const int total = fa::SHT_CTAS * fa::SHT_EV;
+  if (n > total) n = total;
+  if (cudaMemcpyFromSymbol(host, fa::g_trace_short, n * sizeof(unsigned long long)) != cudaSuccess)
+    return FA_ERR_LAUNCH;
+  return n;
+}
+#endif
+
 #ifdef FA_TRACE_UNITS
 int fa_debug_trace_units_read(unsigned long long* host, int n) {
   const int total = 3 * fa::TRU_N * fa::TRU_EV;
@@ -1236,6 +1244,14 @@ extern "C" int fa_fwd_noalloc(const void* q, const void* k, const void* v, void*
                                               nd->status)
                    : launch_short<128, __half>(q, k, v, o, lse, B, H, H, Nq, Nkv, scale, causal, bsnd, s, nd->num_sms,
                                                nd->status);
+  }
+  if (d == 128 && !causal) {  // as fa_fwd: the one-row-per-thread kernel, its counter in slot 0
+    if (cudaMemsetAsync(nd->scratch, 0, sizeof(fa::SchedSlot), s) != cudaSuccess) return FA_ERR_LAUNCH;
+    return dtype == FA_DTYPE_BF16
+               ? launch_tc2<128, __nv_bfloat16>(q, k, v, o, lse, B, H, H, Nq, Nkv, scale, causal, bsnd, s,
+                                                nd->num_sms, nd->status, nd->scratch)
+               : launch_tc2<128, __half>(q, k, v, o, lse, B, H, H, Nq, Nkv, scale, causal, bsnd, s, nd->num_sms,
+                                         nd->status, nd->scratch);
   }
   if (dtype == FA_DTYPE_BF16) {
     return d == 64 ? launch_tc_noalloc<64, __nv_bfloat16>(q, k, v, o, lse, B, H, Nq, Nkv, scale, causal, bsnd, s, *nd)

@@ -37,8 +37,8 @@
 //               then dS^T = P^T o (dP^T - D); P^T and dS^T go back to tensor
 //               memory as 16-bit pairs, dS^T also to shared memory in the
 //               128-byte-swizzled layout; then the thread reads one query row
-//               of dQ and adds it to the accumulator (a bulk reduction of
-//               each 32-column piece, staged through the dS tile).  After the last step it
+//               of dQ and adds it to the accumulator (vector reductions).
+//               After the last step it
 //               writes its key row of dV and scale * dK.
 //
 // TMEM (512 columns): R_S [0, 128), R_DP [128, 256), dV [256, 256 + D),
@@ -52,16 +52,18 @@
 
 #include <type_traits>
 
-#include "fa_fwd_short.cuh"  // sh_mma_ss, sh_mma_ts, sh_tmem_st16, sh_pack2
+#include "tc_common.cuh"
 #include "ptx.cuh"
 
 namespace fa {
 
 #ifndef FA_BWD_BULK_DQ
-#define FA_BWD_BULK_DQ 1
+#define FA_BWD_BULK_DQ 0
 #endif
-// 1: dQ rows reach the accumulator as bulk reductions from shared memory (one
-// per thread and 32 columns); 0: as per-thread 16-byte vector reductions.
+// 0 (default): dQ rows reach the accumulator as per-thread 16-byte vector
+// reductions; 1: as bulk reductions from shared memory (one per thread and 32
+// columns), measured slower on the LLaMA-13B 8K backward (310 against 383
+// TFLOP/s).
 constexpr int BWD_BULK_DQ = FA_BWD_BULK_DQ;
 constexpr int BWD_WARP_MMA = 4;
 constexpr int BWD_WARP_TMA = 5;

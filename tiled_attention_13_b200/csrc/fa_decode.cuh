@@ -35,7 +35,7 @@
 
 #include <type_traits>
 
-#include "fa_fwd_short.cuh"  // sh_pack2
+#include "tc_common.cuh"
 #include "ptx.cuh"
 
 namespace fa {

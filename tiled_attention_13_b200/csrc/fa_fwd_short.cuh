@@ -45,8 +45,24 @@
 #include <type_traits>
 
 #include "ptx.cuh"
+#include "tc_common.cuh"
 
 namespace fa {
+
+// Optional timeline (compile with -DFA_TRACE_SHORT): %globaltimer stamps of
+// a few events of every CTA, readable through fa_debug_short_trace_read().
+#ifdef FA_TRACE_SHORT
+constexpr int SHT_CTAS = 160, SHT_EV = 16;
+__device__ unsigned long long g_trace_short[SHT_CTAS * SHT_EV];
+#define FA_SHT(cond, ev)                                                         \
+  do {                                                                           \
+    if ((cond) && blockIdx.x < SHT_CTAS) g_trace_short[blockIdx.x * SHT_EV + (ev)] = globaltimer_ns(); \
+  } while (0)
+#else
+#define FA_SHT(cond, ev) \
+  do {                   \
+  } while (0)
+#endif
 
 constexpr int SH_WARP_MMA = 8;
 constexpr int SH_WARP_TMA = 9;
@@ -104,78 +120,6 @@ __host__ __device__ __forceinline__ void sh_range(int c, int G, int n_tiles, int
   t1 = (int)(((long long)(c + 1) * n_tiles) / G);
 }
 
-// One MMA, issued by the lane elect.sync picks: D (+)= A * B, A and B from
-// shared-memory descriptors (ss) or A from tensor memory (ts).
-__device__ __forceinline__ void sh_mma_ss(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "l"(a), "l"(b), "r"(idesc), "r"(acc)
-      : "memory");
-}
-__device__ __forceinline__ void sh_mma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64_t b, uint32_t idesc, uint32_t acc) {
-  asm volatile(
-      "{\n\t.reg .pred p, e;\n\t"
-      "elect.sync _|e, 0xffffffff;\n\t"
-      "setp.ne.b32 p, %4, 0;\n\t"
-      "@e tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}" ::"r"(d_tmem),
-      "r"(a_tmem), "l"(b), "r"(idesc), "r"(acc)
-      : "memory");
-}
-
-// 4-D tiled bulk tensor store shared -> global (the tensor map clips rows
-// outside the tensor), then the bulk-group bookkeeping.
-__device__ __forceinline__ void sh_tma_store_4d(const void* tmap, uint32_t src, int c0, int c1, int c2, int c3) {
-  asm volatile("cp.async.bulk.tensor.4d.global.shared::cta.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(tmap),
-               "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
-               : "memory");
-}
-__device__ __forceinline__ void sh_bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void sh_bulk_wait_read0() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
-__device__ __forceinline__ void sh_bulk_wait0() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
-
-// Poll of an mbarrier phase for issue loops that watch several barriers:
-// the waiting thread may be suspended for at most a few tens of nanoseconds
-// (the suspend-time hint), so a barrier that is not ready yet neither holds
-// up the others for long (a plain try_wait may suspend for a
-// system-dependent time) nor lets the poll spin on issue slots the softmax
-// warps of the same sub-partition need.
-__device__ __forceinline__ bool mbar_poll(uint32_t bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(bar), "r"(parity), "r"(40u)
-      : "memory");
-  return ok != 0;
-}
-
-// Store 16 columns (one 32-bit register each) per thread.
-__device__ __forceinline__ void sh_tmem_st16(uint32_t taddr, const uint32_t* r) {
-  asm volatile(
-      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
-      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
-      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]),
-      "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15])
-      : "memory");
-}
-
-template <typename T>
-__device__ __forceinline__ uint32_t sh_pack2(float lo, float hi);
-template <>
-__device__ __forceinline__ uint32_t sh_pack2<__nv_bfloat16>(float lo, float hi) {
-  __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
-template <>
-__device__ __forceinline__ uint32_t sh_pack2<__half>(float lo, float hi) {
-  __half2 v = __floats2half2_rn(lo, hi);
-  return *reinterpret_cast<uint32_t*>(&v);
-}
 
 template <int D, typename T>
 __global__ void __launch_bounds__(SH_THREADS, 1)
@@ -201,6 +145,7 @@ __global__ void __launch_bounds__(SH_THREADS, 1)
   int t0, t1;
   sh_range(blockIdx.x, gridDim.x, p.n_tiles, t0, t1);
   const int n = t1 - t0;  // this CTA's tiles, >= 1
+  FA_SHT(threadIdx.x == 0, 0);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < KQ; ++s) {
@@ -235,6 +180,7 @@ __global__ void __launch_bounds__(SH_THREADS, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   WaitCtx wctx{abort_flag, status_word, p.timeout_ns, 1u};
+  FA_SHT(threadIdx.x == 0, 1);
 
   if (warp == SH_WARP_TMA) {
     // ------------------------------------------------------------ TMA producer
@@ -280,6 +226,7 @@ __global__ void __launch_bounds__(SH_THREADS, 1)
         }
         q_last[s] = i;
       }
+      FA_SHT(true, 11);
       // Every copy this thread started lands before the CTA may exit.
       WaitCtx drain{abort_flag, status_word, p.timeout_ns, 1u};
       volatile int no_abort = 0;
@@ -325,6 +272,8 @@ __global__ void __launch_bounds__(SH_THREADS, 1)
         for (int kk = 0; kk < p.kv_steps; ++kk)
           sh_mma_ts(tO, tS + 8 * kk, dV + (uint64_t)((kk * 2048) >> 4), IDESC_PV, kk > 0 ? 1u : 0u);
         mma_commit_elect(bar(B_OFULL + b));
+        FA_SHT(lane == 0 && jp == 0, 3);
+        FA_SHT(lane == 0 && jp == n - 1, 4);
         // the K/V slot is free once the last tile that reads it is done
         if (jp + 1 == n || sh_decode(t0 + jp + 1, p).kv != x.kv) mma_commit_elect(bar(B_KVEMPTY + slot));
         ++jp;
@@ -349,6 +298,7 @@ __global__ void __launch_bounds__(SH_THREADS, 1)
             sh_mma_ss(tS, dQ + o, dK + o, idesc_s, kk > 0 ? 1u : 0u);
           }
           mma_commit_elect(bar(B_SFULL + (js & 1)));
+          FA_SHT(lane == 0 && js == 0, 2);
           ++js;
           did = true;
         }
@@ -357,7 +307,8 @@ __global__ void __launch_bounds__(SH_THREADS, 1)
         idle_since = 0;
         continue;
       }
-      // nothing was ready: give up on abort or after the wait limit
+      // nothing was ready: back off, and give up on abort or after the wait limit
+      poll_backoff();
       const uint64_t now = globaltimer_ns();
       if (idle_since == 0) idle_since = now;
       const int give_up = __shfl_sync(0xffffffffu, (*abort_flag != 0 || now - idle_since > p.timeout_ns) ? 1 : 0, 0);
@@ -396,6 +347,8 @@ __global__ void __launch_bounds__(SH_THREADS, 1)
       const uint32_t ph = (uint32_t)((i >> 1) & 1);
       ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SFULL + b), ph, wctx));
       if (!ok) break;
+      FA_SHT(storer && i == 0, 5);
+      FA_SHT(storer && i == 1, 10);
       tc_fence_after();
       // Two passes over the tile's S columns in tensor memory (32 at a time,
       // so few registers stay live): the row max, then the exps.  P for keys
@@ -440,9 +393,11 @@ __global__ void __launch_bounds__(SH_THREADS, 1)
       tmem_wait_st();
       tc_fence_before();
       if (p.fault_mode != 1) mbar_arrive_warp(bar(B_PFULL + b));
+      FA_SHT(storer && i == 0, 6);
       // ---------------------------------------------------------- epilogue
       ok = __all_sync(0xffffffffu, mbar_wait(bar(B_OFULL + b), ph, wctx));
       if (!ok) break;
+      FA_SHT(storer && i == 0, 7);
       tc_fence_after();
       const float inv_l = 1.f / l;
       // O / l into the tile's Q stage (its MMAs are done), 128-byte swizzle:
@@ -477,7 +432,9 @@ __global__ void __launch_bounds__(SH_THREADS, 1)
             sh_tma_store_4d(&tm_o, qs + g * C::CHUNK_BYTES, g * 64, row0, x.h, x.b);
         }
         sh_bulk_commit();
+        FA_SHT(i == 0, 8);
         sh_bulk_wait_read0();  // the stage may be refilled once the store has read it
+        FA_SHT(i == 0, 9);
         mbar_arrive(bar(B_QEMPTY + s));
       }
       if (row < p.Nq && p.lse != nullptr &&
@@ -485,6 +442,7 @@ __global__ void __launch_bounds__(SH_THREADS, 1)
         p.lse[((long long)x.b * p.H + x.h) * p.Nq + row] = (m2 + __log2f(l)) * 0.69314718055994530942f;
     }
     if (storer) sh_bulk_wait0();  // this thread's stores are complete before the CTA exits
+    FA_SHT(storer && b == 0, 12);
     tmem_wait_st();
   }
 
@@ -492,6 +450,7 @@ __global__ void __launch_bounds__(SH_THREADS, 1)
   __syncthreads();
   tc_fence_after();
   if (warp == SH_WARP_MMA) tmem_dealloc(tmem, 512);
+  FA_SHT(threadIdx.x == 0, 13);
 }
 
 }  // namespace fa

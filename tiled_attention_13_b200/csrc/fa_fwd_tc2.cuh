@@ -40,7 +40,7 @@
 
 #include <type_traits>
 
-#include "fa_fwd_short.cuh"  // sh_tmem_st16, sh_pack2
+#include "tc_common.cuh"
 #include "fa_fwd_tc.cuh"     // TcParams, Unit, decode_unit, SchedSlot
 #include "ptx.cuh"
 
@@ -51,9 +51,11 @@ constexpr int T2_WARP_MMA = 8;
 constexpr int T2_WARP_TMA = 9;
 constexpr int T2_THREADS = 32 * 10;
 #ifndef FA_T2_POLY_EVERY
-#define FA_T2_POLY_EVERY 0
+#define FA_T2_POLY_EVERY 4
 #endif
-constexpr int T2_POLY_EVERY = FA_T2_POLY_EVERY;  // > 0: one exp pair in T2_POLY_EVERY on the FMA pipe
+// > 0: on steps without masked scores, one exp pair in T2_POLY_EVERY is
+// computed on the FMA pipe (exp2_poly_x2) instead of the SFU; 4 measured best
+constexpr int T2_POLY_EVERY = FA_T2_POLY_EVERY;
 constexpr int T2_POLY_MOD = T2_POLY_EVERY > 0 ? T2_POLY_EVERY : 1;
 
 template <int D>

@@ -48,7 +48,7 @@
 
 #include <type_traits>
 
-#include "fa_fwd_short.cuh"  // sh_mma_ss, sh_mma_ts, sh_tmem_st16, sh_pack2
+#include "tc_common.cuh"
 #include "fa_fwd_tc.cuh"     // SchedSlot
 #include "ptx.cuh"
 
@@ -60,6 +60,17 @@ constexpr int T1_WARP_V = 6;
 constexpr int T1_THREADS = 32 * 7;
 constexpr int T1_MAX_WORDS = 128;  // BLOCK: bit-set words per unit, i.e. at most 4096 key tiles (Nkv <= 524288)
 constexpr float T1_RESCALE_THRESHOLD = 8.0f;  // log2 units
+// d = 256: one exp pair in 4 on the FMA pipe on steps without masked scores
+// (measured 1250 against 1178 TFLOP/s on the 8K d = 256 workload); the
+// block-sparse d <= 128 instantiations measured slightly slower with it.
+// FA_T1_POLY_EVERY overrides the choice for every head dim.
+#ifdef FA_T1_POLY_EVERY
+template <int D>
+constexpr int t1_poly_every() { return FA_T1_POLY_EVERY; }
+#else
+template <int D>
+constexpr int t1_poly_every() { return D == 256 ? 4 : 0; }
+#endif
 
 template <int D>
 struct T1Cfg {
@@ -139,6 +150,8 @@ __global__ void __launch_bounds__(T1_THREADS, 1)
   using C = T1Cfg<D>;
   constexpr bool IS_BF16 = std::is_same<T, __nv_bfloat16>::value;
   constexpr int QST = C::QST, KST = C::KST;
+  constexpr int T1_POLY_EVERY = t1_poly_every<D>();
+  constexpr int T1_POLY_MOD = T1_POLY_EVERY > 0 ? T1_POLY_EVERY : 1;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -432,6 +445,7 @@ __global__ void __launch_bounds__(T1_THREADS, 1)
           idle_since = 0;
           continue;
         }
+        poll_backoff();  // nothing was ready
         const uint64_t now = globaltimer_ns();
         if (idle_since == 0) idle_since = now;
         const int give_up = __shfl_sync(0xffffffffu, (*abort_flag != 0 || now - idle_since > p.timeout_ns) ? 1 : 0, 0);
@@ -512,7 +526,8 @@ __global__ void __launch_bounds__(T1_THREADS, 1)
         for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, *reinterpret_cast<float(*)[32]>(sc + 32 * c));
         const int col0 = kt * 128;
         int lim = p.causal ? (row + 1 < p.Nkv ? row + 1 : p.Nkv) : p.Nkv;
-        if (__any_sync(0xffffffffu, col0 + 127 >= lim)) {
+        const bool masked = __any_sync(0xffffffffu, col0 + 127 >= lim);
+        if (masked) {
 #pragma unroll
           for (int c = 0; c < 128; ++c)
             if (col0 + c >= lim) sc[c] = -INFINITY;
@@ -545,20 +560,35 @@ __global__ void __launch_bounds__(T1_THREADS, 1)
         const float mu = (m_new == -INFINITY) ? 0.f : m_new;
         const uint64_t scale2 = f2_pack(sl2, sl2), negm2 = f2_pack(-mu, -mu);
         uint64_t acc2[2] = {0ull, 0ull};
+        // With T1_POLY_EVERY > 0, on steps without masked scores one exp pair
+        // in T1_POLY_EVERY is computed on the FMA pipe (exp2_poly_x2: masked
+        // scores of -inf must not reach it).
+        auto exps = [&](auto use_poly) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          uint32_t pk[16];
+          for (int c = 0; c < 4; ++c) {
+            uint32_t pk[16];
 #pragma unroll
-          for (int t = 0; t < 16; ++t) {
-            const uint64_t x2 = f2_fma(f2_pack(sc[32 * c + 2 * t], sc[32 * c + 2 * t + 1]), scale2, negm2);
-            float x0, x1;
-            f2_unpack(x2, x0, x1);
-            const float p0 = ex2(x0), p1 = ex2(x1);
-            acc2[t & 1] = f2_add(acc2[t & 1], f2_pack(p0, p1));
-            pk[t] = sh_pack2<T>(p0, p1);
+            for (int t = 0; t < 16; ++t) {
+              const uint64_t x2 = f2_fma(f2_pack(sc[32 * c + 2 * t], sc[32 * c + 2 * t + 1]), scale2, negm2);
+              float p0, p1;
+              if (decltype(use_poly)::value && (t % T1_POLY_MOD) == T1_POLY_MOD - 1) {
+                exp2_poly_x2(x2, p0, p1);
+              } else {
+                float x0, x1;
+                f2_unpack(x2, x0, x1);
+                p0 = ex2(x0);
+                p1 = ex2(x1);
+              }
+              acc2[t & 1] = f2_add(acc2[t & 1], f2_pack(p0, p1));
+              pk[t] = sh_pack2<T>(p0, p1);
+            }
+            sh_tmem_st16(tS + 16 * c, pk);
           }
-          sh_tmem_st16(tS + 16 * c, pk);
-        }
+        };
+        if (T1_POLY_EVERY > 0 && !masked)
+          exps(std::integral_constant<bool, (T1_POLY_EVERY > 0)>{});
+        else
+          exps(std::false_type{});
         {
           float a0, a1;
           f2_unpack(f2_add(acc2[0], acc2[1]), a0, a1);

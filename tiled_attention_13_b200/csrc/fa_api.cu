@@ -102,8 +102,8 @@ bool set_decode_attrs() {
          set_smem_attr(fa::fa_decode_kernel<D, T, 8>, fa::DecCfg<D>::SMEM_BYTES);
 }
 
-// Shared-memory attributes of the backward kernels.
-bool set_bwd_attrs() {
+// Shared-memory attributes of the backward, decode and one-row two-tile kernels.
+bool set_more_attrs() {
   bool ok = true;
   ok &= set_smem_attr(fa::fa_fwd_tc2_kernel<128, __nv_bfloat16>, fa::T2Cfg<128>::SMEM_BYTES);
   ok &= set_smem_attr(fa::fa_fwd_tc2_kernel<128, __half>, fa::T2Cfg<128>::SMEM_BYTES);
@@ -157,7 +157,7 @@ int device_setup(int dev, DeviceInfo** out) {
       ok &= set_smem_attr(fa::fa_fwd_simt_kernel<128>, fa::simt_smem_bytes<128>());
       ok &= set_short_attrs();
       ok &= set_t1_attrs();
-      ok &= set_bwd_attrs();
+      ok &= set_more_attrs();
       if (!ok) return FA_ERR_LAUNCH;
       // The tile scheduler's ticket counters: one slot per launch in flight,
       // each put back to zero by the last CTA of its launch.
@@ -1134,6 +1134,7 @@ int noalloc_setup(int dev, NoAllocDevice** out) {
       ok &= set_smem_attr(fa::fa_fwd_simt_kernel<128>, fa::simt_smem_bytes<128>());
       ok &= set_short_attrs();
       ok &= set_t1_attrs();
+      ok &= set_more_attrs();  // also the one-row two-tile and decode kernels
       if (!ok) return FA_ERR_LAUNCH;
       if (g_encode == nullptr) {
         void* fn = nullptr;

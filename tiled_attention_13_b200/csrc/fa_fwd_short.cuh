@@ -350,26 +350,11 @@ __global__ void __launch_bounds__(SH_THREADS, 1)
       FA_SHT(storer && i == 0, 5);
       FA_SHT(storer && i == 1, 10);
       tc_fence_after();
-      // Two passes over the tile's S columns in tensor memory (32 at a time,
-      // so few registers stay live): the row max, then the exps.  P for keys
-      // [32c, 32c + 32) goes to packed columns [16c, 16c + 16), which pass 2
-      // has already read by then.
       const int lim = p.causal ? (row + 1 < p.Nkv ? row + 1 : p.Nkv) : p.Nkv;  // visible keys [0, lim)
-      float mx = -INFINITY;
-#pragma unroll 1
-      for (int c = 0; c < nc; ++c) {
-        float sc[32];
-        tmem_ld32(tS + 32 * c, sc);
-#pragma unroll
-        for (int t = 0; t < 32; ++t) mx = fmaxf(mx, 32 * c + t < lim ? sc[t] : -INFINITY);
-      }
-      const float m2 = mx * sl2;  // finite: every row sees key 0
-      const uint64_t scale2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m2, -m2);
+      float m2, l;
       uint64_t acc2 = 0ull;
-#pragma unroll 1
-      for (int c = 0; c < nc; ++c) {
-        float sc[32];
-        tmem_ld32(tS + 32 * c, sc);
+      // exps of 32 keys from registers to packed P columns [16c, 16c + 16)
+      auto exps32 = [&](const float* sc, int c, uint64_t scale2, uint64_t negm2) {
         uint32_t pk[16];
 #pragma unroll
         for (int t = 0; t < 16; ++t) {
@@ -383,8 +368,49 @@ __global__ void __launch_bounds__(SH_THREADS, 1)
           pk[t] = sh_pack2<T>(p0, p1);
         }
         sh_tmem_st16(tS + 16 * c, pk);
+      };
+      // Up to 96 keys: one pass, the scores loaded together and kept in
+      // registers.  More: two passes over tensor memory, 32 columns at a time
+      // (the row max, then the exps; P for keys [32c, 32c + 32) goes to packed
+      // columns [16c, 16c + 16), which pass 2 has already read by then).
+      auto one_pass = [&](auto NCc) {
+        constexpr int NC = decltype(NCc)::value;
+        float sc[32 * NC];
+#pragma unroll
+        for (int c = 0; c < NC; ++c) tmem_ld32_nowait(tS + 32 * c, sc + 32 * c);
+        tmem_wait_ld();
+        float mx = -INFINITY;
+#pragma unroll
+        for (int t = 0; t < 32 * NC; ++t) mx = fmaxf(mx, t < lim ? sc[t] : -INFINITY);
+        m2 = mx * sl2;  // finite: every row sees key 0
+        const uint64_t scale2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m2, -m2);
+#pragma unroll
+        for (int c = 0; c < NC; ++c) exps32(sc + 32 * c, c, scale2, negm2);
+      };
+      if (nc == 1) {
+        one_pass(std::integral_constant<int, 1>{});
+      } else if (nc == 2) {
+        one_pass(std::integral_constant<int, 2>{});
+      } else if (nc == 3) {
+        one_pass(std::integral_constant<int, 3>{});
+      } else {
+        float mx = -INFINITY;
+#pragma unroll 1
+        for (int c = 0; c < nc; ++c) {
+          float sc[32];
+          tmem_ld32(tS + 32 * c, sc);
+#pragma unroll
+          for (int t = 0; t < 32; ++t) mx = fmaxf(mx, 32 * c + t < lim ? sc[t] : -INFINITY);
+        }
+        m2 = mx * sl2;
+        const uint64_t scale2 = f2_pack(sl2, sl2), negm2 = f2_pack(-m2, -m2);
+#pragma unroll 1
+        for (int c = 0; c < nc; ++c) {
+          float sc[32];
+          tmem_ld32(tS + 32 * c, sc);
+          exps32(sc, c, scale2, negm2);
+        }
       }
-      float l;
       {
         float a0, a1;
         f2_unpack(acc2, a0, a1);

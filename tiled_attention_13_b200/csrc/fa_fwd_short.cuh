@@ -376,9 +376,12 @@ __global__ void __launch_bounds__(SH_THREADS, 1)
       auto one_pass = [&](auto NCc) {
         constexpr int NC = decltype(NCc)::value;
         float sc[32 * NC];
-#pragma unroll
-        for (int c = 0; c < NC; ++c) tmem_ld32_nowait(tS + 32 * c, sc + 32 * c);
-        tmem_wait_ld();
+        if constexpr (NC == 1)
+          tmem_ld32(tS, *reinterpret_cast<float(*)[32]>(sc));
+        else if constexpr (NC == 2)
+          tmem_ld64(tS, *reinterpret_cast<float(*)[64]>(sc));
+        else
+          tmem_ld96(tS, sc);
         float mx = -INFINITY;
 #pragma unroll
         for (int t = 0; t < 32 * NC; ++t) mx = fmaxf(mx, t < lim ? sc[t] : -INFINITY);

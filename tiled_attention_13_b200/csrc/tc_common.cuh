@@ -81,22 +81,30 @@ __device__ __forceinline__ void poll_backoff() {
 #endif
 }
 
-// Load 32 columns (one 32-bit register each) per thread without waiting;
-// tmem_wait_ld() waits for every load this thread has started.
-__device__ __forceinline__ void tmem_ld32_nowait(uint32_t taddr, float* v) {
+// Load 96 columns (one 32-bit register each) per thread, then wait: one
+// x64 and one x32 load in flight together.
+__device__ __forceinline__ void tmem_ld96(uint32_t taddr, float* v) {
   uint32_t* r = reinterpret_cast<uint32_t*>(v);
 #define FA_R8(b) "=r"(r[b + 0]), "=r"(r[b + 1]), "=r"(r[b + 2]), "=r"(r[b + 3]), "=r"(r[b + 4]), "=r"(r[b + 5]), \
                  "=r"(r[b + 6]), "=r"(r[b + 7])
   asm volatile(
-      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{\n\t.reg .b32 ta;\n\t"
+      "add.u32 ta, %96, 64;\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x64.b32 "
       "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
-      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
-      : FA_R8(0), FA_R8(8), FA_R8(16), FA_R8(24)
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, "
+      "%32, %33, %34, %35, %36, %37, %38, %39, %40, %41, %42, %43, %44, %45, %46, %47, "
+      "%48, %49, %50, %51, %52, %53, %54, %55, %56, %57, %58, %59, %60, %61, %62, %63}, [%96];\n\t"
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%64, %65, %66, %67, %68, %69, %70, %71, %72, %73, %74, %75, %76, %77, %78, %79, "
+      "%80, %81, %82, %83, %84, %85, %86, %87, %88, %89, %90, %91, %92, %93, %94, %95}, [ta];\n\t"
+      "tcgen05.wait::ld.sync.aligned;\n\t}"
+      : FA_R8(0), FA_R8(8), FA_R8(16), FA_R8(24), FA_R8(32), FA_R8(40), FA_R8(48), FA_R8(56), FA_R8(64), FA_R8(72),
+        FA_R8(80), FA_R8(88)
       : "r"(taddr)
       : "memory");
 #undef FA_R8
 }
-__device__ __forceinline__ void tmem_wait_ld() { asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory"); }
 
 // Store 16 columns (one 32-bit register each) per thread.
 __device__ __forceinline__ void sh_tmem_st16(uint32_t taddr, const uint32_t* r) {

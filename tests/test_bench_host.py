@@ -38,7 +38,29 @@ def test_traffic_record_follows_kernel_source():
     else:
         assert t is None
     assert 0.5 < rec["dram_bytes_per_launch"] / rec["algorithmic_bytes_per_launch"] < 2
-    assert bench.captured_traffic("b4-8k") is None  # no record for that workload
+    assert bench.captured_traffic("b4-8k-causal") is None  # no record for that workload
+
+
+def test_every_traffic_record_is_keyed_by_its_sources():
+    """Each committed record names its workload, the kernel's source files
+    (each of which exists) and a hash; the bench reports its traffic only
+    while those files hash to the recorded value."""
+    import glob
+    import hashlib
+
+    csrc = os.path.join(bench.ROOT, "tiled_attention_13_b200", "csrc")
+    recs = sorted(glob.glob(os.path.join(bench.ROOT, "profiles", "*.json")))
+    assert len(recs) >= 7
+    for path in recs:
+        rec = json.load(open(path))
+        assert rec["workload"] in WORKLOADS, path
+        files = rec.get("source_files", ["fa_fwd_tc.cuh", "ptx.cuh"])
+        assert all(os.path.exists(os.path.join(csrc, f)) for f in files), path
+        sha = hashlib.sha256(b"".join(open(os.path.join(csrc, f), "rb").read() for f in files)).hexdigest()
+        t = bench.captured_traffic(rec["workload"])
+        if sha == rec["kernel_source_sha256"]:
+            assert t == float(rec["dram_bytes_per_launch"]), path
+        assert rec["dram_bytes_per_launch"] > 0
 
 
 def test_traffic_record_rejected_when_source_changes(tmp_path, monkeypatch):

@@ -259,8 +259,9 @@ int fa_fwd_paged(const void* q, const void* k_cache, const void* v_cache, const 
  *
  *   num_splits       > 0: that many slices, at most one per key tile;
  *                    <= 0: chosen by the library for num_sms SMs (a wave
- *                    model of its persistent grid: enough units to fill the
- *                    SMs in whole waves, slices no shorter than needed)
+ *                    model of its grid: enough units to fill the SMs in
+ *                    whole waves, slices no shorter than needed; for
+ *                    Nq <= 8 two CTAs per SM, the decoding kernel's)
  *   num_sms          SMs to plan for; <= 0: the current device's (which then
  *                    needs a usable sm_100 device, else FA_ERR_NO_DEVICE)
  *   *splits          out: the slice count the call will use (1 means the call

@@ -8,6 +8,7 @@
 #include <vector>
 
 #include "fa_fwd_short.cuh"
+#include "fa_fwd_short_wg.cuh"
 #include "fa_fwd_tc.cuh"
 
 using fa::TcParams;
@@ -170,11 +171,50 @@ static void check_short(int B, int H, int Hkv, int Nq, int G) {
   for (size_t i = 0; i < seen.size(); ++i) CHECK(seen[i] == 1, "short: tile %zu scheduled %d times", i, seen[i]);
 }
 
+// The four-pipeline short-key kernel: the same contiguous CTA ranges, and
+// warpgroup w of a CTA with n tiles takes tiles w, w + 4, ... (its count
+// `mine`, as the kernel computes it), so the four warpgroups cover the range
+// exactly once; every tile decodes inside the problem.
+static void check_short_wg(int B, int H, int Hkv, int Nq, int G) {
+  fa::SwParams p{};
+  p.B = B; p.H = H; p.Nq = Nq;
+  p.qtiles = cdiv(Nq, 128);
+  p.n_tiles = B * H * p.qtiles;
+  p.kv_group = H / Hkv;
+  if (G > p.n_tiles) G = p.n_tiles;
+  std::vector<int> seen((size_t)p.n_tiles, 0);
+  int expect = 0;
+  for (int c = 0; c < G; ++c) {
+    int t0, t1;
+    fa::sw_range(c, G, p.n_tiles, t0, t1);
+    CHECK(t0 == expect && t1 > t0, "short-wg B%d H%d Nq%d G%d: CTA %d range [%d, %d)", B, H, Nq, G, c, t0, t1);
+    expect = t1;
+    const int n = t1 - t0;
+    for (int wg = 0; wg < fa::SW_WGS; ++wg) {
+      const int mine = n > wg ? (n - wg + fa::SW_WGS - 1) / fa::SW_WGS : 0;
+      for (int j = 0; j < mine; ++j) {
+        const int t = t0 + wg + fa::SW_WGS * j;
+        CHECK(t < t1, "short-wg: warpgroup %d tile %d past its CTA's range", wg, t);
+        const fa::SwTile x = fa::sw_decode(t, p);
+        CHECK(x.b >= 0 && x.b < B && x.h >= 0 && x.h < H && x.qt >= 0 && x.qt < p.qtiles,
+              "short-wg: tile %d decodes outside the problem", t);
+        CHECK(x.kv == x.b * Hkv + x.h / (H / Hkv), "short-wg: tile %d K/V key %d", t, x.kv);
+        if (t >= 0 && t < p.n_tiles) seen[(size_t)t]++;
+      }
+    }
+  }
+  CHECK(expect == p.n_tiles, "short-wg B%d H%d Nq%d G%d: ranges end at %d", B, H, Nq, G, expect);
+  for (size_t i = 0; i < seen.size(); ++i) CHECK(seen[i] == 1, "short-wg: tile %zu scheduled %d times", i, seen[i]);
+}
+
 int main() {
   const int short_shapes[][4] = {{1, 1, 1, 1}, {2, 8, 8, 4096}, {4, 32, 32, 4096}, {5, 200, 100, 100},
                                  {1, 8, 2, 2000}, {3, 7, 7, 129}};
   for (const auto& s : short_shapes)
-    for (int G : {1, 7, 148, 1 << 20}) check_short(s[0], s[1], s[2], s[3], G);
+    for (int G : {1, 7, 148, 1 << 20}) {
+      check_short(s[0], s[1], s[2], s[3], G);
+      check_short_wg(s[0], s[1], s[2], s[3], G);
+    }
 
   const int shapes[][4] = {{1, 1, 1, 1}, {1, 2, 300, 333}, {2, 3, 129, 127}, {1, 40, 1024, 1024},
                            {2, 5, 777, 2000}, {3, 7, 4096, 77}, {1, 1, 8192, 8192}};

@@ -172,10 +172,12 @@ def _plan_cost(base, nt, s, sms):
 def test_splitkv_plan_follows_its_wave_model(fa_lib, B, H, Nq, Nkv):
     """fa_splitkv_plan with an explicit SM count (no GPU needed): the chosen
     slice count has the least modelled cost of every count up to about four
-    units per SM, no slice is empty, and the workspace is splits * B*H*Nq *
-    (d + 1) fp32 values (none for one slice)."""
-    sms, d = 148, 128
-    S, nbytes = fa.splitkv_plan(B, H, Nq, Nkv, d, 0, sms)
+    units per CTA slot (two slots per SM for Nq <= 8, where the decoding
+    kernel runs two CTAs on an SM), no slice is empty, and the workspace is
+    splits * B*H*Nq * (d + 1) fp32 values (none for one slice)."""
+    d = 128
+    S, nbytes = fa.splitkv_plan(B, H, Nq, Nkv, d, 0, 148)
+    sms = 2 * 148 if Nq <= 8 else 148
     nt = -(-Nkv // 128)
     base = B * H * (-(-(-(-Nq // 128)) // 2))
     smax = min(nt, -(-4 * sms // base), 4096)

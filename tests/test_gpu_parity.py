@@ -449,6 +449,26 @@ def test_paged_splitkv(block_size, num_splits):
         _paged_parity(wl, num_splits=num_splits)
 
 
+PAGED_DECODE_CASES = [  # (B, H, Hkv, Nq, Nkv, d, layout, dtype, block_size, num_splits)
+    (3, 4, 4, 1, 1000, 64, "BHND", "bf16", 32, 0),      # d = 64, q and O in BHND
+    (1, 8, 1, 1, 70000, 128, "BSND", "fp16", 16, 2),    # multi-query, long slices: table read in many batches
+    (2, 6, 3, 4, 2049, 128, "BSND", "bf16", 256, 0),    # 8 rows per K/V head, large blocks, ragged tail
+    (1, 2, 2, 1, 17, 64, "BSND", "bf16", 16, 1),        # one slice: O written directly
+]
+
+
+@pytest.mark.parametrize("case", PAGED_DECODE_CASES,
+                         ids=lambda c: "x".join(map(str, c[:6])) + c[6] + c[7] + f"bs{c[8]}s{c[9]}")
+def test_paged_decode_kernel(case):
+    """Decoding-shaped paged split-KV calls (at most 8 query rows per K/V
+    head) run on the CUDA-core decode kernel, which reads each 16-key chunk
+    through the block table; against the oracle's gather-then-attend."""
+    B, H, hkv, nq, nkv, d, layout, dtype, bs, S = case
+    wl = Workload("decode-paged", B=B, H=H, Hkv=hkv, Nq=nq, Nkv=nkv, d=d, dtype=dtype, layout=layout, causal=False,
+                  seed=nkv + bs + S, block_size=bs)
+    _paged_parity(wl, num_splits=S)
+
+
 def test_splitkv_rejects_a_short_workspace():
     """The workspace is checked against the plan before anything is launched."""
     B, H, nq, nkv, d = 1, 4, 1, 4096, 128
@@ -483,6 +503,11 @@ SHORT_CASES = [  # (B, H, Hkv, Nq, Nkv, d, layout, causal, dtype)
     (1, 4, 4, 90, 128, 128, "BSND", False, "fp16"),
     (2, 8, 8, 1024, 77, 64, "BHND", False, "bf16"),
     (1, 8, 2, 2000, 77, 128, "BSND", False, "bf16"),
+    (1, 4, 1, 700, 97, 64, "BHND", True, "bf16"),
+    (3, 2, 2, 384, 80, 64, "BSND", False, "fp16"),
+    (1, 2, 2, 77, 77, 64, "BHND", True, "bf16"),
+    (1, 6, 3, 130, 112, 64, "BSND", False, "bf16"),
+    (1, 1, 1, 5000, 48, 64, "BHND", True, "fp16"),
 ]
 
 
@@ -506,11 +531,41 @@ def test_short_keys_many_tiles_per_cta_and_head_switches(d):
     compare_sampled(wl, [(0, 0), (4, 199), (2, 101), (3, 50), (1, 1)], rows_per_head=20)
 
 
-def test_short_keys_bounded_wait_expires_and_context_survives():
-    """The failure hook on the short-key kernel: P is never signalled, the MMA
-    warp's bounded wait expires, every role leaves its loop and the status
-    word reads FA_ERR_TIMEOUT; the next normal call is correct."""
-    wl = Workload("short-fault", B=2, H=8, Nq=1024, Nkv=77, d=64, dtype="bf16", layout="BHND", causal=False, seed=4)
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+@pytest.mark.parametrize("causal", [False, True])
+def test_short_keys_reference_max_raised(causal, dtype):
+    """The d = 64 short-key kernel takes its reference max from a row's first
+    32 keys and raises it when a later 32-key chunk's max passes it by more
+    than 2^8, rescaling the P already written.  Keys whose scale grows chunk by
+    chunk (x0.1, x1, x4, x8) make that happen two or three times in most
+    rows; the result must still be the softmax of the scores.  Bound as for
+    page 1's regression inputs: half an output ulp, 2^-9 max|V| for rounding
+    P to 16 bits, 1e-3 for the fp32 accumulation."""
+    from oracle import attention_batched
+
+    tdt = torch.bfloat16 if dtype == "bf16" else torch.float16
+    g = torch.Generator().manual_seed(31)
+    B, H, Nq, Nkv, d = 1, 2, 300, 120, 64
+    q = torch.randn(B, H, Nq, d, generator=g)
+    k = torch.randn(B, H, Nkv, d, generator=g)
+    k *= torch.tensor([0.1] * 32 + [1.0] * 32 + [4.0] * 32 + [8.0] * 24).view(1, 1, -1, 1)
+    v = torch.randn(B, H, Nkv, d, generator=g)
+    q, k, v = (t.to(tdt) for t in (q, k, v))
+    o, lse = fa.forward(q.cuda(), k.cuda(), v.cuda(), causal=causal)
+    o_ref, l_ref = attention_batched(q, k, v, causal=causal)
+    err = np.abs(o.double().cpu().numpy() - o_ref)
+    bar = half_ulp(o_ref, dtype) + 2.0 ** -9 * float(v.float().abs().max()) + 1e-3
+    assert np.all(err <= bar), err.max()
+    assert np.abs(lse.double().cpu().numpy() - l_ref).max() <= 1e-3
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_short_keys_bounded_wait_expires_and_context_survives(d):
+    """The failure hook on the short-key kernels (d = 64: four tile pipelines
+    per CTA; d = 128: two warpgroups): P is never signalled, the MMA issuer's
+    bounded wait expires, every role leaves its loop and the status word
+    reads FA_ERR_TIMEOUT; the next normal call is correct."""
+    wl = Workload("short-fault", B=2, H=8, Nq=1024, Nkv=77, d=d, dtype="bf16", layout="BHND", causal=False, seed=4)
     q, k, v = (t.cuda() for t in make_qkv(wl))
     assert fa.fa_get_device_status(None) == 0
     prev_t = fa.fa_set_wait_timeout_us(50_000)

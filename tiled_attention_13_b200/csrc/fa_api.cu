@@ -13,8 +13,15 @@
 #include <cstdint>
 #include <mutex>
 #include <type_traits>
+#include <utility>
 
 #include "fa.h"
+
+// Head dim 64 with at most 128 keys on the four-pipeline short-key kernel
+// (0: on the two-warpgroup one, for comparison).
+#ifndef FA_SHORT_WG
+#define FA_SHORT_WG 1
+#endif
 
 namespace fa {
 // Bit 0: a bounded wait expired.  Written by kernels, read and cleared by
@@ -23,6 +30,7 @@ __device__ unsigned int g_status_word = 0;
 }  // namespace fa
 
 #include "fa_fwd_short.cuh"
+#include "fa_fwd_short_wg.cuh"
 #include "fa_fwd_simt.cuh"
 #include "fa_fwd_tc.cuh"
 #include "fa_fwd_tile1.cuh"
@@ -56,6 +64,28 @@ using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t
                                    CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
 EncodeTiledFn g_encode = nullptr;
 
+// Launch with programmatic stream serialization (FA_PDL != 0): the kernel
+// may start while the previous kernel of the stream drains, and waits for it
+// (griddepcontrol.wait) before touching global data.
+#ifndef FA_PDL
+#define FA_PDL 1
+#endif
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kernel)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = FA_PDL ? 1 : 0;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args>(args)...);
+}
+
 template <typename K>
 bool set_smem_attr(K kernel, int bytes) {
   return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) == cudaSuccess;
@@ -68,6 +98,8 @@ bool set_short_attrs() {
   ok &= set_smem_attr(fa::fa_fwd_short_kernel<128, __nv_bfloat16>, fa::ShCfg<128>::SMEM_BYTES);
   ok &= set_smem_attr(fa::fa_fwd_short_kernel<64, __half>, fa::ShCfg<64>::SMEM_BYTES);
   ok &= set_smem_attr(fa::fa_fwd_short_kernel<128, __half>, fa::ShCfg<128>::SMEM_BYTES);
+  ok &= set_smem_attr(fa::fa_fwd_short_wg_kernel<__nv_bfloat16>, fa::SW_SMEM_MAX);
+  ok &= set_smem_attr(fa::fa_fwd_short_wg_kernel<__half>, fa::SW_SMEM_MAX);
   return ok;
 }
 
@@ -94,12 +126,16 @@ bool set_t1_attrs() {
 }
 
 // Shared-memory attributes of the decode kernels (every row count).
+template <int D, typename T, bool PAGED>
+bool set_decode_attrs_p() {
+  return set_smem_attr(fa::fa_decode_kernel<D, T, 1, PAGED>, fa::DecCfg<D>::SMEM_BYTES) &&
+         set_smem_attr(fa::fa_decode_kernel<D, T, 2, PAGED>, fa::DecCfg<D>::SMEM_BYTES) &&
+         set_smem_attr(fa::fa_decode_kernel<D, T, 4, PAGED>, fa::DecCfg<D>::SMEM_BYTES) &&
+         set_smem_attr(fa::fa_decode_kernel<D, T, 8, PAGED>, fa::DecCfg<D>::SMEM_BYTES);
+}
 template <int D, typename T>
 bool set_decode_attrs() {
-  return set_smem_attr(fa::fa_decode_kernel<D, T, 1>, fa::DecCfg<D>::SMEM_BYTES) &&
-         set_smem_attr(fa::fa_decode_kernel<D, T, 2>, fa::DecCfg<D>::SMEM_BYTES) &&
-         set_smem_attr(fa::fa_decode_kernel<D, T, 4>, fa::DecCfg<D>::SMEM_BYTES) &&
-         set_smem_attr(fa::fa_decode_kernel<D, T, 8>, fa::DecCfg<D>::SMEM_BYTES);
+  return set_decode_attrs_p<D, T, false>() && set_decode_attrs_p<D, T, true>();
 }
 
 // Shared-memory attributes of the backward, decode and one-row two-tile kernels.
@@ -214,11 +250,11 @@ bool make_tmap(CUtensorMap* tm, const void* base, bool bf16, bool bsnd, int64_t 
 // min(block_size, 128) rows of one (block, head), 128-byte swizzle, reads
 // outside the cache (e.g. block index num_blocks) fill with zeros.
 bool make_tmap_paged(CUtensorMap* tm, const void* base, bool bf16, int64_t Hkv, int64_t bs, int64_t num_blocks,
-                     int64_t D) {
+                     int64_t D, int64_t box_rows = 128) {
   const cuuint64_t es = 2;
   cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)Hkv, (cuuint64_t)bs, (cuuint64_t)num_blocks};
   cuuint64_t strides[3] = {D * es, Hkv * D * es, bs * Hkv * D * es};
-  cuuint32_t box[4] = {64, 1, (cuuint32_t)(bs < 128 ? bs : 128), 1}, estr[4] = {1, 1, 1, 1};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)(bs < box_rows ? bs : box_rows), 1}, estr[4] = {1, 1, 1, 1};
   CUresult r = g_encode(tm, bf16 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_FLOAT16, 4,
                         const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                         CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -254,6 +290,13 @@ struct SplitKV {
 // standing for a unit's fixed cost (its Q load, the pipeline's fill and the
 // epilogue); the first count with the lowest cost wins, trying up to about
 // four units per SM.
+// CTAs that run at once, for the split plan: decoding-shaped calls (Nq <= 8
+// rows; at most 8 rows per K/V head go to the CUDA-core decode kernel, which
+// fits two CTAs on an SM) count two per SM, others one.
+int64_t plan_slots(int64_t Nq, int num_sms) {
+  return Nq <= fa::DEC_ROWS ? (int64_t)fa::DEC_CTAS_PER_SM * num_sms : (int64_t)num_sms;
+}
+
 void split_plan(int64_t base_units, int64_t kv_tiles, int requested, int num_sms, int* n_splits,
                 int* split_tiles) {
   int64_t S = 1;
@@ -358,9 +401,10 @@ int launch_tc(const void* q, const void* k, const void* v, void* o, float* lse, 
   if (sk != nullptr) {  // combine the slices into O and LSE, in stream order
     const int64_t rows = B * H * Nq;
     const int64_t blocks = (rows + fa::MERGE_ROWS_PER_CTA - 1) / fa::MERGE_ROWS_PER_CTA;
-    fa::fa_splitkv_merge_kernel<D, T><<<(unsigned int)blocks, fa::MERGE_THREADS, 0, stream>>>(
-        sk->o_part, sk->lse_part, static_cast<T*>(o), lse, (int)B, (int)H, (int)Nq, sk->n_splits, bsnd ? 1 : 0);
-    if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+    if (launch_pdl(fa::fa_splitkv_merge_kernel<D, T>, dim3((unsigned int)blocks), dim3(fa::MERGE_THREADS), 0, stream,
+                   (const float*)sk->o_part, (const float*)sk->lse_part, static_cast<T*>(o), lse, (int)B, (int)H,
+                   (int)Nq, sk->n_splits, bsnd ? 1 : 0) != cudaSuccess)
+      return FA_ERR_LAUNCH;
   }
   return FA_OK;
 }
@@ -368,11 +412,49 @@ int launch_tc(const void* q, const void* k, const void* v, void* o, float* lse, 
 // Keys fit one KV tile (Nkv <= 128): the short-key kernel, one pass of
 // softmax per query tile, a static schedule and no work counter.  Plain
 // (contiguous, causal or not, grouped or not) bf16/fp16 calls.
+// The short-key kernel with four query-tile pipelines per CTA (head dim 64).
+// K / V tensor maps load n_s = Nkv rounded up to 16 rows; two Q stages per
+// pipeline when they fit in shared memory, else one.
+template <typename T>
+int launch_short_wg(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
+                    int64_t Hkv, int64_t Nq, int64_t Nkv, float scale, int causal, bool bsnd, cudaStream_t stream,
+                    int num_sms, unsigned int* status) {
+  constexpr bool BF16 = std::is_same<T, __nv_bfloat16>::value;
+  const int n_s = (int)((Nkv + 15) / 16) * 16;
+  CUtensorMap tq, tk, tv, to;
+  if (!make_tmap(&tq, q, BF16, bsnd, B, H, Nq, 64) || !make_tmap(&tk, k, BF16, bsnd, B, Hkv, Nkv, 64, n_s) ||
+      !make_tmap(&tv, v, BF16, bsnd, B, Hkv, Nkv, 64, n_s) || !make_tmap(&to, o, BF16, bsnd, B, H, Nq, 64))
+    return FA_ERR_LAUNCH;
+  fa::SwParams p;
+  p.lse = lse;
+  p.B = (int)B; p.H = (int)H; p.Nq = (int)Nq; p.Nkv = (int)Nkv;
+  p.bsnd = bsnd ? 1 : 0;
+  p.causal = causal;
+  p.scale_log2 = scale * 1.4426950408889634f;
+  p.qtiles = (int)((Nq + 127) / 128);
+  const int64_t tiles = B * H * (int64_t)p.qtiles;
+  if (tiles > INT32_MAX) return FA_ERR_UNSUPPORTED;
+  p.n_tiles = (int)tiles;
+  p.kv_group = (int)(H / Hkv);
+  p.n_s = n_s;
+  p.ns = fa::sw_smem_bytes(n_s, 2) <= fa::SW_SMEM_MAX ? 2 : 1;
+  p.timeout_ns = (uint64_t)g_timeout_us.load() * 1000ull;
+  p.fault_mode = g_fault_mode.load();
+  const int grid = (int)(tiles < num_sms ? tiles : num_sms);
+  const cudaError_t e = launch_pdl(fa::fa_fwd_short_wg_kernel<T>, dim3(grid), dim3(fa::SW_THREADS),
+                                   (size_t)fa::sw_smem_bytes(n_s, p.ns), stream, tq, tk, tv, to, p, status);
+  return e == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
+}
+
 template <int D, typename T>
 int launch_short(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
                  int64_t Hkv, int64_t Nq, int64_t Nkv, float scale, int causal, bool bsnd, cudaStream_t stream,
                  int num_sms, unsigned int* status) {
   constexpr bool BF16 = std::is_same<T, __nv_bfloat16>::value;
+#if FA_SHORT_WG
+  if constexpr (D == 64)  // four tile pipelines per CTA
+    return launch_short_wg<T>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, stream, num_sms, status);
+#endif
   CUtensorMap tq, tk, tv, to;
   if (!make_tmap(&tq, q, BF16, bsnd, B, H, Nq, D) || !make_tmap(&tk, k, BF16, bsnd, B, Hkv, Nkv, D) ||
       !make_tmap(&tv, v, BF16, bsnd, B, Hkv, Nkv, D) || !make_tmap(&to, o, BF16, bsnd, B, H, Nq, D))
@@ -537,13 +619,23 @@ int launch_tc2(const void* q, const void* k, const void* v, void* o, float* lse,
 template <int D, typename T>
 int launch_decode(const void* q, const void* k, const void* v, void* o, float* lse, int64_t B, int64_t H,
                   int64_t Hkv, int64_t Nq, int64_t Nkv, float scale, bool bsnd, cudaStream_t stream,
-                  unsigned int* status, const SplitKV* sk) {
+                  unsigned int* status, const SplitKV* sk, const PagedKV* pg) {
   constexpr bool BF16 = std::is_same<T, __nv_bfloat16>::value;
   CUtensorMap tk, tv;
-  if (!make_tmap(&tk, k, BF16, bsnd, B, Hkv, Nkv, D, fa::DEC_CHUNK) ||
-      !make_tmap(&tv, v, BF16, bsnd, B, Hkv, Nkv, D, fa::DEC_CHUNK))
+  if (pg != nullptr) {
+    if (!make_tmap_paged(&tk, k, BF16, Hkv, pg->block_size, pg->num_blocks, D, fa::DEC_CHUNK) ||
+        !make_tmap_paged(&tv, v, BF16, Hkv, pg->block_size, pg->num_blocks, D, fa::DEC_CHUNK))
+      return FA_ERR_LAUNCH;
+  } else if (!make_tmap(&tk, k, BF16, bsnd, B, Hkv, Nkv, D, fa::DEC_CHUNK) ||
+             !make_tmap(&tv, v, BF16, bsnd, B, Hkv, Nkv, D, fa::DEC_CHUNK)) {
     return FA_ERR_LAUNCH;
+  }
   fa::DecParams p;
+  p.block_table = pg != nullptr ? pg->block_table : nullptr;
+  p.max_blocks = pg != nullptr ? (int)pg->max_blocks : 0;
+  p.bs_log2 = 0;
+  if (pg != nullptr)
+    while ((int64_t(1) << p.bs_log2) < pg->block_size) ++p.bs_log2;
   p.q = q;
   p.o = sk != nullptr ? static_cast<void*>(sk->o_part) : o;
   p.lse = sk != nullptr ? sk->lse_part : lse;
@@ -558,21 +650,23 @@ int launch_decode(const void* q, const void* k, const void* v, void* o, float* l
   const int64_t R = Nq * (H / Hkv);  // rows per (batch, K/V head), at most fa::DEC_ROWS
   const dim3 grid((unsigned int)ctas);
   const int sm = fa::DecCfg<D>::SMEM_BYTES;
-  if (R <= 1)
-    fa::fa_decode_kernel<D, T, 1><<<grid, fa::DEC_THREADS, sm, stream>>>(tk, tv, p, status);
-  else if (R <= 2)
-    fa::fa_decode_kernel<D, T, 2><<<grid, fa::DEC_THREADS, sm, stream>>>(tk, tv, p, status);
-  else if (R <= 4)
-    fa::fa_decode_kernel<D, T, 4><<<grid, fa::DEC_THREADS, sm, stream>>>(tk, tv, p, status);
-  else
-    fa::fa_decode_kernel<D, T, 8><<<grid, fa::DEC_THREADS, sm, stream>>>(tk, tv, p, status);
-  if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+  auto kern = pg != nullptr ? (R <= 1   ? fa::fa_decode_kernel<D, T, 1, true>
+                               : R <= 2 ? fa::fa_decode_kernel<D, T, 2, true>
+                               : R <= 4 ? fa::fa_decode_kernel<D, T, 4, true>
+                                        : fa::fa_decode_kernel<D, T, 8, true>)
+                            : (R <= 1   ? fa::fa_decode_kernel<D, T, 1, false>
+                               : R <= 2 ? fa::fa_decode_kernel<D, T, 2, false>
+                               : R <= 4 ? fa::fa_decode_kernel<D, T, 4, false>
+                                        : fa::fa_decode_kernel<D, T, 8, false>);
+  if (launch_pdl(kern, grid, dim3(fa::DEC_THREADS), (size_t)sm, stream, tk, tv, p, status) != cudaSuccess)
+    return FA_ERR_LAUNCH;
   if (sk != nullptr) {
     const int64_t rows = B * H * Nq;
     const int64_t blocks = (rows + fa::MERGE_ROWS_PER_CTA - 1) / fa::MERGE_ROWS_PER_CTA;
-    fa::fa_splitkv_merge_kernel<D, T><<<(unsigned int)blocks, fa::MERGE_THREADS, 0, stream>>>(
-        sk->o_part, sk->lse_part, static_cast<T*>(o), lse, (int)B, (int)H, (int)Nq, sk->n_splits, bsnd ? 1 : 0);
-    if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
+    if (launch_pdl(fa::fa_splitkv_merge_kernel<D, T>, dim3((unsigned int)blocks), dim3(fa::MERGE_THREADS), 0, stream,
+                   (const float*)sk->o_part, (const float*)sk->lse_part, static_cast<T*>(o), lse, (int)B, (int)H,
+                   (int)Nq, sk->n_splits, bsnd ? 1 : 0) != cudaSuccess)
+      return FA_ERR_LAUNCH;
   }
   return FA_OK;
 }
@@ -731,7 +825,8 @@ int splitkv_common(const void* q, const void* k, const void* v, const PagedKV* p
   if (st != FA_OK) return st;
   const int64_t qtiles = (Nq + fa::TC_BM - 1) / fa::TC_BM;
   int S = 1, tiles = 0;
-  split_plan(B * H * ((qtiles + 1) / 2), (Nkv + fa::TC_BN - 1) / fa::TC_BN, num_splits, di->num_sms, &S, &tiles);
+  split_plan(B * H * ((qtiles + 1) / 2), (Nkv + fa::TC_BN - 1) / fa::TC_BN, num_splits,
+             (int)plan_slots(Nq, di->num_sms), &S, &tiles);
   const int64_t need = split_workspace_bytes(B, H, Nq, d, S);
   if (need > 0) {
     if (workspace == nullptr || workspace_bytes < need) return FA_ERR_INVALID_ARG;
@@ -743,14 +838,16 @@ int splitkv_common(const void* q, const void* k, const void* v, const PagedKV* p
   const SplitKV* skp = S > 1 ? &sk : nullptr;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool bsnd = layout == FA_LAYOUT_BSND;
-  if (pg == nullptr && Nq * (H / Hkv) <= fa::DEC_ROWS) {  // decoding-shaped: the CUDA-core kernel
+  if (Nq * (H / Hkv) <= fa::DEC_ROWS) {  // decoding-shaped: the CUDA-core kernel, contiguous or paged
     if (dtype == FA_DTYPE_BF16)
       return d == 64 ? launch_decode<64, __nv_bfloat16>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, bsnd, s,
-                                                        di->status, skp)
+                                                        di->status, skp, pg)
                      : launch_decode<128, __nv_bfloat16>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, bsnd, s,
-                                                         di->status, skp);
-    return d == 64 ? launch_decode<64, __half>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, bsnd, s, di->status, skp)
-                   : launch_decode<128, __half>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, bsnd, s, di->status, skp);
+                                                         di->status, skp, pg);
+    return d == 64 ? launch_decode<64, __half>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, bsnd, s, di->status, skp,
+                                               pg)
+                   : launch_decode<128, __half>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, bsnd, s, di->status, skp,
+                                                pg);
   }
   if (dtype == FA_DTYPE_BF16)
     return d == 64 ? launch_tc<64, __nv_bfloat16>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, 0, bsnd, s, *di, pg,
@@ -987,7 +1084,8 @@ int fa_splitkv_plan(int64_t B, int64_t H, int64_t Nq, int64_t Nkv, int64_t d, in
   int S = 1, tiles = 0;
   if (B > 0 && H > 0 && Nq > 0 && Nkv > 0) {
     const int64_t qtiles = (Nq + fa::TC_BM - 1) / fa::TC_BM;
-    split_plan(B * H * ((qtiles + 1) / 2), (Nkv + fa::TC_BN - 1) / fa::TC_BN, num_splits, num_sms, &S, &tiles);
+    split_plan(B * H * ((qtiles + 1) / 2), (Nkv + fa::TC_BN - 1) / fa::TC_BN, num_splits,
+               (int)plan_slots(Nq, num_sms), &S, &tiles);
   }
   *splits = S;
   *workspace_bytes = split_workspace_bytes(B, H, Nq, d, S);
@@ -1043,12 +1141,13 @@ int fa_debug_set_fault(int mode) { return g_fault_mode.exchange(mode); }
 int fa_abi_version(void) { return (1 << 16) | 7; }
 
 #ifdef FA_TRACE_SHORT
-int fa_debug_short_trace_read(unsigned long long* host, int n) {
-  const int total = fa::SHT_CTAS * fa::SHT_EV;
+// which = 0: the two-warpgroup short-key kernel's timeline, 1: the four-pipeline one's
+int fa_debug_short_trace_read(unsigned long long* host, int n, int which) {
+  const int total = which ? fa::SWT_CTAS * fa::SWT_EV : fa::SHT_CTAS * fa::SHT_EV;
   if (n > total) n = total;
-  if (cudaMemcpyFromSymbol(host, fa::g_trace_short, n * sizeof(unsigned long long)) != cudaSuccess)
-    return FA_ERR_LAUNCH;
-  return n;
+  const cudaError_t e = which ? cudaMemcpyFromSymbol(host, fa::g_trace_short_wg, n * sizeof(unsigned long long))
+                              : cudaMemcpyFromSymbol(host, fa::g_trace_short, n * sizeof(unsigned long long));
+  return e == cudaSuccess ? n : FA_ERR_LAUNCH;
 }
 #endif
 

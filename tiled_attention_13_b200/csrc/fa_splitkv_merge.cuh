@@ -59,6 +59,9 @@ __global__ void __launch_bounds__(MERGE_THREADS)
     fa_splitkv_merge_kernel(const float* __restrict__ o_part, const float* __restrict__ lse_part, T* __restrict__ o,
                             float* __restrict__ lse, int B, int H, int Nq, int n_splits, int bsnd) {
   constexpr int E = D / 32;  // 4 (d = 128) or 2 (d = 64)
+  // a dependent launch: the partial results are read once the split kernel has completed
+  pdl_launch_dependents();
+  pdl_wait();
   const long long rows = (long long)B * H * Nq;
   const long long r = (long long)blockIdx.x * MERGE_ROWS_PER_CTA + (threadIdx.x >> 5);
   if (r >= rows) return;

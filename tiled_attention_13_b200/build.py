@@ -23,7 +23,7 @@ LIB_NAME = "libfa_b200.so"
 LIB_PATH = os.path.join(PKG, LIB_NAME)
 
 SOURCES = ["fa_api.cu"]
-DEPS = ["fa_api.cu", "tc_common.cuh", "fa_fwd_tc2.cuh", "fa_decode.cuh", "fa_bwd.cuh", "fa_fwd_tile1.cuh", "fa_fwd_short.cuh", "fa_fwd_short_wg.cuh", "fa_fwd_tc.cuh", "fa_fwd_simt.cuh", "fa_splitkv_merge.cuh", "ptx.cuh"]
+DEPS = ["fa_api.cu", "tc_common.cuh", "fa_fwd_tc2.cuh", "fa_decode.cuh", "fa_bwd.cuh", "fa_fwd_tile1.cuh", "fa_fwd_short.cuh", "fa_fwd_short_wg.cuh", "fa_fwd_tc.cuh", "fa_fwd_simt.cuh", "fa_splitkv_merge.cuh", "pdl.cuh", "ptx.cuh"]
 
 NVCC_FLAGS = [
     "-gencode", "arch=compute_100a,code=sm_100a",

@@ -40,6 +40,7 @@
 #include <type_traits>
 
 #include "tc_common.cuh"
+#include "pdl.cuh"
 #include "ptx.cuh"
 
 namespace fa {

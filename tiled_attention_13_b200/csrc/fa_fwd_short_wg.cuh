@@ -38,6 +38,7 @@
 
 #include <type_traits>
 
+#include "pdl.cuh"
 #include "ptx.cuh"
 #include "tc_common.cuh"
 

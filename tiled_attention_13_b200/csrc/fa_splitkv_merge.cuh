@@ -19,6 +19,7 @@
 
 #include <cstdint>
 
+#include "pdl.cuh"
 #include "ptx.cuh"  // FA_INDEX_OK
 
 namespace fa {

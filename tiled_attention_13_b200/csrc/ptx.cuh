@@ -297,16 +297,6 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const uint32_t (&r)[8])
 
 __device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
 
-// ---------------------------------------------------------------- dependent launches
-// A kernel launched with programmatic stream serialization may start while
-// the previous kernel in the stream is still running.  pdl_wait() blocks
-// until that kernel has completed and its writes are visible; every thread
-// calls it before its first global access of data another kernel may touch.
-// pdl_launch_dependents() lets the next such kernel launch early (its CTAs
-// take SMs as this grid's CTAs exit and wait in pdl_wait()).
-__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
-__device__ __forceinline__ void pdl_launch_dependents() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
-
 // ---------------------------------------------------------------- sm_100 ALU forms
 // max of three floats in one instruction.
 __device__ __forceinline__ float fmax3(float a, float b, float c) {

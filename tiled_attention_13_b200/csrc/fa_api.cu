@@ -543,11 +543,20 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
                void* dq, void* dk, void* dv, void* ws, int64_t B, int64_t H, int64_t Hkv, int64_t Nq, int64_t Nkv,
                float scale, int causal, bool bsnd, cudaStream_t stream, unsigned int* status) {
   constexpr bool BF16 = std::is_same<T, __nv_bfloat16>::value;
-  CUtensorMap tq, tk, tv, tdo;
+  CUtensorMap tq, tk, tv, tdo, tdq;
   if (!make_tmap(&tq, q, BF16, bsnd, B, H, Nq, D) || !make_tmap(&tk, k, BF16, bsnd, B, Hkv, Nkv, D) ||
       !make_tmap(&tv, v, BF16, bsnd, B, Hkv, Nkv, D) || !make_tmap(&tdo, dout, BF16, bsnd, B, H, Nq, D))
     return FA_ERR_LAUNCH;
   const BwdLayout L = bwd_layout(B, H, Nq, D);
+  {  // the fp32 dQ accumulator [B, H, Nq, D], for the kernel's reduce-adds: 32 x 32 boxes, 128-byte swizzle
+    cuuint64_t dims[4] = {(cuuint64_t)D, (cuuint64_t)Nq, (cuuint64_t)H, (cuuint64_t)B};
+    cuuint64_t strides[3] = {(cuuint64_t)D * 4, (cuuint64_t)(Nq * D * 4), (cuuint64_t)(H * Nq * D * 4)};
+    cuuint32_t box[4] = {32, 32, 1, 1}, estr[4] = {1, 1, 1, 1};
+    if (g_encode(&tdq, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, ws, dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                 CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                 CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
+      return FA_ERR_LAUNCH;
+  }
   fa::BwdParams p;
   p.o = o; p.dout = dout; p.lse = lse;
   p.dq_acc = static_cast<float*>(ws);
@@ -570,8 +579,8 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   if (cudaMemsetAsync(p.dq_acc, 0, (size_t)(B * H * Nq * D * 4), stream) != cudaSuccess) return FA_ERR_LAUNCH;
   fa::fa_bwd_pre_kernel<D, T><<<(unsigned int)((pre_rows + 255) / 256), 256, 0, stream>>>(p);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
-  fa::fa_bwd_kernel<D, T><<<(unsigned int)ctas, fa::BWD_THREADS, fa::BwdCfg<D>::SMEM_BYTES, stream>>>(tq, tk, tv, tdo,
-                                                                                                    p, status);
+  fa::fa_bwd_kernel<D, T><<<(unsigned int)ctas, fa::BWD_THREADS, fa::BwdCfg<D>::SMEM_BYTES, stream>>>(
+      tq, tk, tv, tdo, tdq, p, status);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
   fa::fa_bwd_post_kernel<D, T><<<(unsigned int)((post_items + 255) / 256), 256, 0, stream>>>(p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_LAUNCH;
@@ -1148,6 +1157,15 @@ int fa_debug_short_trace_read(unsigned long long* host, int n, int which) {
   const cudaError_t e = which ? cudaMemcpyFromSymbol(host, fa::g_trace_short_wg, n * sizeof(unsigned long long))
                               : cudaMemcpyFromSymbol(host, fa::g_trace_short, n * sizeof(unsigned long long));
   return e == cudaSuccess ? n : FA_ERR_LAUNCH;
+}
+#endif
+
+#ifdef FA_TRACE_BWD
+int fa_debug_bwd_trace_read(unsigned long long* host, int n) {
+  const int total = fa::BWT_CTAS * fa::BWT_STEPS * fa::BWT_EV;
+  if (n > total) n = total;
+  return cudaMemcpyFromSymbol(host, fa::g_trace_bwd, n * sizeof(unsigned long long)) == cudaSuccess ? n
+                                                                                                    : FA_ERR_LAUNCH;
 }
 #endif
 

@@ -20,26 +20,33 @@
 //                        of every query head that reads this K/V head (under
 //                        a causal mask only the query tiles at or after the
 //                        key tile).  dQ of each step is added to an fp32
-//                        accumulator in the workspace (vector reductions).
+//                        accumulator in the workspace (TMA reduce-adds).
 //   fa_bwd_post_kernel   dQ = scale * accumulator, rounded to the input dtype.
 //
-// fa_bwd_kernel, per query tile (step s):
-//   warp 5      TMA: K, V once; Q(s) and dO(s) into a two-stage ring.
-//   warp 4      MMA issuer (whole warp, elect.sync):
+// fa_bwd_kernel, per query tile (step s), 320 threads:
+//   warp 9      TMA: K, V once; Q(s) and dO(s) into a two-stage ring.  Once
+//               the elementwise warps have staged dQ(s) in that stage, the
+//               same thread adds it to the accumulator (TMA reduce-adds of
+//               32 x 32 fp32 boxes) and reloads the stage for step s + 2
+//               when the adds have read it.
+//   warp 8      MMA issuer (whole warp, elect.sync):
 //                 S^T = K Q^T -> R_S;  dP^T = V dO^T -> R_DP;
-//                 then, once P^T and dS^T are written:
-//                 dV += P^T dO (A = P^T from TMEM), dK += dS^T Q (A = dS^T
-//                 from TMEM), dQ = dS K (A = dS from shared memory, read
-//                 M-major from the transposed tile) -> R_DQ.
-//   warps 0-3   one key row (one TMEM lane) per thread: P^T = 2^(S^T scale
-//               log2 e - LSE log2 e) for its 128 query columns (the column
-//               statistics come from the workspace by uniform vector loads),
-//               then dS^T = P^T o (dP^T - D); P^T and dS^T go back to tensor
-//               memory as 16-bit pairs, dS^T also to shared memory in the
-//               128-byte-swizzled layout; then the thread reads one query row
-//               of dQ and adds it to the accumulator (vector reductions).
-//               After the last step it
-//               writes its key row of dV and scale * dK.
+//                 dV += P^T dO (A = P^T from TMEM) as soon as P^T is written;
+//                 once dS^T is: dK += dS^T Q (A = dS^T from TMEM), dQ = dS K
+//                 (A = dS from shared memory, read M-major from the
+//                 transposed tile) -> R_DQ; then S^T of the next step.
+//   warps 0-7   two warpgroups; group g takes query columns [64 g, 64 g +
+//               64) of each step, warp w % 4 of a group TMEM lanes 32 w ..
+//               32 w + 31, one key row per thread: P^T = 2^(S^T scale log2 e
+//               - LSE log2 e) (the column statistics by uniform vector loads,
+//               prefetched into L1 a step ahead), then dS^T = P^T o (dP^T -
+//               D); P^T and dS^T go back to tensor memory as 16-bit pairs
+//               over columns the group has read, dS^T also to shared memory
+//               (128-byte swizzle); then each thread reads its query row of
+//               dQ (columns [g D/2, g D/2 + D/2)) and stages it in the step's
+//               Q (group 0) or dO (group 1) tile, whose MMAs are done.  After
+//               the last step: dV and scale * dK of its key row, the group's
+//               columns.
 //
 // TMEM (512 columns): R_S [0, 128), R_DP [128, 256), dV [256, 256 + D),
 // dK [256 + D, 256 + 2D); R_DQ is [256 + 2D, 256 + 3D) when D = 64, and R_DP
@@ -57,17 +64,45 @@
 
 namespace fa {
 
-#ifndef FA_BWD_BULK_DQ
-#define FA_BWD_BULK_DQ 0
+#ifndef FA_BWD_VEC_DQ
+#define FA_BWD_VEC_DQ 0
 #endif
-// 0 (default): dQ rows reach the accumulator as per-thread 16-byte vector
-// reductions; 1: as bulk reductions from shared memory (one per thread and 32
-// columns), measured slower on the LLaMA-13B 8K backward (310 against 383
-// TFLOP/s).
-constexpr int BWD_BULK_DQ = FA_BWD_BULK_DQ;
-constexpr int BWD_WARP_MMA = 4;
-constexpr int BWD_WARP_TMA = 5;
-constexpr int BWD_THREADS = 32 * 6;
+// How dQ(s) reaches the fp32 accumulator.  0 (default): each warp stages its
+// 32 query rows in shared memory (128-byte swizzle) and one lane adds them
+// with TMA tensor reduce-adds, 32 x 32 fp32 per instruction; 1: per-thread
+// 16-byte vector reductions (red.global.add.v4.f32), one row per thread: 32
+// separate 16-byte atomics per warp instruction, which the step trace showed
+// taking 2.9 us of a 7.3 us step.
+constexpr int BWD_VEC_DQ = FA_BWD_VEC_DQ;
+
+// TMA tensor reduce-add shared -> global (4-D tile, fp32 add; rows outside the
+// tensor are skipped by the tensor map).
+__device__ __forceinline__ void bwd_tma_reduce_add_4d(const void* tmap, uint32_t src, int c0, int c1, int c2, int c3) {
+  asm volatile("cp.reduce.async.bulk.tensor.4d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3, %4, %5}], [%1];" ::"l"(
+                   tmap),
+               "r"(src), "r"(c0), "r"(c1), "r"(c2), "r"(c3)
+               : "memory");
+}
+
+// Optional timeline (compile with -DFA_TRACE_BWD): %globaltimer stamps of the
+// first steps of a few CTAs, readable through fa_debug_bwd_trace_read().
+#ifdef FA_TRACE_BWD
+constexpr int BWT_CTAS = 8, BWT_STEPS = 8, BWT_EV = 8;
+__device__ unsigned long long g_trace_bwd[BWT_CTAS * BWT_STEPS * BWT_EV];
+#define FA_BWT(cond, s, ev)                                                                             \
+  do {                                                                                                 \
+    if ((cond) && blockIdx.x < BWT_CTAS && (s) < BWT_STEPS)                                            \
+      g_trace_bwd[(blockIdx.x * BWT_STEPS + (s)) * BWT_EV + (ev)] = globaltimer_ns();                  \
+  } while (0)
+#else
+#define FA_BWT(cond, s, ev) \
+  do {                      \
+  } while (0)
+#endif
+constexpr int BWD_EW_WARPS = 8;  // elementwise warps: two warpgroups, one per half of a step's query columns
+constexpr int BWD_WARP_MMA = 8;
+constexpr int BWD_WARP_TMA = 9;
+constexpr int BWD_THREADS = 32 * 10;
 
 template <int D>
 struct BwdCfg {
@@ -81,8 +116,8 @@ struct BwdCfg {
   static constexpr int OFF_DO = OFF_Q + QST * TILE_BYTES;
   static constexpr int OFF_DS = OFF_DO + QST * TILE_BYTES;  // dS^T, 128 keys x 128 queries, 16-bit
   static constexpr int OFF_BAR = OFF_DS + 128 * 128 * 2;
-  // kv_full qd_full[QST] qd_empty[QST] s_full dp_full p_ready dq_full dq_free ds_free dkdv_full drain
-  static constexpr int NBAR = 1 + 2 * QST + 8;
+  // kv_full qd_full[QST] qd_empty[QST] s_full dp_full p_ready dq_full dq_free ds_free dkdv_full drain pt_ready
+  static constexpr int NBAR = 1 + 2 * QST + 9;
   static constexpr int USED = OFF_BAR + NBAR * 8 + 16 + 1024;
   // At least 120 KB, so that one CTA (and its 512 TMEM columns) fits an SM.
   static constexpr int SMEM_BYTES = USED > 120 * 1024 ? USED : 120 * 1024;
@@ -183,8 +218,8 @@ __global__ void fa_bwd_post_kernel(BwdParams p) {
 template <int D, typename T>
 __global__ void __launch_bounds__(BWD_THREADS, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_k,
-                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do, BwdParams p,
-                  unsigned int* status_word) {
+                  const __grid_constant__ CUtensorMap tm_v, const __grid_constant__ CUtensorMap tm_do,
+                  const __grid_constant__ CUtensorMap tm_dq, BwdParams p, unsigned int* status_word) {
   using C = BwdCfg<D>;
   constexpr bool IS_BF16 = std::is_same<T, __nv_bfloat16>::value;
   constexpr int QST = C::QST;
@@ -194,7 +229,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   const int B_KV = 0, B_QFULL = 1, B_QEMPTY = 1 + QST, B_SFULL = 1 + 2 * QST, B_DPFULL = B_SFULL + 1,
             B_PREADY = B_SFULL + 2, B_DQFULL = B_SFULL + 3, B_DQFREE = B_SFULL + 4, B_DSFREE = B_SFULL + 5,
-            B_DKDV = B_SFULL + 6, B_DRAIN = B_SFULL + 7;
+            B_DKDV = B_SFULL + 6, B_DRAIN = B_SFULL + 7, B_PTREADY = B_SFULL + 8;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
@@ -216,16 +251,17 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     mbar_init(bar(B_KV), 1);
     for (int s = 0; s < QST; ++s) {
       mbar_init(bar(B_QFULL + s), 1);
-      mbar_init(bar(B_QEMPTY + s), 1);
+      mbar_init(bar(B_QEMPTY + s), BWD_EW_WARPS);  // released by the warps once their dQ adds read it
     }
     mbar_init(bar(B_SFULL), 1);
     mbar_init(bar(B_DPFULL), 1);
-    mbar_init(bar(B_PREADY), 4);
+    mbar_init(bar(B_PREADY), BWD_EW_WARPS);
     mbar_init(bar(B_DQFULL), 1);
-    mbar_init(bar(B_DQFREE), 4);
+    mbar_init(bar(B_DQFREE), BWD_EW_WARPS);
     mbar_init(bar(B_DSFREE), 1);
     mbar_init(bar(B_DKDV), 1);
     mbar_init(bar(B_DRAIN), 1);
+    mbar_init(bar(B_PTREADY), BWD_EW_WARPS);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -238,6 +274,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     prefetch_tmap(&tm_k);
     prefetch_tmap(&tm_v);
     prefetch_tmap(&tm_do);
+    prefetch_tmap(&tm_dq);
   }
   __syncwarp();
   tc_fence_before();
@@ -261,11 +298,32 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           tma_load_4d(sbase + C::OFF_V + c * C::CHUNK_BYTES, &tm_v, bar(B_KV), c * 64, kt * 128, hk, b, pol_kv);
         }
       }
+      // dQ of step sd, staged by the eight elementwise warps in the Q and dO
+      // tiles of its stage, goes to the accumulator: one reduce-add per
+      // 32 x 32 box, then wait until they have read the stage.
+      constexpr int DH = D / 2;
+      auto add_dq = [&](int sd) {
+        const int hd = hk * group + sd / nqt, qtd = qt0 + sd % nqt, std_ = sd % QST;
+        if (!BWD_VEC_DQ) {
+          for (int gg = 0; gg < 2; ++gg) {
+            const uint32_t base = sbase + (gg == 0 ? C::OFF_Q : C::OFF_DO) + std_ * C::TILE_BYTES;
+            for (int w = 0; w < 4; ++w)
+              for (int k2 = 0; k2 < DH / 32; ++k2)
+                bwd_tma_reduce_add_4d(&tm_dq, base + (w * (DH / 32) + k2) * 4096, DH * gg + 32 * k2,
+                                      qtd * 128 + 32 * w, hd, b);
+          }
+          sh_bulk_commit();
+          sh_bulk_wait_read0();
+        }
+      };
       int s = 0;
       for (; s < n; ++s) {
         const int h = hk * group + s / nqt, qt = qt0 + s % nqt;
         const int st = s % QST;
-        if (!mbar_wait(bar(B_QEMPTY + st), ((s / QST) & 1) ^ 1, wctx)) break;
+        if (s >= QST) {  // the stage's previous step: its dQ staged (so its MMAs are done), then added
+          if (!mbar_wait(bar(B_QEMPTY + st), ((s / QST) - 1) & 1, wctx)) break;
+          add_dq(s - QST);
+        }
         mbar_arrive_expect_tx(bar(B_QFULL + st), 2 * C::TILE_BYTES);
         const uint32_t qd = sbase + C::OFF_Q + st * C::TILE_BYTES, dd = sbase + C::OFF_DO + st * C::TILE_BYTES;
         for (int c = 0; c < C::CHUNKS; ++c) {
@@ -278,7 +336,13 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
           }
         }
       }
-      // Every copy this thread started lands before the CTA may exit.
+      // the last steps' dQ
+      if (s == n)
+        for (int sd = (n > QST ? n - QST : 0); sd < n; ++sd) {
+          if (!mbar_wait(bar(B_QEMPTY + sd % QST), (sd / QST) & 1, wctx)) break;
+          add_dq(sd);
+        }
+      // Every copy this thread started lands (and every add completes) before the CTA may exit.
       WaitCtx drain{abort_flag, status_word, p.timeout_ns, 1u};
       volatile int no_abort = 0;
       drain.abort_flag = &no_abort;
@@ -287,6 +351,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         const int g = s - i;
         mbar_wait(bar(B_QFULL + g % QST), (g / QST) & 1, drain);
       }
+      sh_bulk_wait0();
     }
     __syncwarp();
   } else if (warp == BWD_WARP_MMA) {
@@ -335,19 +400,26 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         sh_mma_ss(tmem + C::R_DP, dV_k + o, ddo + o, ID_KK, kk > 0 ? 1u : 0u);
       }
       mma_commit_elect(bar(B_DPFULL));
-      if (!wait_all(B_PREADY, s & 1)) { ok = false; break; }
+      // dV += P^T dO(s) as soon as P^T is written (the warps compute dS^T
+      // meanwhile); dK and dQ once dS^T is
+      if (!wait_all(B_PTREADY, s & 1)) { ok = false; break; }
       tc_fence_after();
       const uint64_t dom = dO_mn0 + (uint64_t)((st * C::TILE_BYTES) >> 4);
+      // 8 steps of 16 query columns; queries 64 g + 16 i (g the warpgroup)
+      // sit packed at column 64 g + 8 i
+#pragma unroll
+      for (int kk = 0; kk < 8; ++kk)
+        sh_mma_ts(tmem + C::R_DV, tmem + C::R_S + 64 * (kk >> 2) + 8 * (kk & 3), dom + (uint64_t)((kk * 2048) >> 4),
+                  ID_TB, (s > 0 || kk > 0) ? 1u : 0u);
+      if (!wait_all(B_PREADY, s & 1)) { ok = false; break; }
+      FA_BWT(lane == 0, s, 7);
+      tc_fence_after();
       const uint64_t dqm = dQ_mn0 + (uint64_t)((st * C::TILE_BYTES) >> 4);
-      // dV += P^T dO(s), dK += dS^T Q(s): 8 steps of 16 query columns each
+      // dK += dS^T Q(s), in the same packed layout
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
-        sh_mma_ts(tmem + C::R_DV, tmem + C::R_S + 8 * kk, dom + (uint64_t)((kk * 2048) >> 4), ID_TB,
-                  (s > 0 || kk > 0) ? 1u : 0u);
-#pragma unroll
-      for (int kk = 0; kk < 8; ++kk)
-        sh_mma_ts(tmem + C::R_DK, tmem + C::R_DP + 8 * kk, dqm + (uint64_t)((kk * 2048) >> 4), ID_TB,
-                  (s > 0 || kk > 0) ? 1u : 0u);
+        sh_mma_ts(tmem + C::R_DK, tmem + C::R_DP + 64 * (kk >> 2) + 8 * (kk & 3), dqm + (uint64_t)((kk * 2048) >> 4),
+                  ID_TB, (s > 0 || kk > 0) ? 1u : 0u);
       // dQ(s) = dS K: 8 steps of 16 keys
 #pragma unroll
       for (int kk = 0; kk < 8; ++kk)
@@ -355,7 +427,6 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
                   kk > 0 ? 1u : 0u);
       mma_commit_elect(bar(B_DQFULL));
       mma_commit_elect(bar(B_DSFREE));
-      mma_commit_elect(bar(B_QEMPTY + st));
       if (s + 1 < n && !issue_s(s + 1)) { ok = false; break; }
     }
     if (n > 0) mma_commit_elect(bar(B_DKDV));
@@ -368,28 +439,46 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     }
     __syncwarp();
   } else {
-    // ------------------------------------------------------------ elementwise + dQ + epilogue (warps 0-3)
-    const int r = warp * 32 + lane;  // TMEM lane: key row (S^T, dP^T, dV, dK) or query row (dQ)
-    const uint32_t lane_base = (uint32_t)(warp * 32) << 16;
+    // ------------------------------------------------------------ elementwise + dQ + epilogue (warps 0-7)
+    // Warpgroup g takes query columns [64 g, 64 g + 64) of every step (and,
+    // for dQ, dV and dK, columns [g D / 2, g D / 2 + D / 2) of d); warp
+    // w = warp % 4 of either group owns TMEM lanes 32 w .. 32 w + 31.
+    const int g = warp >> 2, wq = warp & 3;
+    const int r = wq * 32 + lane;  // TMEM lane: key row (S^T, dP^T, dV, dK) or query row (dQ)
+    const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
     const uint32_t tl = tmem + lane_base;
     const int key = kt * 128 + r;
     const float sl2 = p.scale_log2;
+    constexpr int DH = D / 2;  // columns of d per warpgroup
+    // L1 prefetch of a step's column statistics for this group (LSE * log2 e
+    // and D, 64 floats each: two 128-byte lines apiece, lanes 0-3)
+    auto prefetch_stats = [&](int s2) {
+      if (lane < 4) {
+        const int h2 = hk * group + s2 / nqt, qt2 = qt0 + s2 % nqt;
+        const long long o2 = ((long long)b * p.H + h2) * p.nq_pad + qt2 * 128 + 64 * g + 32 * (lane & 1);
+        asm volatile("prefetch.global.L1 [%0];" ::"l"((lane < 2 ? p.lse2 : p.delta) + o2));
+      }
+    };
+    if (n > 0) prefetch_stats(0);
     bool ok = true;
     for (int s = 0; s < n && ok; ++s) {
       const int h = hk * group + s / nqt, qt = qt0 + s % nqt;
+      const int st = s % QST;
       const long long bh = (long long)b * p.H + h;
-      const float* lse2 = p.lse2 + bh * p.nq_pad + qt * 128;  // 128 query columns (padded)
-      const float* dlt = p.delta + bh * p.nq_pad + qt * 128;
+      const float* lse2 = p.lse2 + bh * p.nq_pad + qt * 128 + 64 * g;  // this group's 64 query columns (padded)
+      const float* dlt = p.delta + bh * p.nq_pad + qt * 128 + 64 * g;
+      FA_BWT(threadIdx.x == 0, s, 0);
       ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SFULL), s & 1, wctx));
       if (!ok) break;
+      FA_BWT(threadIdx.x == 0, s, 1);
       tc_fence_after();
       // visible iff key < Nkv and (causal) key <= query
       const bool need_mask = (kt * 128 + 128 > p.Nkv) || (p.causal && kt == qt);
-      float pr[128];
+      float pr[64];
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         float sc[32];
-        tmem_ld32(tl + C::R_S + 32 * c, sc);
+        tmem_ld32(tl + C::R_S + 64 * g + 32 * c, sc);
         float4 l4[8];
 #pragma unroll
         for (int t = 0; t < 8; ++t) l4[t] = reinterpret_cast<const float4*>(lse2 + 32 * c)[t];
@@ -399,23 +488,28 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         for (int t = 0; t < 32; ++t) {
           float x = fmaf(sc[t], sl2, -lv[t]);
           if (need_mask) {
-            const int qi = qt * 128 + 32 * c + t;
+            const int qi = qt * 128 + 64 * g + 32 * c + t;
             if (key >= p.Nkv || (p.causal && key > qi)) x = -INFINITY;
           }
           pr[32 * c + t] = ex2(x);
         }
 #pragma unroll
         for (int t = 0; t < 16; ++t) pk[t] = sh_pack2<T>(pr[32 * c + 2 * t], pr[32 * c + 2 * t + 1]);
-        sh_tmem_st16(tl + C::R_S + 16 * c, pk);  // P^T over columns already read
+        sh_tmem_st16(tl + C::R_S + 64 * g + 16 * c, pk);  // P^T over this group's columns already read
       }
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive_warp(bar(B_PTREADY));
+      FA_BWT(threadIdx.x == 0, s, 2);
       ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DPFULL), s & 1, wctx));
+      FA_BWT(threadIdx.x == 0, s, 3);
       if (ok && s > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DSFREE), (s - 1) & 1, wctx));
       if (!ok) break;
       tc_fence_after();
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < 2; ++c) {
         float dp[32];
-        tmem_ld32(tl + C::R_DP + 32 * c, dp);
+        tmem_ld32(tl + C::R_DP + 64 * g + 32 * c, dp);
         float4 d4[8];
 #pragma unroll
         for (int t = 0; t < 8; ++t) d4[t] = reinterpret_cast<const float4*>(dlt + 32 * c)[t];
@@ -425,13 +519,13 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         for (int t = 0; t < 16; ++t)
           pk[t] = sh_pack2<T>(pr[32 * c + 2 * t] * (dp[2 * t] - dv[2 * t]),
                               pr[32 * c + 2 * t + 1] * (dp[2 * t + 1] - dv[2 * t + 1]));
-        sh_tmem_st16(tl + C::R_DP + 16 * c, pk);  // dS^T over columns already read
+        sh_tmem_st16(tl + C::R_DP + 64 * g + 16 * c, pk);  // dS^T over columns already read
         // the same 32 query columns of this key row into the shared dS^T tile:
-        // 64-column chunk c / 2, 16-byte pieces 4 (c % 2) .. + 3, 128-byte swizzle
-        const uint32_t rowb = sbase + C::OFF_DS + (c >> 1) * C::CHUNK_BYTES + r * 128;
+        // 64-column chunk g, 16-byte pieces 4 c .. 4 c + 3, 128-byte swizzle
+        const uint32_t rowb = sbase + C::OFF_DS + g * C::CHUNK_BYTES + r * 128;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
-          const int piece = 4 * (c & 1) + j;
+          const int piece = 4 * c + j;
           st_shared_v4(rowb + ((piece ^ (r & 7)) << 4), pk[4 * j], pk[4 * j + 1], pk[4 * j + 2], pk[4 * j + 3]);
         }
       }
@@ -439,55 +533,52 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive_warp(bar(B_PREADY));
-      // dQ(s): this thread's query row qt * 128 + r, added to the accumulator
+      FA_BWT(threadIdx.x == 0, s, 4);
+      if (s + 1 < n) prefetch_stats(s + 1);  // lands in L1 while the MMAs of this step run
+      // dQ(s): query rows qt * 128 + r, this group's D / 2 columns
       ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DQFULL), s & 1, wctx));
       if (!ok) break;
+      FA_BWT(threadIdx.x == 0, s, 5);
       tc_fence_after();
       const int qrow = qt * 128 + r;
-      float* acc = p.dq_acc + (bh * p.Nq + qrow) * D;
-      const bool qvalid = qrow < p.Nq && FA_INDEX_OK(status_word, (bh * p.Nq + qrow) < (long long)p.B * p.H * p.Nq);
-      if constexpr (BWD_BULK_DQ) {
-        // 32 columns at a time through the dS tile (free: dQ's MMA has read
-        // it): this thread's 128 bytes at a row stride of 144 bytes (eight
-        // consecutive rows then fall on different banks), then one bulk add
-        // of them into the accumulator row.
-        const uint32_t rowb = sbase + C::OFF_DS + r * 144;
-#pragma unroll 1
-        for (int c0 = 0; c0 < D; c0 += 32) {
-          float v[32];
-          tmem_ld32(tl + C::R_DQ + c0, v);
-          if (c0 > 0) asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");
-#pragma unroll
-          for (int j = 0; j < 8; ++j)
-            st_shared_v4(rowb + j * 16, __float_as_uint(v[4 * j]), __float_as_uint(v[4 * j + 1]),
-                         __float_as_uint(v[4 * j + 2]), __float_as_uint(v[4 * j + 3]));
-          fence_proxy_async_smem();
-          if (qvalid)
-            asm volatile("cp.reduce.async.bulk.global.shared::cta.bulk_group.add.f32 [%0], [%1], 128;" ::"l"(acc + c0),
-                         "r"(rowb)
-                         : "memory");
-          asm volatile("cp.async.bulk.commit_group;" ::: "memory");
-        }
-        asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory");  // the dS tile is written again next step
+      float v[DH];
+      if constexpr (DH == 64) {
+        tmem_ld64(tl + C::R_DQ + DH * g, v);
       } else {
-#pragma unroll 1
-        for (int c = 0; c < D; c += 32) {
-          float v[32];
-          tmem_ld32(tl + C::R_DQ + c, v);
-          if (qvalid) {
-#pragma unroll
-            for (int t = 0; t < 8; ++t)
-              asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(acc + c + 4 * t), "f"(v[4 * t]),
-                           "f"(v[4 * t + 1]), "f"(v[4 * t + 2]), "f"(v[4 * t + 3])
-                           : "memory");
-          }
-        }
+        tmem_ld32(tl + C::R_DQ + DH * g, v);
       }
       tc_fence_before();
-      mbar_arrive_warp(bar(B_DQFREE));
+      mbar_arrive_warp(bar(B_DQFREE));  // dQ is read: R_DQ may be written again
+      FA_BWT(threadIdx.x == 0, s, 6);
+      if constexpr (!BWD_VEC_DQ) {
+        // Stage this warp's 32 rows x D / 2 columns in the step's Q or dO
+        // tile (group 0 / 1; every MMA that reads them is done), as 32 x 32
+        // boxes at 128-byte swizzle; the TMA warp adds them to the
+        // accumulator.
+        const uint32_t stage = sbase + (g == 0 ? C::OFF_Q : C::OFF_DO) + st * C::TILE_BYTES + wq * (DH / 32) * 4096;
+#pragma unroll
+        for (int k2 = 0; k2 < DH / 32; ++k2) {
+          const uint32_t rowb = stage + k2 * 4096 + lane * 128;
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            st_shared_v4(rowb + ((j ^ (lane & 7)) << 4), __float_as_uint(v[32 * k2 + 4 * j]),
+                         __float_as_uint(v[32 * k2 + 4 * j + 1]), __float_as_uint(v[32 * k2 + 4 * j + 2]),
+                         __float_as_uint(v[32 * k2 + 4 * j + 3]));
+        }
+        fence_proxy_async_smem();
+      } else {
+        if (qrow < p.Nq && FA_INDEX_OK(status_word, (bh * p.Nq + qrow) < (long long)p.B * p.H * p.Nq)) {
+          float* acc = p.dq_acc + (bh * p.Nq + qrow) * D + DH * g;
+#pragma unroll
+          for (int t = 0; t < DH / 4; ++t)
+            asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(acc + 4 * t), "f"(v[4 * t]),
+                         "f"(v[4 * t + 1]), "f"(v[4 * t + 2]), "f"(v[4 * t + 3])
+                         : "memory");
+        }
+      }
+      mbar_arrive_warp(bar(B_QEMPTY + st));  // staged (or added): the TMA warp takes the stage from here
     }
-    if constexpr (BWD_BULK_DQ) asm volatile("cp.async.bulk.wait_group 0;" ::: "memory");  // dQ adds complete
-    // ---------------------------------------------------------- dK, dV of this key row
+    // ---------------------------------------------------------- dK, dV of this key row, this group's columns
     if (ok && n > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DKDV), 0, wctx));
     if (ok) {
       tc_fence_after();
@@ -497,7 +588,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       T* dvp = static_cast<T*>(p.dv) + off;
       T* dkp = static_cast<T*>(p.dk) + off;
 #pragma unroll 1
-      for (int c = 0; c < D; c += 32) {
+      for (int c = DH * g; c < DH * g + DH; c += 32) {
         float v[32], k2[32];
         if (n > 0) {
           tmem_ld32(tl + C::R_DV + c, v);

@@ -79,7 +79,10 @@ typedef enum {
  * tile scheduler's per-launch work counters (kept until the process exits;
  * make that first call outside any stream capture); later calls allocate
  * nothing.  The call is asynchronous: it validates, encodes TMA descriptors
- * on the host and launches one kernel on `stream`.
+ * on the host and launches one kernel on `stream`.  (Head dim 64 with
+ * Nkv <= 128 runs a dependent launch: the kernel may start while the
+ * previous work on the stream drains, and waits for it before touching any
+ * memory.)
  *
  * Returns FA_OK (also for B*H*Nq == 0, a no-op), or FA_ERR_INVALID_ARG /
  * FA_ERR_UNSUPPORTED / FA_ERR_MISALIGNED before anything is launched, or
@@ -254,6 +257,15 @@ int fa_fwd_paged(const void* q, const void* k_cache, const void* v_cache, const 
  * causal = 0 (these forms take no mask: every query row sees every key, as
  * a decoding step's new tokens see the whole cache).  O and LSE differ from
  * the unsplit call only by rounding.
+ *
+ * Calls with at most 8 query rows per K/V head (Nq * H / Hkv <= 8),
+ * contiguous or paged, run a CUDA-core streaming kernel instead of the
+ * tensor-core units: one CTA per (slice, batch, K/V head) takes all of the
+ * K/V head's query rows; same plan, workspace and merge.  That kernel and
+ * the merge are launched as dependent launches (programmatic stream
+ * serialisation): each may start while the previous work on the stream
+ * drains, and waits for it before touching any memory, so stream order is
+ * kept.
  *
  * fa_splitkv_plan -- the slice count and workspace size of a split-KV call.
  *

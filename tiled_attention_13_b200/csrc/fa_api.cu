@@ -17,6 +17,12 @@
 
 #include "fa.h"
 
+// Causal d = 128 calls on the one-row-per-thread kernel as well (build option,
+// for comparison: measured slower than the two-tile kernel with a mask).
+#ifndef FA_TC2_CAUSAL
+#define FA_TC2_CAUSAL 0
+#endif
+
 // Head dim 64 with at most 128 keys on the four-pipeline short-key kernel
 // (0: on the two-warpgroup one, for comparison).
 #ifndef FA_SHORT_WG
@@ -774,7 +780,7 @@ int fwd_common(const void* q, const void* k, const void* v, void* o, float* lse,
                    : launch_short<128, __half>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s,
                                                di->num_sms, di->status);
   }
-  if (d == 128 && !causal) {  // the one-row-per-thread kernel: measured faster without a mask
+  if (d == 128 && (!causal || FA_TC2_CAUSAL)) {  // the one-row-per-thread kernel: measured faster without a mask
     fa::SchedSlot* slot = di->sched + (di->launches.fetch_add(1) % kSchedSlots);
     return dtype == FA_DTYPE_BF16
                ? launch_tc2<128, __nv_bfloat16>(q, k, v, o, lse, B, H, Hkv, Nq, Nkv, scale, causal, bsnd, s,
@@ -1363,7 +1369,7 @@ extern "C" int fa_fwd_noalloc(const void* q, const void* k, const void* v, void*
                    : launch_short<128, __half>(q, k, v, o, lse, B, H, H, Nq, Nkv, scale, causal, bsnd, s, nd->num_sms,
                                                nd->status);
   }
-  if (d == 128 && !causal) {  // as fa_fwd: the one-row-per-thread kernel, its counter in slot 0
+  if (d == 128 && (!causal || FA_TC2_CAUSAL)) {  // as fa_fwd: the one-row-per-thread kernel, its counter in slot 0
     if (cudaMemsetAsync(nd->scratch, 0, sizeof(fa::SchedSlot), s) != cudaSuccess) return FA_ERR_LAUNCH;
     return dtype == FA_DTYPE_BF16
                ? launch_tc2<128, __nv_bfloat16>(q, k, v, o, lse, B, H, H, Nq, Nkv, scale, causal, bsnd, s,

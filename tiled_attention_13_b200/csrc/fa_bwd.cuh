@@ -474,25 +474,29 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       tc_fence_after();
       // visible iff key < Nkv and (causal) key <= query
       const bool need_mask = (kt * 128 + 128 > p.Nkv) || (p.causal && kt == qt);
+      // the group's 64 scores of this key row in one tensor-memory read,
+      // then P^T in place (64 independent exps per thread)
       float pr[64];
+      tmem_ld64(tl + C::R_S + 64 * g, pr);
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        float sc[32];
-        tmem_ld32(tl + C::R_S + 64 * g + 32 * c, sc);
-        float4 l4[8];
+      for (int t8 = 0; t8 < 8; ++t8) {
+        const float4 la = reinterpret_cast<const float4*>(lse2)[2 * t8];
+        const float4 lb = reinterpret_cast<const float4*>(lse2)[2 * t8 + 1];
+        const float lv[8] = {la.x, la.y, la.z, la.w, lb.x, lb.y, lb.z, lb.w};
 #pragma unroll
-        for (int t = 0; t < 8; ++t) l4[t] = reinterpret_cast<const float4*>(lse2 + 32 * c)[t];
-        const float* lv = reinterpret_cast<const float*>(l4);
-        uint32_t pk[16];
-#pragma unroll
-        for (int t = 0; t < 32; ++t) {
-          float x = fmaf(sc[t], sl2, -lv[t]);
+        for (int u = 0; u < 8; ++u) {
+          const int t = 8 * t8 + u;
+          float x = fmaf(pr[t], sl2, -lv[u]);
           if (need_mask) {
-            const int qi = qt * 128 + 64 * g + 32 * c + t;
+            const int qi = qt * 128 + 64 * g + t;
             if (key >= p.Nkv || (p.causal && key > qi)) x = -INFINITY;
           }
-          pr[32 * c + t] = ex2(x);
+          pr[t] = ex2(x);
         }
+      }
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        uint32_t pk[16];
 #pragma unroll
         for (int t = 0; t < 16; ++t) pk[t] = sh_pack2<T>(pr[32 * c + 2 * t], pr[32 * c + 2 * t + 1]);
         sh_tmem_st16(tl + C::R_S + 64 * g + 16 * c, pk);  // P^T over this group's columns already read
@@ -510,15 +514,15 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       for (int c = 0; c < 2; ++c) {
         float dp[32];
         tmem_ld32(tl + C::R_DP + 64 * g + 32 * c, dp);
-        float4 d4[8];
-#pragma unroll
-        for (int t = 0; t < 8; ++t) d4[t] = reinterpret_cast<const float4*>(dlt + 32 * c)[t];
-        const float* dv = reinterpret_cast<const float*>(d4);
         uint32_t pk[16];
 #pragma unroll
-        for (int t = 0; t < 16; ++t)
-          pk[t] = sh_pack2<T>(pr[32 * c + 2 * t] * (dp[2 * t] - dv[2 * t]),
-                              pr[32 * c + 2 * t + 1] * (dp[2 * t + 1] - dv[2 * t + 1]));
+        for (int t4 = 0; t4 < 8; ++t4) {
+          const float4 d4 = reinterpret_cast<const float4*>(dlt + 32 * c)[t4];
+          const int t = 4 * t4;
+          pk[2 * t4] = sh_pack2<T>(pr[32 * c + t] * (dp[t] - d4.x), pr[32 * c + t + 1] * (dp[t + 1] - d4.y));
+          pk[2 * t4 + 1] =
+              sh_pack2<T>(pr[32 * c + t + 2] * (dp[t + 2] - d4.z), pr[32 * c + t + 3] * (dp[t + 3] - d4.w));
+        }
         sh_tmem_st16(tl + C::R_DP + 64 * g + 16 * c, pk);  // dS^T over columns already read
         // the same 32 query columns of this key row into the shared dS^T tile:
         // 64-column chunk g, 16-byte pieces 4 c .. 4 c + 3, 128-byte swizzle

@@ -191,8 +191,10 @@ def test_polynomial_exp_option(tmp_path):
 def test_index_checks_build(tmp_path):
     """The debug build (FA_CHECKS: every computed global index checked on the
     device, a violation reported as FA_ERR_CHECK) runs the contiguous, fp32,
-    paged, paged split-KV, band and split-KV paths on ragged shapes with a
-    clean status and the usual parity, in a process of its own."""
+    paged, paged split-KV, band and split-KV paths, the short-key kernels
+    (d = 64 and 128), the decoding kernel (contiguous and paged), d = 256,
+    block-sparse masks and the backward on ragged shapes with a clean status
+    and the usual parity, in a process of its own."""
     import os
     import subprocess
     import sys
@@ -215,6 +217,15 @@ def test_index_checks_build(tmp_path):
             "t._paged_parity(pw, num_splits=3)\n"
             "t.test_band_bf16(t.BAND_CASES[1])\n"
             "t.test_splitkv(t.SPLIT_CASES[1])\n"
+            "for d, c in ((64, True), (128, False)):\n"
+            "    compare_full(Workload('chks', B=2, H=3, Nq=300, Nkv=77, d=d, dtype='bf16', layout='BSND', causal=c,"
+            " seed=11))\n"
+            "t.test_paged_decode_kernel(t.PAGED_DECODE_CASES[0])\n"
+            "from tests import test_gpu_tile1 as t1, test_gpu_bwd as tb\n"
+            "t1.test_d256_bf16(t1.D256_SHAPES[2], True, 'BSND')\n"
+            "t1.test_block_sparse(t1.BSP_CASES[0])\n"
+            "tb.test_bwd_bf16(tb.SHAPES[3], 128, True, 'BSND')\n"
+            "tb.test_bwd_bf16(tb.SHAPES[6], 64, False, 'BHND')\n"
             "assert fa.fa_get_device_status(None) == 0\n"
             "print('ok')\n")
     r = subprocess.run([sys.executable, "-c", code], cwd=root, env={**os.environ, "FA_B200_LIB": lib},

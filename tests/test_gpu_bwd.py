@@ -2,10 +2,10 @@
 float64 oracle ``attention_backward_batched`` (page 1, "CANN ops-transformer
 FlashAttentionScore", section 反向传播的重算策略及其合理性).
 
-The stated tolerances are the forward's; the gradients' bar is derived from
-the arithmetic (it is one of the readings the design notes list): P and dS
-are rounded to 16 bits before their products (2^-9 relative each), D comes
-from the forward's rounded O, and the outputs are rounded to the input dtype.
+The stated tolerances are the forward's; the pages give none for the
+gradients, so their bar is derived from the arithmetic: P and dS are rounded
+to 16 bits before their products (2^-9 relative each), D comes from the
+forward's rounded O, and the outputs are rounded to the input dtype.
 Each gradient X must satisfy max|X - X_ref| <= 2^-6 max|X_ref| + 1e-3 and
 ||X - X_ref||_F <= 2^-7 ||X_ref||_F (+ 1e-3 for all-zero references).
 """

@@ -542,6 +542,47 @@ def test_short_keys_many_tiles_per_cta_and_head_switches(d):
     compare_sampled(wl, [(0, 0), (4, 199), (2, 101), (3, 50), (1, 1)], rows_per_head=20)
 
 
+def test_dependent_launches_keep_stream_order():
+    """The short-key (d = 64), decode and merge kernels are dependent
+    launches: they may start while the previous kernel drains and wait for it
+    before touching memory.  Chains where each call reads the previous call's
+    output, with no synchronisation in between, must equal the same chains
+    synchronised after every call (the kernels are deterministic)."""
+    g = torch.Generator().manual_seed(5)
+    # cross-attention shape: O of one call is Q of the next
+    q = torch.randn(2, 8, 1024, 64, generator=g).to(torch.bfloat16).cuda()
+    k = torch.randn(2, 8, 77, 64, generator=g).to(torch.bfloat16).cuda()
+    v = torch.randn(2, 8, 77, 64, generator=g).to(torch.bfloat16).cuda()
+    def chain(x, sync):
+        outs = []
+        for _ in range(4):
+            x, _ = fa.forward(x, k, v)  # reads the previous call's output directly
+            outs.append(x)
+            if sync:
+                torch.cuda.synchronize()
+        return outs
+    a, b = chain(q, False), chain(q, True)
+    torch.cuda.synchronize()
+    assert all(torch.equal(x, y) for x, y in zip(a, b))
+    # decoding shape (split-KV decode kernel and merge): the query of the next
+    # step is this step's output
+    kd = torch.randn(1, 4096, 8, 128, generator=g).to(torch.bfloat16).cuda()
+    vd = torch.randn(1, 4096, 8, 128, generator=g).to(torch.bfloat16).cuda()
+    qd = torch.randn(1, 1, 8, 128, generator=g).to(torch.bfloat16).cuda()
+    def dchain(x, sync):
+        outs = []
+        for _ in range(4):
+            x, _ = fa.forward(x, kd, vd, layout="BSND", num_splits=0)
+            outs.append(x)
+            if sync:
+                torch.cuda.synchronize()
+        return outs
+    a, b = dchain(qd, False), dchain(qd, True)
+    torch.cuda.synchronize()
+    assert all(torch.equal(x, y) for x, y in zip(a, b))
+    assert fa.fa_get_device_status(None) == 0
+
+
 @pytest.mark.parametrize("dtype", ["bf16", "fp16"])
 @pytest.mark.parametrize("causal", [False, True])
 def test_short_keys_reference_max_raised(causal, dtype):

@@ -24,7 +24,10 @@
 //   fa_bwd_post_kernel   dQ = scale * accumulator, rounded to the input dtype.
 //
 // fa_bwd_kernel, per query tile (step s), 320 threads:
-//   warp 9      TMA: K, V once; Q(s) and dO(s) into a two-stage ring.  Once
+//   warp 9      TMA: K, V once; Q(s) and dO(s) into a two-stage ring; the
+//               step's column statistics (LSE * log2 e and D, 512 bytes
+//               each) into single-stage shared buffers, each reloaded as
+//               soon as the phase that reads it has handed over.  Once
 //               the elementwise warps have staged dQ(s) in that stage, the
 //               same thread adds it to the accumulator (TMA reduce-adds of
 //               32 x 32 fp32 boxes) and reloads the stage for step s + 2
@@ -38,8 +41,8 @@
 //   warps 0-7   two warpgroups; group g takes query columns [64 g, 64 g +
 //               64) of each step, warp w % 4 of a group TMEM lanes 32 w ..
 //               32 w + 31, one key row per thread: P^T = 2^(S^T scale log2 e
-//               - LSE log2 e) (the column statistics by uniform vector loads,
-//               prefetched into L1 a step ahead), then dS^T = P^T o (dP^T -
+//               - LSE log2 e) (the column statistics read from shared
+//               memory), then dS^T = P^T o (dP^T -
 //               D); P^T and dS^T go back to tensor memory as 16-bit pairs
 //               over columns the group has read, dS^T also to shared memory
 //               (128-byte swizzle); then each thread reads its query row of
@@ -84,6 +87,14 @@ __device__ __forceinline__ void bwd_tma_reduce_add_4d(const void* tmap, uint32_t
                : "memory");
 }
 
+// Untiled bulk copy global -> shared of `bytes` (a multiple of 16; both
+// addresses 16-byte aligned), completing on the mbarrier's transaction count.
+__device__ __forceinline__ void bwd_bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
+               "l"(src), "r"(bytes), "r"(bar)
+               : "memory");
+}
+
 // Optional timeline (compile with -DFA_TRACE_BWD): %globaltimer stamps of the
 // first steps of a few CTAs, readable through fa_debug_bwd_trace_read().
 #ifdef FA_TRACE_BWD
@@ -115,9 +126,11 @@ struct BwdCfg {
   static constexpr int OFF_Q = 2 * TILE_BYTES;
   static constexpr int OFF_DO = OFF_Q + QST * TILE_BYTES;
   static constexpr int OFF_DS = OFF_DO + QST * TILE_BYTES;  // dS^T, 128 keys x 128 queries, 16-bit
-  static constexpr int OFF_BAR = OFF_DS + 128 * 128 * 2;
+  static constexpr int OFF_STATS = OFF_DS + 128 * 128 * 2;  // LSE * log2 e [128], then D [128], fp32
+  static constexpr int OFF_BAR = OFF_STATS + 2 * 128 * 4;
   // kv_full qd_full[QST] qd_empty[QST] s_full dp_full p_ready dq_full dq_free ds_free dkdv_full drain pt_ready
-  static constexpr int NBAR = 1 + 2 * QST + 9;
+  // lse_full delta_full
+  static constexpr int NBAR = 1 + 2 * QST + 11;
   static constexpr int USED = OFF_BAR + NBAR * 8 + 16 + 1024;
   // At least 120 KB, so that one CTA (and its 512 TMEM columns) fits an SM.
   static constexpr int SMEM_BYTES = USED > 120 * 1024 ? USED : 120 * 1024;
@@ -229,7 +242,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + C::OFF_BAR);
   const int B_KV = 0, B_QFULL = 1, B_QEMPTY = 1 + QST, B_SFULL = 1 + 2 * QST, B_DPFULL = B_SFULL + 1,
             B_PREADY = B_SFULL + 2, B_DQFULL = B_SFULL + 3, B_DQFREE = B_SFULL + 4, B_DSFREE = B_SFULL + 5,
-            B_DKDV = B_SFULL + 6, B_DRAIN = B_SFULL + 7, B_PTREADY = B_SFULL + 8;
+            B_DKDV = B_SFULL + 6, B_DRAIN = B_SFULL + 7, B_PTREADY = B_SFULL + 8, B_LSEF = B_SFULL + 9,
+            B_DLTF = B_SFULL + 10;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bars + C::NBAR);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
   auto bar = [&](int i) { return smem_u32(&bars[i]); };
@@ -262,6 +276,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     mbar_init(bar(B_DKDV), 1);
     mbar_init(bar(B_DRAIN), 1);
     mbar_init(bar(B_PTREADY), BWD_EW_WARPS);
+    mbar_init(bar(B_LSEF), 1);
+    mbar_init(bar(B_DLTF), 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -317,6 +333,7 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
         }
       };
       int s = 0;
+      int qd_issued = 0, stats_lse = 0, stats_dlt = 0;  // Q/dO stages and statistics loads issued
       for (; s < n; ++s) {
         const int h = hk * group + s / nqt, qt = qt0 + s % nqt;
         const int st = s % QST;
@@ -335,6 +352,20 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
             tma_load_4d(dd + c * C::CHUNK_BYTES, &tm_do, bar(B_QFULL + st), c * 64, qt * 128, h, b, pol_q);
           }
         }
+        qd_issued = s + 1;
+        // Column statistics of step s: the LSE row once P^T(s - 1) has read
+        // the buffer (the warps' arrivals on pt_ready), the D row once
+        // dS^T(s - 1) has (p_ready).  Both waits come in the order the steps
+        // produce them, after this step's Q and dO are on their way.
+        const long long srow = ((long long)b * p.H + h) * p.nq_pad + (long long)qt * 128;
+        if (s > 0 && !mbar_wait(bar(B_PTREADY), (s - 1) & 1, wctx)) break;
+        mbar_arrive_expect_tx(bar(B_LSEF), 512);
+        bwd_bulk_load(sbase + C::OFF_STATS, p.lse2 + srow, 512, bar(B_LSEF));
+        if (s > 0 && !mbar_wait(bar(B_PREADY), (s - 1) & 1, wctx)) { ++stats_lse; break; }
+        mbar_arrive_expect_tx(bar(B_DLTF), 512);
+        bwd_bulk_load(sbase + C::OFF_STATS + 512, p.delta + srow, 512, bar(B_DLTF));
+        ++stats_lse;
+        ++stats_dlt;
       }
       // the last steps' dQ
       if (s == n)
@@ -347,10 +378,12 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       volatile int no_abort = 0;
       drain.abort_flag = &no_abort;
       mbar_wait(bar(B_KV), 0, drain);
-      for (int i = 1; i <= QST && s - i >= 0; ++i) {
-        const int g = s - i;
+      for (int i = 1; i <= QST && qd_issued - i >= 0; ++i) {
+        const int g = qd_issued - i;
         mbar_wait(bar(B_QFULL + g % QST), (g / QST) & 1, drain);
       }
+      if (stats_lse > 0) mbar_wait(bar(B_LSEF), (stats_lse - 1) & 1, drain);
+      if (stats_dlt > 0) mbar_wait(bar(B_DLTF), (stats_dlt - 1) & 1, drain);
       sh_bulk_wait0();
     }
     __syncwarp();
@@ -450,25 +483,16 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
     const int key = kt * 128 + r;
     const float sl2 = p.scale_log2;
     constexpr int DH = D / 2;  // columns of d per warpgroup
-    // L1 prefetch of a step's column statistics for this group (LSE * log2 e
-    // and D, 64 floats each: two 128-byte lines apiece, lanes 0-3)
-    auto prefetch_stats = [&](int s2) {
-      if (lane < 4) {
-        const int h2 = hk * group + s2 / nqt, qt2 = qt0 + s2 % nqt;
-        const long long o2 = ((long long)b * p.H + h2) * p.nq_pad + qt2 * 128 + 64 * g + 32 * (lane & 1);
-        asm volatile("prefetch.global.L1 [%0];" ::"l"((lane < 2 ? p.lse2 : p.delta) + o2));
-      }
-    };
-    if (n > 0) prefetch_stats(0);
+    // this group's 64 column statistics of the current step in shared memory
+    const float4* lse_s = reinterpret_cast<const float4*>(smem + C::OFF_STATS) + 16 * g;
+    const float4* dlt_s = reinterpret_cast<const float4*>(smem + C::OFF_STATS + 512) + 16 * g;
     bool ok = true;
     for (int s = 0; s < n && ok; ++s) {
       const int h = hk * group + s / nqt, qt = qt0 + s % nqt;
       const int st = s % QST;
       const long long bh = (long long)b * p.H + h;
-      const float* lse2 = p.lse2 + bh * p.nq_pad + qt * 128 + 64 * g;  // this group's 64 query columns (padded)
-      const float* dlt = p.delta + bh * p.nq_pad + qt * 128 + 64 * g;
       FA_BWT(threadIdx.x == 0, s, 0);
-      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SFULL), s & 1, wctx));
+      ok = __all_sync(0xffffffffu, mbar_wait(bar(B_SFULL), s & 1, wctx) && mbar_wait(bar(B_LSEF), s & 1, wctx));
       if (!ok) break;
       FA_BWT(threadIdx.x == 0, s, 1);
       tc_fence_after();
@@ -480,8 +504,8 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       tmem_ld64(tl + C::R_S + 64 * g, pr);
 #pragma unroll
       for (int t8 = 0; t8 < 8; ++t8) {
-        const float4 la = reinterpret_cast<const float4*>(lse2)[2 * t8];
-        const float4 lb = reinterpret_cast<const float4*>(lse2)[2 * t8 + 1];
+        const float4 la = lse_s[2 * t8];
+        const float4 lb = lse_s[2 * t8 + 1];
         const float lv[8] = {la.x, la.y, la.z, la.w, lb.x, lb.y, lb.z, lb.w};
 #pragma unroll
         for (int u = 0; u < 8; ++u) {
@@ -508,16 +532,22 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DPFULL), s & 1, wctx));
       FA_BWT(threadIdx.x == 0, s, 3);
       if (ok && s > 0) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DSFREE), (s - 1) & 1, wctx));
+      if (ok) ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DLTF), s & 1, wctx));
       if (!ok) break;
       tc_fence_after();
 #pragma unroll
       for (int c = 0; c < 2; ++c) {
+        // D of these 32 columns first: its shared-memory reads overlap the
+        // tensor-memory read of dP^T
+        float4 dv4[8];
+#pragma unroll
+        for (int t4 = 0; t4 < 8; ++t4) dv4[t4] = dlt_s[8 * c + t4];
         float dp[32];
         tmem_ld32(tl + C::R_DP + 64 * g + 32 * c, dp);
         uint32_t pk[16];
 #pragma unroll
         for (int t4 = 0; t4 < 8; ++t4) {
-          const float4 d4 = reinterpret_cast<const float4*>(dlt + 32 * c)[t4];
+          const float4 d4 = dv4[t4];
           const int t = 4 * t4;
           pk[2 * t4] = sh_pack2<T>(pr[32 * c + t] * (dp[t] - d4.x), pr[32 * c + t + 1] * (dp[t + 1] - d4.y));
           pk[2 * t4 + 1] =
@@ -538,7 +568,6 @@ __global__ void __launch_bounds__(BWD_THREADS, 1)
       tc_fence_before();
       mbar_arrive_warp(bar(B_PREADY));
       FA_BWT(threadIdx.x == 0, s, 4);
-      if (s + 1 < n) prefetch_stats(s + 1);  // lands in L1 while the MMAs of this step run
       // dQ(s): query rows qt * 128 + r, this group's D / 2 columns
       ok = __all_sync(0xffffffffu, mbar_wait(bar(B_DQFULL), s & 1, wctx));
       if (!ok) break;

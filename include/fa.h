@@ -149,8 +149,8 @@ int fa_bwd_workspace_size(int64_t B, int64_t H, int64_t Nq, int64_t d, int64_t* 
  *
  * Errors: as for fa_fwd_gqa, plus FA_ERR_INVALID_ARG for a missing or too
  * small workspace and FA_ERR_MISALIGNED for a misaligned one, both before
- * any launch.  The call clears the accumulator (cudaMemsetAsync) and
- * launches three kernels on `stream`; Nq == 0 only clears dk and dv.  The
+ * any launch.  The call launches three kernels on `stream` (the first
+ * also clears the accumulator); Nq == 0 only clears dk and dv.  The
  * first-call allocation is fa_fwd's.
  */
 int fa_bwd(const void* q, const void* k, const void* v, const void* o, const void* dout, const float* lse,

@@ -579,11 +579,11 @@ int launch_bwd(const void* q, const void* k, const void* v, const void* o, const
   p.nq_pad = (int)L.nq_pad;
   p.timeout_ns = (uint64_t)g_timeout_us.load() * 1000ull;
   const int64_t ctas = (int64_t)p.kvtiles * B * Hkv;
-  const int64_t pre_rows = B * H * L.nq_pad, post_items = B * H * Nq * (D / 8);
-  if (ctas > INT32_MAX || pre_rows > (int64_t)INT32_MAX * 256 || post_items > (int64_t)INT32_MAX * 256)
+  // pre kernel: D / 8 threads per padded query row (it also clears the dQ accumulator)
+  const int64_t pre_items = B * H * L.nq_pad * (D / 8), post_items = B * H * Nq * (D / 8);
+  if (ctas > INT32_MAX || pre_items > (int64_t)INT32_MAX * 256 || post_items > (int64_t)INT32_MAX * 256)
     return FA_ERR_UNSUPPORTED;
-  if (cudaMemsetAsync(p.dq_acc, 0, (size_t)(B * H * Nq * D * 4), stream) != cudaSuccess) return FA_ERR_LAUNCH;
-  fa::fa_bwd_pre_kernel<D, T><<<(unsigned int)((pre_rows + 255) / 256), 256, 0, stream>>>(p);
+  fa::fa_bwd_pre_kernel<D, T><<<(unsigned int)((pre_items + 255) / 256), 256, 0, stream>>>(p);
   if (cudaGetLastError() != cudaSuccess) return FA_ERR_LAUNCH;
   fa::fa_bwd_kernel<D, T><<<(unsigned int)ctas, fa::BWD_THREADS, fa::BwdCfg<D>::SMEM_BYTES, stream>>>(
       tq, tk, tv, tdo, tdq, p, status);

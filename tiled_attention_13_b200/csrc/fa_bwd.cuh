@@ -13,7 +13,8 @@
 // Three kernels go out on the stream:
 //   fa_bwd_pre_kernel    D and LSE * log2(e) per query row, into the caller's
 //                        workspace, padded to whole 128-row tiles (padding:
-//                        LSE = +inf, so P = 0 there, and D = 0).
+//                        LSE = +inf, so P = 0 there, and D = 0); it also
+//                        clears the fp32 dQ accumulator.
 //   fa_bwd_kernel        one CTA per (batch, K/V head, 128-key tile), head-major, keeping
 //                        that tile's K and V in shared memory and its dK and
 //                        dV in tensor memory while it walks every query tile
@@ -177,34 +178,47 @@ __host__ __device__ __forceinline__ long long bwd_row(int bsnd, int b, int h, in
   return bsnd ? (((long long)b * N + n) * H + h) * D : (((long long)b * H + h) * N + n) * D;
 }
 
-// One thread per padded query row: D = sum dO o O (fp32), LSE * log2 e.
+// D = sum dO o O (fp32) and LSE * log2 e per padded query row, and the
+// row's fp32 dQ accumulator cleared: D / 8 lanes per row, each reading 16
+// bytes of O and of dO (a row's reads are one contiguous segment per
+// tensor) and clearing 32 bytes of the accumulator; a shuffle reduction
+// within the row's lanes forms D.
 template <int D, typename T>
 __global__ void fa_bwd_pre_kernel(BwdParams p) {
-  const long long idx = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  constexpr int LPR = D / 8;  // lanes per row; divides 32, so a row's lanes share a warp
+  const long long gid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long idx = gid / LPR;  // padded row (b, h, n) in [B, H, nq_pad] order
+  const int part = (int)(gid % LPR);
   const long long rows = (long long)p.B * p.H * p.nq_pad;
-  if (idx >= rows) return;
+  if (idx >= rows) return;  // whole rows leave together
   const int n = (int)(idx % p.nq_pad);
   const long long bh = idx / p.nq_pad;
-  const int h = (int)(bh % p.H), b = (int)(bh / p.H);
   if (n >= p.Nq) {
-    p.lse2[idx] = INFINITY;
-    p.delta[idx] = 0.f;
+    if (part == 0) {
+      p.lse2[idx] = INFINITY;
+      p.delta[idx] = 0.f;
+    }
     return;
   }
-  const long long off = bwd_row(p.bsnd, b, h, n, p.H, p.Nq, D);
-  const uint4* o4 = reinterpret_cast<const uint4*>(static_cast<const T*>(p.o) + off);
-  const uint4* d4 = reinterpret_cast<const uint4*>(static_cast<const T*>(p.dout) + off);
+  const int h = (int)(bh % p.H), b = (int)(bh / p.H);
+  const long long off = bwd_row(p.bsnd, b, h, n, p.H, p.Nq, D) + 8 * part;
+  const uint4 a = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.o) + off);
+  const uint4 g = *reinterpret_cast<const uint4*>(static_cast<const T*>(p.dout) + off);
+  float4* acc_row = reinterpret_cast<float4*>(p.dq_acc + (bh * p.Nq + n) * D + 8 * part);
+  acc_row[0] = make_float4(0.f, 0.f, 0.f, 0.f);
+  acc_row[1] = make_float4(0.f, 0.f, 0.f, 0.f);
+  const T* ae = reinterpret_cast<const T*>(&a);
+  const T* ge = reinterpret_cast<const T*>(&g);
   float acc = 0.f;
-#pragma unroll 4
-  for (int c = 0; c < D / 8; ++c) {
-    const uint4 a = o4[c], g = d4[c];
-    const T* ae = reinterpret_cast<const T*>(&a);
-    const T* ge = reinterpret_cast<const T*>(&g);
 #pragma unroll
-    for (int t = 0; t < 8; ++t) acc = fmaf(bwd_to_f<T>(ae[t]), bwd_to_f<T>(ge[t]), acc);
+  for (int t = 0; t < 8; ++t) acc = fmaf(bwd_to_f<T>(ae[t]), bwd_to_f<T>(ge[t]), acc);
+  const unsigned gmask = (LPR == 32) ? 0xffffffffu : (((1u << LPR) - 1u) << ((threadIdx.x & 31) & ~(LPR - 1)));
+#pragma unroll
+  for (int o = LPR / 2; o > 0; o >>= 1) acc += __shfl_xor_sync(gmask, acc, o);
+  if (part == 0) {
+    p.delta[idx] = acc;
+    p.lse2[idx] = p.lse[bh * p.Nq + n] * 1.4426950408889634f;
   }
-  p.delta[idx] = acc;
-  p.lse2[idx] = p.lse[bh * p.Nq + n] * 1.4426950408889634f;
 }
 
 // dQ = scale * accumulator in q's layout and dtype: one thread per 8 values.

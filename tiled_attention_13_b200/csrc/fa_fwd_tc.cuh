@@ -389,13 +389,22 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
 
   if (warp == WARP_TMA) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
+    // Lane 0 claims the tickets, keeps the unit ring and the barriers, and
+    // issues every Q copy and a contiguous K/V tile's copies.  A paged K/V
+    // tile takes up to TC_BN / 16 sub-boxes, one per cache block: there the
+    // whole warp runs the loop (warp-uniform control flow) and lane u reads
+    // sub-box u's table entry and issues its copies, so that the table reads
+    // overlap and the copies go out in parallel rather than one by one.
+    const unsigned pmask = PAGED ? 0xffffffffu : 1u;  // the lanes that run the loop
+    if (PAGED || lane == 0) {
+      const bool lead = PAGED ? lane == 0 : true;  // a compile-time true for contiguous K/V
       const uint64_t pol_q = l2_policy_evict_first();
       const uint64_t pol_kv = l2_policy_evict_last();
       uint32_t q_phase[2] = {0, 0};
       int st = 0;
       uint32_t kv_phase = 0;
-      // outstanding-load bookkeeping for the drain at exit
+      // outstanding-load bookkeeping for the drain at exit (every lane keeps
+      // the same copy)
       uint32_t k_issued[C::KST], v_issued[C::KST], q_issued[2];
       bool k_pend[C::KST], v_pend[C::KST], q_pend[2];
       for (int s = 0; s < C::KST; ++s) { k_pend[s] = v_pend[s] = false; k_issued[s] = v_issued[s] = 0; }
@@ -405,74 +414,83 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
       uint32_t uphase = 0;
       int n_claimed = 0;
       (void)n_claimed;
+      auto wait_p = [&](uint32_t bb, uint32_t ph) {
+        if constexpr (PAGED)
+          return __all_sync(pmask, mbar_wait(bb, ph, wctx));
+        else
+          return mbar_wait(bb, ph, wctx);
+      };
       // One 128-key K or V tile from a paged cache: TC_BN / pbox sub-boxes of
       // pbox = min(block size, 128) rows, sub-box u from physical block
-      // phys[u].  Blocks past the sequence read at block index num_blocks,
-      // outside the tensor map, which the copy fills with zeros.
+      // phys_u of lane u.  Blocks past the sequence read at block index
+      // num_blocks, outside the tensor map, which the copy fills with zeros.
       constexpr int PSUB = TC_BN / 16;  // sub-boxes per tile at the smallest block size
       const int pbox = PAGED ? (p.block_size < TC_BN ? p.block_size : TC_BN) : TC_BN;
       const int pvalid = PAGED ? (p.Nkv + p.block_size - 1) / p.block_size : 0;
-      int phys[PSUB];
-      // the tile's table entries, read together (independent loads) before
-      // any of its copies is issued, and used for both K and V
+      const bool sub_lane = lane < PSUB && lane * pbox < TC_BN;  // this lane owns sub-box `lane`
+      int phys_u = 0;
+      // the tile's table entry of this lane's sub-box, used for both K and V
       auto paged_lookup = [&](int kv0, int b) {
-#pragma unroll
-        for (int u = 0; u < PSUB; ++u) {
-          const int lb = (kv0 + u * pbox) / p.block_size;
-          phys[u] = (u * pbox < TC_BN && lb < pvalid &&
-                     FA_INDEX_OK(status_word, lb < p.max_blocks && b < p.B))
-                        ? p.block_table[(long long)b * p.max_blocks + lb]
-                                                      : p.num_blocks;
+        int ph = p.num_blocks;
+        if (sub_lane) {
+          const int lb = (kv0 + lane * pbox) / p.block_size;
+          if (lb < pvalid && FA_INDEX_OK(status_word, lb < p.max_blocks && b < p.B))
+            ph = p.block_table[(long long)b * p.max_blocks + lb];
         }
+        phys_u = ph;
       };
       auto paged_load = [&](uint32_t dst, const CUtensorMap* tm, uint32_t b_full, int kv0, int hk, uint64_t pol) {
-#pragma unroll
-        for (int u = 0; u < PSUB; ++u) {
-          if (u * pbox >= TC_BN) break;
-          const int key = kv0 + u * pbox;
-          const int off = key % p.block_size;
+        if (sub_lane) {
+          const int off = (kv0 + lane * pbox) % p.block_size;
           for (int c = 0; c < C::CHUNKS; ++c)
-            tma_load_4d(dst + c * C::CHUNK_BYTES + u * pbox * 128, tm, b_full, c * 64, hk, off, phys[u], pol);
+            tma_load_4d(dst + c * C::CHUNK_BYTES + lane * pbox * 128, tm, b_full, c * 64, hk, off, phys_u, pol);
         }
       };
       while (ok) {
         // claim the next ticket and hand it to the other roles
         // (decoded here once: its integer divisions stay off the other roles)
-        const unsigned int t = atomicAdd(&p.sched->next, 1u);
+        unsigned int t = 0;
+        if (lead) t = atomicAdd(&p.sched->next, 1u);
+        if constexpr (PAGED) t = __shfl_sync(pmask, t, 0);
         const int tk = (t < (unsigned int)p.n_units) ? (int)t : -1;
         int sp = 0;
         const Unit w = decode_unit_t<BAND, SPLIT>(tk < 0 ? 0 : tk, p, sp);
-        if (!mbar_wait(bar(B_UEMPTY + uslot), uphase ^ 1, wctx)) break;
-        ring_put(uslot, tk, w, sp);
-        mbar_arrive(bar(B_UFULL + uslot));
+        if (!wait_p(bar(B_UEMPTY + uslot), uphase ^ 1)) break;
+        if (lead) {
+          ring_put(uslot, tk, w, sp);
+          mbar_arrive(bar(B_UFULL + uslot));
+        }
         if (++uslot == C::UNIT_SLOTS) { uslot = 0; uphase ^= 1; }
         if (tk < 0) break;
-        FA_TRU(true, 0, n_claimed, 0);
+        FA_TRU(lead, 0, n_claimed, 0);
         for (int i = 0; i < 2 && ok; ++i) {
           if (i == 1 && !w.active1) break;
-          if (!mbar_wait(bar(B_QEMPTY + i), q_phase[i] ^ 1, wctx)) { ok = false; break; }
-          const uint32_t dst = sbase + C::OFF_Q + i * C::TILE_BYTES;
-          mbar_arrive_expect_tx(bar(B_QFULL + i), C::TILE_BYTES);
-          const int row0 = (w.qt0 + i) * TC_BM;
-          for (int c = 0; c < C::CHUNKS; ++c) {
-            if (p.bsnd)
-              tma_load_4d(dst + c * C::CHUNK_BYTES, &tm_q, bar(B_QFULL + i), c * 64, w.h, row0, w.b, pol_q);
-            else
-              tma_load_4d(dst + c * C::CHUNK_BYTES, &tm_q, bar(B_QFULL + i), c * 64, row0, w.h, w.b, pol_q);
+          if (!wait_p(bar(B_QEMPTY + i), q_phase[i] ^ 1)) { ok = false; break; }
+          if (lead) {
+            const uint32_t dst = sbase + C::OFF_Q + i * C::TILE_BYTES;
+            mbar_arrive_expect_tx(bar(B_QFULL + i), C::TILE_BYTES);
+            const int row0 = (w.qt0 + i) * TC_BM;
+            for (int c = 0; c < C::CHUNKS; ++c) {
+              if (p.bsnd)
+                tma_load_4d(dst + c * C::CHUNK_BYTES, &tm_q, bar(B_QFULL + i), c * 64, w.h, row0, w.b, pol_q);
+              else
+                tma_load_4d(dst + c * C::CHUNK_BYTES, &tm_q, bar(B_QFULL + i), c * 64, row0, w.h, w.b, pol_q);
+            }
           }
           q_pend[i] = true; q_issued[i] = q_phase[i];
           q_phase[i] ^= 1;
         }
-        FA_TRU(true, 0, n_claimed, 1);
+        FA_TRU(lead, 0, n_claimed, 1);
         const int N = w.n0 > w.s1 + w.n1 ? w.n0 : w.s1 + w.n1;  // KV tiles lo0 .. lo0 + N - 1
         const int hk = w.h / p.kv_group;  // this unit's K/V head
         for (int j = 0; j < N && ok; ++j) {
           const int kv0 = (w.lo0 + j) * TC_BN;
-          if (!mbar_wait(bar(B_KEMPTY + st), kv_phase ^ 1, wctx)) { ok = false; break; }
-          mbar_arrive_expect_tx(bar(B_KFULL + st), C::TILE_BYTES);
+          if constexpr (PAGED) paged_lookup(kv0, w.b);  // before the wait: the read overlaps it
+          if (!wait_p(bar(B_KEMPTY + st), kv_phase ^ 1)) { ok = false; break; }
+          if (lead) mbar_arrive_expect_tx(bar(B_KFULL + st), C::TILE_BYTES);
           const uint32_t kdst = sbase + C::OFF_K + st * C::TILE_BYTES;
           if constexpr (PAGED) {
-            paged_lookup(kv0, w.b);
+            __syncwarp();  // lane 0's expected byte count is set before any lane's copy
             paged_load(kdst, &tm_k, bar(B_KFULL + st), kv0, hk, pol_kv);
           } else {
             for (int c = 0; c < C::CHUNKS; ++c) {
@@ -483,10 +501,11 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             }
           }
           k_pend[st] = true; k_issued[st] = kv_phase;
-          if (!mbar_wait(bar(B_VEMPTY + st), kv_phase ^ 1, wctx)) { ok = false; break; }
-          mbar_arrive_expect_tx(bar(B_VFULL + st), C::TILE_BYTES);
+          if (!wait_p(bar(B_VEMPTY + st), kv_phase ^ 1)) { ok = false; break; }
+          if (lead) mbar_arrive_expect_tx(bar(B_VFULL + st), C::TILE_BYTES);
           const uint32_t vdst = sbase + C::OFF_V + st * C::TILE_BYTES;
           if constexpr (PAGED) {
+            __syncwarp();
             paged_load(vdst, &tm_v, bar(B_VFULL + st), kv0, hk, pol_kv);
           } else {
             for (int c = 0; c < C::CHUNKS; ++c) {
@@ -497,12 +516,12 @@ __global__ void __launch_bounds__(TC_THREADS, 1)
             }
           }
           v_pend[st] = true; v_issued[st] = kv_phase;
-          FA_TRU(j == N - 1, 0, n_claimed, 2);
+          FA_TRU(lead && j == N - 1, 0, n_claimed, 2);
           if (++st == C::KST) { st = 0; kv_phase ^= 1; }
         }
         ++n_claimed;
       }
-      // Every copy this thread started lands before the CTA may exit (their
+      // Every copy this warp started lands before the CTA may exit (their
       // barriers complete on their own; the waits are bounded regardless).
       WaitCtx drain{abort_flag, status_word, p.timeout_ns, 1u};
       volatile int no_abort = 0;

@@ -82,6 +82,32 @@ def test_bwd_fp16(d, causal):
     compare_bwd(Workload("bwd16", B=2, H=2, Nq=260, Nkv=300, d=d, dtype="fp16", layout="BSND", causal=causal, seed=9))
 
 
+def test_bwd_workspace_contents_do_not_matter():
+    """The call clears the fp32 dQ accumulator itself (in its first kernel):
+    a workspace whose bytes are all 0xFF (NaN as fp32) gives the same
+    gradients as a fresh one, dK and dV bit for bit (no atomics) and dQ
+    within the bound of the determinism test below (its fp32 additions
+    come in no fixed order)."""
+    wl = Workload("bwdws", B=1, H=2, Nq=400, Nkv=300, d=128, dtype="bf16", layout="BHND", causal=True, seed=5)
+    q, k, v = (t.cuda() for t in make_qkv(wl))
+    do = _grad_out(wl).cuda()
+    o, lse = fa.forward(q, k, v, causal=True)
+    ref = fa.backward(q, k, v, o, lse, do, causal=True)
+    rc, need = fa.fa_bwd_workspace_size(1, 2, 400, 128)
+    assert rc == 0
+    ws = torch.full((need,), 0xFF, dtype=torch.uint8, device="cuda")
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    args = [q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), do.data_ptr(), lse.data_ptr(), dq.data_ptr(),
+            dk.data_ptr(), dv.data_ptr()]
+    tail = [1, 2, 2, 400, 300, 128, -1.0, 1, fa.FA_LAYOUT_BHND, fa.FA_DTYPE_BF16, None]
+    torch.cuda.synchronize()
+    assert fa.fa_bwd(*args, ws.data_ptr(), need, *tail) == 0
+    torch.cuda.synchronize()
+    assert torch.isfinite(dq.float()).all()
+    assert torch.equal(dk, ref[1]) and torch.equal(dv, ref[2])
+    assert (dq.float() - ref[0].float()).abs().max().item() <= 2.0 ** -6 * ref[0].float().abs().max().item()
+
+
 def test_bwd_deterministic_dk_dv_and_workspace_checks():
     """dK and dV come from one CTA per key tile without atomics: two calls give
     the same bits (dQ is summed with fp32 atomics, so only its value is
